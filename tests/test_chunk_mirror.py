@@ -1,0 +1,56 @@
+"""The chunked factorisation used by the kernels (NumPy fp64 model) equals
+the token-by-token oracle; with bf16-rounded operands it stays inside the
+bf16 tolerance.  CPU only."""
+import numpy as np
+import pytest
+
+import oracle
+from chunk_mirror import chunked_kda
+
+
+def _inputs(rng, T, H, d, g_mode="softplus"):
+    un = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)
+    q = un(rng.standard_normal((T, H, d)))
+    k = un(rng.standard_normal((T, H, d)))
+    v = rng.standard_normal((T, H, d))
+    if g_mode == "floor":
+        g = -5.0 * rng.uniform(0.8, 1.0, (T, H, d))
+    else:
+        g = np.maximum(-5.0, -np.log1p(np.exp(rng.standard_normal((T, H, d)))))
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((T, H))))
+    return q, k, v, g, beta
+
+
+@pytest.mark.parametrize("C", [16, 32, 64])
+@pytest.mark.parametrize("g_mode", ["softplus", "floor"])
+def test_mirror_matches_oracle_fp64(C, g_mode):
+    rng = np.random.default_rng(C)
+    T, H, d = 200, 2, 32          # several chunks and a ragged tail
+    q, k, v, g, beta = _inputs(rng, T, H, d, g_mode)
+    S0 = rng.standard_normal((H, d, d)) * 0.02
+    z = rng.standard_normal((T, H, d))
+    o_ref, S_ref = oracle.kda_fwd_ref(q, k, v, g, beta, S0=S0[None], gate=z)
+    o, S = chunked_kda(q, k, v, g, beta, S0=S0, gate=z, C=C)
+    assert oracle.rel_err(o, o_ref) < 1e-10
+    assert oracle.rel_err(S, S_ref[0]) < 1e-10
+
+
+def test_mirror_below_floor_values_are_clamped():
+    rng = np.random.default_rng(3)
+    q, k, v, g, beta = _inputs(rng, 70, 1, 16)
+    g = g * 3.0  # many values below -5
+    o_ref, S_ref = oracle.kda_fwd_ref(q, k, v, g, beta)
+    o, S = chunked_kda(q, k, v, g, beta, C=64)
+    assert oracle.rel_err(o, o_ref) < 1e-10
+    assert oracle.rel_err(S, S_ref[0]) < 1e-10
+
+
+@pytest.mark.parametrize("g_mode", ["softplus", "floor"])
+def test_mirror_bf16_operands_within_tolerance(g_mode):
+    rng = np.random.default_rng(7)
+    T, H, d = 256, 2, 64
+    q, k, v, g, beta = _inputs(rng, T, H, d, g_mode)
+    o_ref, S_ref = oracle.kda_fwd_ref(q, k, v, g, beta)
+    o, S = chunked_kda(q, k, v, g, beta, C=64, bf16_ops=True)
+    eo, es = oracle.rel_err(o, o_ref), oracle.rel_err(S, S_ref[0])
+    assert eo < 2e-2 and es < 2e-2, (eo, es)
