@@ -26,8 +26,12 @@ The 16-token blocks are where the per-step floor matters: within a block
 every factor is bounded by e^{-16 floor}, inside bf16/fp32 range for floor >= -5.45
 (fupanwang.com Kimi K3 report digest, KDA section, Fig. 3).
 
-``bf16_ops=True`` rounds the tensor-core operands to bf16 where the
-tcgen05 kernel does, to estimate that kernel's error against the oracle.
+``prec`` (a dict operand -> "bf16" | "tf32") rounds the tensor-core
+operands the way a kernel stores them; ``KERNEL_PREC`` is the mixed plan of
+the tcgen05 kernel: tf32 for the operands the output is sensitive to (the
+intra-chunk A operands, A_qk, V_new, K^) and bf16 for the rest.  beta is
+folded into the columns of T (T' = T Diag(beta)) so that U = T' V multiplies
+the exact bf16 input V.
 """
 from __future__ import annotations
 
@@ -41,6 +45,25 @@ def _bf16(x):
     lsb = (u >> 16) & 1
     u = (u + 0x7FFF + lsb) & 0xFFFF0000
     return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def _tf32(x):
+    """Round fp64 -> fp32 -> tf32 (10-bit mantissa, nearest even) -> fp64."""
+    f = np.asarray(x, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 13) & 1
+    u = (u + 0xFFF + lsb) & 0xFFFFE000
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+_ROUND = {"bf16": _bf16, "tf32": _tf32, "fp32": lambda x: np.asarray(x, np.float32).astype(np.float64)}
+
+# operand -> storage precision in the tcgen05 kernel
+KERNEL_PREC = {
+    "Arow": "tf32", "Acol": "tf32",       # q~, k~ and K^(b) for A_qk / A_kk
+    "Aqk": "tf32", "Vn": "tf32", "Khat": "tf32",
+    "T": "bf16", "KG": "bf16", "W": "bf16", "S": "bf16", "QG": "bf16",
+}
 
 
 def _block_inverse(A, sub=16):
@@ -70,7 +93,7 @@ def _block_inverse(A, sub=16):
 
 
 def chunked_kda(q, k, v, g, beta, S0=None, scale=None, gate=None, g_floor=-5.0,
-                C=64, sub=16, bf16_ops=False):
+                C=64, sub=16, prec=None):
     """One sequence, all heads.  q,k,g [T,H,dk]; v [T,H,dv]; beta [T,H];
     S0 [H,dk,dv].  Returns (o [T,H,dv], S_T [H,dk,dv]) in fp64."""
     q, k, v, g, beta = (np.asarray(x, dtype=np.float64) for x in (q, k, v, g, beta))
@@ -78,7 +101,8 @@ def chunked_kda(q, k, v, g, beta, S0=None, scale=None, gate=None, g_floor=-5.0,
     dv = v.shape[2]
     if scale is None:
         scale = 1.0 / np.sqrt(dk)
-    rb = _bf16 if bf16_ops else (lambda x: x)
+    prec = prec or {}
+    rb = lambda name, x: _ROUND[prec[name]](x) if name in prec else x
     o = np.zeros((T, H, dv))
     S_out = np.zeros((H, dk, dv))
     nb = C // sub
@@ -98,29 +122,30 @@ def chunked_kda(q, k, v, g, beta, S0=None, scale=None, gate=None, g_floor=-5.0,
             blk = np.arange(C) // sub
             Gt = np.exp(G - r[blk])
             Kbar = kc * np.exp(r[blk] - G)
-            D = np.exp(r[:, None, :] - r[None, :, :])      # D[b, b'] (use b >= b')
-            Kb = [Kbar * D[b, blk] for b in range(nb + 1)]   # rows j in blocks > b unused
-            Qt = rb(qc * Gt)
-            Kt = rb(kc * Gt)
+            with np.errstate(over="ignore"):
+                D = np.exp(r[:, None, :] - r[None, :, :])      # D[b, b'] (used for b >= b')
+                Kb = [Kbar * D[b, blk] for b in range(nb + 1)]   # rows j in blocks > b unused
+            Qt = rb("Arow", qc * Gt)
+            Kt = rb("Arow", kc * Gt)
             A_qk = np.zeros((C, C)); A_kk = np.zeros((C, C))
             for b in range(nb):
                 rows = slice(b * sub, (b + 1) * sub)
-                colop = rb(Kb[b])
+                # rows j of K^(b) past block b overflow; they only meet masked (j > i) entries
+                with np.errstate(over="ignore", invalid="ignore"):
+                    colop = rb("Acol", np.where(blk <= b, 1.0, 0.0)[:, None] * np.nan_to_num(Kb[b], posinf=0.0))
                 A_qk[rows] = Qt[rows] @ colop.T
                 A_kk[rows] = Kt[rows] @ colop.T
             ii, jj = np.meshgrid(np.arange(C), np.arange(C), indexing="ij")
             A_qk = np.where(jj <= ii, A_qk, 0.0)
             A_kk = np.where(jj < ii, A_kk, 0.0) * bc[:, None]
-            Tm = _block_inverse(A_kk, sub)
+            Tb = rb("T", _block_inverse(A_kk, sub) * bc[None, :])   # T' = T Diag(beta)
             Dq = D[blk, 0]                                   # exp(r_{b(i)}) = Gamma / Gt
-            W = Tm @ rb(bc[:, None] * kc * Gt * Dq) if not bf16_ops else \
-                rb(rb(Tm) @ rb(bc[:, None] * kc * Gt * Dq))
-            U = Tm @ (bc[:, None] * vc) if not bf16_ops else rb(Tm) @ rb(bc[:, None] * vc)
-            Sb = rb(S)
-            Vn = U - W @ Sb
-            Vnb = rb(Vn)
-            O = scale * (rb(qc * Gt * Dq) @ Sb + rb(A_qk) @ Vnb)
-            S = D[nb, 0][:, None] * S + rb(Kb[nb]).T @ Vnb
+            W = rb("W", Tb @ rb("KG", kc * Gt * Dq))
+            U = Tb @ vc
+            Sb = rb("S", S)
+            Vn = rb("Vn", U - W @ Sb)
+            O = scale * (rb("QG", qc * Gt * Dq) @ Sb + rb("Aqk", A_qk) @ Vn)
+            S = D[nb, 0][:, None] * S + rb("Khat", Kb[nb]).T @ Vn
             o[c0:c0 + L, h] = O[:L]
         S_out[h] = S
     if gate is not None:

@@ -5,7 +5,8 @@ import numpy as np
 import pytest
 
 import oracle
-from chunk_mirror import chunked_kda
+from chunk_mirror import KERNEL_PREC, chunked_kda, _bf16
+from parity import TOL_BF16, rel_max, rel_max_beyond_bf16
 
 
 def _inputs(rng, T, H, d, g_mode="softplus"):
@@ -46,11 +47,37 @@ def test_mirror_below_floor_values_are_clamped():
 
 
 @pytest.mark.parametrize("g_mode", ["softplus", "floor"])
-def test_mirror_bf16_operands_within_tolerance(g_mode):
-    rng = np.random.default_rng(7)
-    T, H, d = 256, 2, 64
-    q, k, v, g, beta = _inputs(rng, T, H, d, g_mode)
+def test_mixed_precision_plan_within_tolerance(g_mode):
+    """The kernel's mixed tf32/bf16 operand plan, fed bf16 inputs and storing
+    o in bf16, stays inside the bf16 bound with margin."""
+    rng = np.random.default_rng(11)
+    T, H, d = 512, 2, 128
+    q, k, v, g, beta = (_bf16(x) for x in _inputs(rng, T, H, d, g_mode))
     o_ref, S_ref = oracle.kda_fwd_ref(q, k, v, g, beta)
-    o, S = chunked_kda(q, k, v, g, beta, C=64, bf16_ops=True)
-    eo, es = oracle.rel_err(o, o_ref), oracle.rel_err(S, S_ref[0])
-    assert eo < 2e-2 and es < 2e-2, (eo, es)
+    o, S = chunked_kda(q, k, v, g, beta, C=64, prec=KERNEL_PREC)
+    eo = rel_max_beyond_bf16(_bf16(o), o_ref)
+    es = rel_max(S, S_ref[0])
+    assert eo < 0.6 * TOL_BF16 and es < 0.6 * TOL_BF16, (eo, es)
+
+
+def test_all_bf16_operands_exceed_tolerance():
+    """Documents why the kernel is mixed precision: with every tensor-core
+    operand in bf16 the error leaves the bound."""
+    rng = np.random.default_rng(11)
+    T, H, d = 512, 2, 128
+    q, k, v, g, beta = (_bf16(x) for x in _inputs(rng, T, H, d, "softplus"))
+    o_ref, S_ref = oracle.kda_fwd_ref(q, k, v, g, beta)
+    allbf = {name: "bf16" for name in KERNEL_PREC}
+    o, S = chunked_kda(q, k, v, g, beta, C=64, prec=allbf)
+    assert max(rel_max_beyond_bf16(_bf16(o), o_ref), rel_max(S, S_ref[0])) > TOL_BF16
+
+
+def test_bf16_storage_alone_exceeds_literal_metric():
+    """The exact result rounded once to bf16 already exceeds 2e-2 on the
+    literal max|d|/RMS metric (heavy-tailed o), and scores ~0 beyond the
+    storage half-ulp."""
+    rng = np.random.default_rng(11)
+    q, k, v, g, beta = (_bf16(x) for x in _inputs(rng, 512, 2, 128, "softplus"))
+    o_ref, _ = oracle.kda_fwd_ref(q, k, v, g, beta)
+    assert rel_max(_bf16(o_ref), o_ref) > TOL_BF16
+    assert rel_max_beyond_bf16(_bf16(o_ref), o_ref) < 1e-6
