@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA forward on B200.
+
+Default workload (one "step"): KDA chunked prefill, bf16 I/O, fp32 state,
+B=8 sequences x T=4096 tokens, H=32 heads, dk=dv=128, S0 = 0, final state
+returned -- the configuration the headline metric is quoted on.  The decode
+hot path is measured in the same run (512 sequences x 64 heads, 128x128 fp32
+state per head, bf16 inputs with a sigmoid output gate, 1000 consecutive
+steps) and reported in the ``decode`` object of the same JSON line.
+
+Prints ONE JSON line on rank 0.  ``--impl reference`` times the fp64 CPU
+oracle (the only reference implementation there is) on a bounded sample of
+the same workload.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs the full
+single-GPU workload on its own GPU (independent units, no data-path
+collective: weak scaling); value = all ranks' tokens / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s + TFLOP/s (% BF16 peak); decode steps/s + state HBM GB/s"
+
+# workload (prefill)
+B, T, H, DK, DV = 8, 4096, 32, 128, 128
+CHUNK_ALG = 64
+# workload (decode)
+DEC_B, DEC_H, DEC_STEPS = 512, 64, 1000
+
+
+def flops_per_token_head(dk=DK, dv=DV, C=CHUNK_ALG):
+    """Algorithmic FLOPs per token and head of the chunked forward: the
+    state products (W S, (Q e^G) S, K^T Vn: 6 dk dv), the intra-chunk
+    products (A_qk, A_kk, W, U, A_qk Vn: C (3 dk + 2 dv), causal halves) and
+    the triangular inverse (C^2 / 3)."""
+    return 6 * dk * dv + C * (3 * dk + 2 * dv) + C * C / 3.0
+
+
+def bytes_per_token_head(dk=DK, dv=DV, esz=2):
+    """Minimum HBM bytes per token and head: read q, k, g, v, beta; write o."""
+    return esz * (3 * dk + dv + 1) + esz * dv
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks / throttle reasons in the background."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.windows = []
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "200"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ts, line in self.lines:
+            if not any(a - 0.25 <= ts <= b + 0.25 for a, b in self.windows):
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]),
+                             "util": float(parts[4]) if parts[4] not in ("", "[N/A]") else 100.0,
+                             "reasons": parts[5:10]})
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [r for r in rows if r["util"] >= 50] or rows
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i in range(1, 5)
+                          if r["reasons"][i].lower() == "active"})
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                "sm_max_mhz": max(r["max"] for r in loaded), "reasons": reasons,
+                "samples": len(loaded)}
+
+
+def gpu_uuid(torch, dev):
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
+
+
+def run_oracle_sample(seconds_target: float, seed: int = 0):
+    """Times the fp64 oracle on a bounded slice of the prefill workload: whole
+    4096-token sequences with all heads, as many sequences as fit the time
+    target.  Returns (token_heads, secs, threads, description)."""
+    import oracle
+    from gated_delta_rule_136_b200 import inputs
+    threads = oracle.max_threads()
+    seqs = max(1, math.ceil(threads / H))
+    inp = inputs.prefill_inputs([T] * seqs, H=H, dk=DK, dv=DV, device="cpu", seed=seed)
+    args = [inp[n] for n in ("q", "k", "v", "g", "beta")]
+    t0 = time.perf_counter()
+    oracle.kda_fwd_ref(*args, cu_seqlens=inp["cu_seqlens_host"], nthreads=threads)
+    dt = time.perf_counter() - t0
+    reps = max(1, min(B, int(seconds_target / max(dt, 1e-3))))
+    if reps > 1:
+        seqs = min(B, seqs * reps)
+        inp = inputs.prefill_inputs([T] * seqs, H=H, dk=DK, dv=DV, device="cpu", seed=seed)
+        args = [inp[n] for n in ("q", "k", "v", "g", "beta")]
+        t0 = time.perf_counter()
+        oracle.kda_fwd_ref(*args, cu_seqlens=inp["cu_seqlens_host"], nthreads=threads)
+        dt = time.perf_counter() - t0
+    th = seqs * T * H
+    desc = (f"{seqs} of {B} sequences x {H} heads x {T} tokens (dk=dv={DK}, bf16-valued "
+            f"inputs, fp64 math) of the prefill workload")
+    return th, dt, threads, desc
+
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    from gated_delta_rule_136_b200 import inputs
+    threads = oracle.max_threads()
+    heads, seqs = H, max(1, math.ceil(threads / H))   # at least one unit per host thread
+    inp = inputs.prefill_inputs([T] * seqs, H=heads, dk=DK, dv=DV, device="cpu", seed=0)
+    a = [inp[n] for n in ("q", "k", "v", "g", "beta")]
+    for _ in range(args.warmup):
+        oracle.kda_fwd_ref(*a, cu_seqlens=inp["cu_seqlens_host"], nthreads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.kda_fwd_ref(*a, cu_seqlens=inp["cu_seqlens_host"], nthreads=threads)
+    dt = time.perf_counter() - t0
+    tok_per_s = (seqs * T * heads / H) * args.steps / dt
+    sample = (f"each step: {seqs} of {B} sequences x {heads} heads x {T} tokens of the prefill "
+              f"workload (fp64 oracle, bf16-valued inputs)")
+    line = {"metric": METRIC, "value": tok_per_s, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"KDA prefill B={B} T={T} H={H} dk=dv={DK}", "global_batch": B,
+                       "seq_len": T, "parallelism": "cpu"},
+            "cpu_baseline": {"value": tok_per_s, "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": tok_per_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--chunk", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import torch
+    import torch.distributed as dist
+    from gated_delta_rule_136_b200 import chunk_fwd, decode_step, device_status, inputs
+    from gated_delta_rule_136_b200 import kda as kbind
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks = load_peaks()
+    kbind.load_library()
+    sampler = ClockSampler(gpu_uuid(torch, dev)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+
+    # ---------------- prefill (headline) ----------------
+    inp = inputs.prefill_inputs([T] * B, H=H, dk=DK, dv=DV, device=dev, seed=rank)
+    q, k, v, g, beta = (inp[n] for n in ("q", "k", "v", "g", "beta"))
+    cu, cu_host = inp["cu_seqlens"], inp["cu_seqlens_host"]
+    o = torch.empty_like(v)
+    S_T = torch.empty((B, H, DK, DV), device=dev, dtype=torch.float32)
+    ws = torch.empty(max(256, kbind.workspace_size(B * T, B, H, DK, DV, cu_seqlens_host=cu_host,
+                                                   chunk=args.chunk)), dtype=torch.uint8, device=dev)
+
+    def prefill_step():
+        chunk_fwd(q, k, v, g, beta, cu_seqlens=cu, cu_seqlens_host=cu_host, out=o,
+                  final_state_out=S_T, workspace=ws, chunk=args.chunk)
+
+    for _ in range(args.warmup):
+        prefill_step()
+    barrier()
+    stream = torch.cuda.current_stream(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t_wall0 = time.time()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        prefill_step()
+        ev[i][1].record(stream)
+    end.record(stream)
+    barrier()
+    t_wall1 = time.time()
+    if sampler:
+        sampler.mark(t_wall0, t_wall1)
+    elapsed_ms = max_over_ranks(start.elapsed_time(end))
+    per_call_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    status = device_status(dev)
+    if status != 0:
+        raise RuntimeError(f"device error word after prefill: {status}")
+
+    th = B * T * H
+    tok_per_step = B * T
+    value = world * tok_per_step * args.steps / (elapsed_ms / 1e3)
+    alg_bytes = th * bytes_per_token_head() + B * H * DK * DV * 4   # + S_T write
+    alg_flops = th * flops_per_token_head()
+    achieved_gbs = alg_bytes / (per_call_ms / 1e3) / 1e9
+    tflops = alg_flops / (per_call_ms / 1e3) / 1e12
+
+    # ---------------- e2e through host buffers ----------------
+    e2e = None
+    if not args.no_e2e:
+        host = {n: inp[n].to("cpu").pin_memory() for n in ("q", "k", "v", "g", "beta")}
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        S_host = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
+        dbuf = {n: torch.empty_like(inp[n]) for n in host}
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = o_host.numel() * o_host.element_size() + S_host.numel() * S_host.element_size()
+
+        def e2e_step():
+            for n in host:
+                dbuf[n].copy_(host[n], non_blocking=True)
+            chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], cu_seqlens=cu,
+                      cu_seqlens_host=cu_host, out=o, final_state_out=S_T, workspace=ws,
+                      chunk=args.chunk)
+            o_host.copy_(o, non_blocking=True)
+            S_host.copy_(S_T, non_blocking=True)
+
+        e2e_steps = max(3, min(args.steps, 10))
+        for _ in range(args.warmup):
+            e2e_step()
+        barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tw0 = time.time()
+        s0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        s1.record(stream)
+        barrier()
+        if sampler:
+            sampler.mark(tw0, time.time())
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1))
+        e2e = {"value": world * tok_per_step * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+        del host, dbuf, o_host, S_host
+
+    del inp, q, k, v, g, beta, o
+    torch.cuda.empty_cache()
+
+    # ---------------- decode ----------------
+    decode = None
+    if not args.no_decode:
+        d = inputs.decode_inputs(batch=DEC_B, H=DEC_H, dk=DK, dv=DV, steps=DEC_STEPS, device=dev,
+                                 seed=rank)
+        S = d["S"]
+        od = torch.empty((DEC_STEPS, DEC_B, DEC_H, DV), dtype=torch.bfloat16, device=dev)
+        for t in range(args.warmup):
+            decode_step(d["q"][t], d["k"][t], d["v"][t], d["g"][t], d["beta"][t], S,
+                        gate=d["gate"][t], out=od[t])
+        barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tw0 = time.time()
+        s0.record(stream)
+        for t in range(DEC_STEPS):
+            decode_step(d["q"][t], d["k"][t], d["v"][t], d["g"][t], d["beta"][t], S,
+                        gate=d["gate"][t], out=od[t])
+        s1.record(stream)
+        barrier()
+        if sampler:
+            sampler.mark(tw0, time.time())
+        dec_ms = max_over_ranks(s0.elapsed_time(s1))
+        if device_status(dev) != 0:
+            raise RuntimeError("device error word after decode")
+        units = DEC_B * DEC_H
+        dec_bytes = units * (2 * DK * DV * 4 + 2 * (3 * DK + DV + 1) + 2 * DV + 2 * DV)
+        per_step_s = dec_ms / 1e3 / DEC_STEPS
+        dec_gbs = dec_bytes / per_step_s / 1e9
+        decode = {"workload": f"KDA decode_step batch={DEC_B} H={DEC_H} dk=dv={DK} fp32 state, "
+                              f"bf16 q/k/v/g/beta, sigmoid gate, {DEC_STEPS} consecutive steps",
+                  "steps_per_s": world / per_step_s, "ms_per_step": per_step_s * 1e3,
+                  "state_hbm_gbs": dec_gbs,
+                  "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"],
+                               "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"],
+                               "traffic": None},
+                  "bytes_per_step": dec_bytes, "gpu_launches": DEC_STEPS}
+        del d, S, od
+        torch.cuda.empty_cache()
+
+    if sampler:
+        sampler.stop()
+        clocks = sampler.summary()
+    else:
+        clocks = None
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        th_s, secs, threads, desc = run_oracle_sample(args.cpu_seconds)
+        cpu_baseline = {"value": th_s / H / secs, "unit": "tokens/s", "cores": threads,
+                        "kind": "oracle", "sample": desc + f"; {secs:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"KDA prefill B={B} T={T} H={H} dk=dv={DK} bf16 I/O fp32 state, "
+                                   f"S0=0, final state returned", "global_batch": B * world,
+                       "seq_len": T, "heads": H, "dk": DK, "dv": DV,
+                       "parallelism": f"dp{world} (independent units per rank)",
+                       "l2": "inputs (1.36 GB per step) larger than L2; no flush"},
+            "tflops": tflops, "pct_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
+            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": None,
+                         "kernel": "kda_chunk_fwd (plan + chunk kernel)",
+                         "alg_bytes_per_launch": alg_bytes, "alg_flops_per_launch": alg_flops,
+                         "peak_source": peaks["source"]},
+            "e2e": e2e, "decode": decode, "cpu_baseline": cpu_baseline,
+            "gpu_launches": 2 * args.steps, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,233 @@
+// kda_lib.cu -- the C ABI of include/kda.h: argument validation, planning,
+// kernel dispatch and device status.  All kernels are included here so the
+// library is one translation unit (the device error word needs no
+// relocatable device code).
+#include "kda.h"
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "kda_common.cuh"
+#include "kda_chunk_simt.cuh"
+#include "kda_decode.cuh"
+#include "kda_plan.cuh"
+
+namespace {
+
+using kda::SimtParams;
+using kda::DecodeParams;
+
+constexpr float kMinFloor = -5.45f;   // 16 * floor must stay above ln(FLT_MIN)
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool supported_dim(int32_t d) { return d == 64 || d == 128; }
+
+struct Range {
+    uintptr_t lo, hi;   // [lo, hi)
+};
+
+inline Range range_of(const void *p, int64_t bytes) {
+    uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return Range{a, a + static_cast<uintptr_t>(bytes)};
+}
+
+inline bool overlaps(Range a, Range b) {
+    if (a.lo == a.hi || b.lo == b.hi || a.lo == 0 || b.lo == 0) return false;
+    return a.lo < b.hi && b.lo < a.hi;
+}
+
+// element count a*b*c without int64 overflow; -1 on overflow
+inline int64_t mul3(int64_t a, int64_t b, int64_t c) {
+    if (a < 0 || b < 0 || c < 0) return -1;
+    const int64_t lim = INT64_MAX / 16;
+    if (a && b > lim / a) return -1;
+    int64_t ab = a * b;
+    if (ab && c > lim / ab) return -1;
+    return ab * c;
+}
+
+kda_status validate_fwd_desc(const kda_fwd_desc *d) {
+    if (!d) return KDA_ERR_INVALID_ARG;
+    if (d->num_seqs < 1 || d->num_heads < 1 || d->total_tokens < 0) return KDA_ERR_INVALID_ARG;
+    if (d->dk <= 0 || d->dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (!supported_dim(d->dk) || !supported_dim(d->dv)) return KDA_ERR_UNSUPPORTED;
+    if (d->io_dtype != KDA_BF16 && d->io_dtype != KDA_FP32) return KDA_ERR_INVALID_ARG;
+    if (!std::isfinite(d->scale)) return KDA_ERR_INVALID_ARG;
+    if (!(d->g_floor >= kMinFloor && d->g_floor <= 0.0f)) return KDA_ERR_INVALID_ARG;
+    if (d->chunk != 0 && d->chunk != 16 && d->chunk != 64) return KDA_ERR_INVALID_ARG;
+    if (d->max_seqlen < 0) return KDA_ERR_INVALID_ARG;
+    if (mul3(d->total_tokens, d->num_heads, 128) < 0) return KDA_ERR_INVALID_ARG;
+    if (mul3(d->num_seqs, d->num_heads, (int64_t)d->dk * d->dv) < 0) return KDA_ERR_INVALID_ARG;
+    return KDA_OK;
+}
+
+kda_status validate_host_seqlens(const kda_fwd_desc *d, const int32_t *cu) {
+    if (!cu) return KDA_OK;
+    if (cu[0] != 0) return KDA_ERR_INVALID_ARG;
+    for (int32_t n = 0; n < d->num_seqs; ++n)
+        if (cu[n + 1] < cu[n]) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)cu[d->num_seqs] != d->total_tokens) return KDA_ERR_INVALID_ARG;
+    if (d->max_seqlen > 0) {
+        for (int32_t n = 0; n < d->num_seqs; ++n)
+            if (cu[n + 1] - cu[n] > d->max_seqlen) return KDA_ERR_INVALID_ARG;
+    }
+    return KDA_OK;
+}
+
+// Workspace layout (each region 256-byte aligned):
+//   [0]  int32 seq_order[N]       sequences longest-first
+size_t fwd_workspace_bytes(const kda_fwd_desc *d, const int32_t *) {
+    return align256(sizeof(int32_t) * (size_t)d->num_seqs);
+}
+
+template <int DK, int DV, typename TIO>
+cudaError_t launch_simt(const SimtParams &p, int32_t num_seqs, cudaStream_t stream) {
+    const size_t smem = kda::simt_smem_bytes<DK, DV>();
+    auto kern = kda::chunk_simt_kernel<DK, DV, TIO>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t blocks = (int64_t)num_seqs * p.num_heads;
+    if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
+    kern<<<(unsigned)blocks, 2 * DV, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename TIO>
+cudaError_t dispatch_simt(int dk, int dv, const SimtParams &p, int32_t n, cudaStream_t s) {
+    if (dk == 128 && dv == 128) return launch_simt<128, 128, TIO>(p, n, s);
+    if (dk == 128 && dv == 64) return launch_simt<128, 64, TIO>(p, n, s);
+    if (dk == 64 && dv == 128) return launch_simt<64, 128, TIO>(p, n, s);
+    return launch_simt<64, 64, TIO>(p, n, s);
+}
+
+template <int DK, int DV, typename TIO>
+cudaError_t launch_decode(const DecodeParams &p, int64_t units, cudaStream_t stream) {
+    if (units > INT32_MAX) return cudaErrorInvalidConfiguration;
+    kda::decode_kernel<DK, DV, TIO><<<(unsigned)units, 256, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename TIO>
+cudaError_t dispatch_decode(int dk, int dv, const DecodeParams &p, int64_t u, cudaStream_t s) {
+    if (dk == 128 && dv == 128) return launch_decode<128, 128, TIO>(p, u, s);
+    if (dk == 128 && dv == 64) return launch_decode<128, 64, TIO>(p, u, s);
+    if (dk == 64 && dv == 128) return launch_decode<64, 128, TIO>(p, u, s);
+    return launch_decode<64, 64, TIO>(p, u, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kda_chunk_fwd_workspace_size(const kda_fwd_desc *desc, const int32_t *cu_seqlens_host) {
+    if (validate_fwd_desc(desc) != KDA_OK) return SIZE_MAX;
+    if (validate_host_seqlens(desc, cu_seqlens_host) != KDA_OK) return SIZE_MAX;
+    return fwd_workspace_bytes(desc, cu_seqlens_host);
+}
+
+kda_status kda_chunk_fwd(const kda_fwd_desc *desc, const void *q, const void *k, const void *v,
+                         const void *g, const void *beta, const float *S0,
+                         const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                         const void *gate, void *o, float *S_T, void *workspace,
+                         size_t workspace_bytes, cudaStream_t stream) {
+    kda_status st = validate_fwd_desc(desc);
+    if (st != KDA_OK) return st;
+    st = validate_host_seqlens(desc, cu_seqlens_host);
+    if (st != KDA_OK) return st;
+    const kda_fwd_desc &d = *desc;
+    if (!cu_seqlens) return KDA_ERR_INVALID_ARG;
+    if (d.total_tokens > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
+
+    const size_t esz = d.io_dtype == KDA_BF16 ? 2 : 4;
+    const int64_t T = d.total_tokens, H = d.num_heads;
+    const int64_t nk = T * H * d.dk * (int64_t)esz, nv = T * H * d.dv * (int64_t)esz;
+    const int64_t nb = T * H * (int64_t)esz;
+    const int64_t ns = (int64_t)d.num_seqs * H * d.dk * d.dv * 4;
+    const Range ins[] = {range_of(q, nk), range_of(k, nk), range_of(g, nk), range_of(v, nv),
+                         range_of(beta, nb), range_of(gate, gate ? nv : 0), range_of(S0, S0 ? ns : 0),
+                         range_of(cu_seqlens, 4 * (int64_t)(d.num_seqs + 1))};
+    const Range ro = range_of(o, nv), rs = range_of(S_T, S_T ? ns : 0);
+    for (const Range &r : ins) {
+        if (overlaps(ro, r) || overlaps(rs, r)) return KDA_ERR_INVALID_ARG;
+    }
+    if (overlaps(ro, rs)) return KDA_ERR_INVALID_ARG;
+
+    const size_t need = fwd_workspace_bytes(desc, cu_seqlens_host);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return KDA_ERR_WORKSPACE;
+        const Range rw = range_of(workspace, (int64_t)need);
+        for (const Range &r : ins)
+            if (overlaps(rw, r)) return KDA_ERR_INVALID_ARG;
+        if (overlaps(rw, ro) || overlaps(rw, rs)) return KDA_ERR_INVALID_ARG;
+    }
+
+    int32_t *seq_order = static_cast<int32_t *>(workspace);
+    cudaError_t e = kda::launch_plan_longest_first(cu_seqlens, d.num_seqs, seq_order, stream);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+
+    SimtParams p{q, k, v, g, beta, gate, S0, cu_seqlens, seq_order, o, S_T,
+                 d.num_heads, d.scale, d.g_floor};
+    e = d.io_dtype == KDA_BF16 ? dispatch_simt<__nv_bfloat16>(d.dk, d.dv, p, d.num_seqs, stream)
+                               : dispatch_simt<float>(d.dk, d.dv, p, d.num_seqs, stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_decode_step(const kda_decode_desc *desc, const void *q, const void *k,
+                           const void *v, const void *g, const void *beta, float *S,
+                           const void *gate, void *o, cudaStream_t stream) {
+    if (!desc) return KDA_ERR_INVALID_ARG;
+    const kda_decode_desc &d = *desc;
+    if (d.batch < 1 || d.num_heads < 1 || d.dk <= 0 || d.dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (!supported_dim(d.dk) || !supported_dim(d.dv)) return KDA_ERR_UNSUPPORTED;
+    if (d.io_dtype != KDA_BF16 && d.io_dtype != KDA_FP32) return KDA_ERR_INVALID_ARG;
+    if (!std::isfinite(d.scale)) return KDA_ERR_INVALID_ARG;
+    if (!(d.g_floor >= kMinFloor && d.g_floor <= 0.0f)) return KDA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !g || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(S) % 16 != 0) return KDA_ERR_INVALID_ARG;
+
+    const int64_t units = (int64_t)d.batch * d.num_heads;
+    const size_t esz = d.io_dtype == KDA_BF16 ? 2 : 4;
+    const int64_t nk = units * d.dk * (int64_t)esz, nv = units * d.dv * (int64_t)esz;
+    const Range rS = range_of(S, units * d.dk * d.dv * 4), ro = range_of(o, nv);
+    const Range ins[] = {range_of(q, nk), range_of(k, nk), range_of(g, nk), range_of(v, nv),
+                         range_of(beta, units * (int64_t)esz), range_of(gate, gate ? nv : 0)};
+    for (const Range &r : ins)
+        if (overlaps(rS, r) || overlaps(ro, r)) return KDA_ERR_INVALID_ARG;
+    if (overlaps(rS, ro)) return KDA_ERR_INVALID_ARG;
+
+    DecodeParams p{q, k, v, g, beta, gate, S, o, d.scale, d.g_floor};
+    cudaError_t e = d.io_dtype == KDA_BF16 ? dispatch_decode<__nv_bfloat16>(d.dk, d.dv, p, units, stream)
+                                           : dispatch_decode<float>(d.dk, d.dv, p, units, stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_get_device_status(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, kda::g_err_word, sizeof(word)) != cudaSuccess) return KDA_ERR_CUDA;
+    if (word && cudaMemcpyToSymbol(kda::g_err_word, &zero, sizeof(zero)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (word & kda::ERR_TIMEOUT) return KDA_ERR_TIMEOUT;
+    if (word & kda::ERR_BOUNDS) return KDA_ERR_DEVICE_BOUNDS;
+    return KDA_OK;
+}
+
+const char *kda_status_string(kda_status s) {
+    switch (s) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+    case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+    case KDA_ERR_DEVICE_BOUNDS: return "KDA_ERR_DEVICE_BOUNDS";
+    }
+    return "KDA_UNKNOWN_STATUS";
+}
+
+int32_t kda_version(void) { return 100; }
+
+}  // extern "C"

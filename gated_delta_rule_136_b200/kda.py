@@ -1,0 +1,252 @@
+"""Python binding of the KDA C ABI (``include/kda.h``).
+
+Argument marshalling only: shape/dtype/device checks, output and workspace
+allocation through PyTorch (device memory and streams are PyTorch's job), and
+raw pointers plus the current CUDA stream handed to the library.  Every step
+of the forward runs in the library's CUDA kernels; there is no CPU or PyTorch
+fallback, and a missing library or GPU raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import threading
+
+import torch
+
+from . import build as _build
+
+KDA_OK = 0
+STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
+                3: "KDA_ERR_WORKSPACE", 4: "KDA_ERR_CUDA", 5: "KDA_ERR_TIMEOUT",
+                6: "KDA_ERR_DEVICE_BOUNDS"}
+KDA_BF16, KDA_FP32 = 0, 1
+
+# Every function include/kda.h declares.
+EXPORTED_SYMBOLS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
+                    "kda_get_device_status", "kda_status_string", "kda_version")
+
+
+class KDAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where} failed: {STATUS_NAMES.get(status, status)}")
+
+
+class FwdDesc(ctypes.Structure):
+    _fields_ = [("total_tokens", ctypes.c_int64), ("num_seqs", ctypes.c_int32),
+                ("num_heads", ctypes.c_int32), ("dk", ctypes.c_int32), ("dv", ctypes.c_int32),
+                ("io_dtype", ctypes.c_int), ("scale", ctypes.c_float),
+                ("g_floor", ctypes.c_float), ("chunk", ctypes.c_int32),
+                ("max_seqlen", ctypes.c_int32)]
+
+
+class DecodeDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_heads", ctypes.c_int32),
+                ("dk", ctypes.c_int32), ("dv", ctypes.c_int32), ("io_dtype", ctypes.c_int),
+                ("scale", ctypes.c_float), ("g_floor", ctypes.c_float)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load (building first if missing or stale) the KDA shared library."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = _build.build() if build_if_missing else _build.LIB_PATH
+        lib = ctypes.CDLL(path)
+        vp, sz, i32p = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(ctypes.c_int32)
+        lib.kda_chunk_fwd_workspace_size.argtypes = [ctypes.POINTER(FwdDesc), i32p]
+        lib.kda_chunk_fwd_workspace_size.restype = sz
+        lib.kda_chunk_fwd.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, vp, vp, vp, vp, i32p,
+                                      vp, vp, vp, vp, sz, vp]
+        lib.kda_chunk_fwd.restype = ctypes.c_int
+        lib.kda_decode_step.argtypes = [ctypes.POINTER(DecodeDesc), vp, vp, vp, vp, vp, vp, vp,
+                                        vp, vp]
+        lib.kda_decode_step.restype = ctypes.c_int
+        lib.kda_get_device_status.argtypes = [vp]
+        lib.kda_get_device_status.restype = ctypes.c_int
+        lib.kda_status_string.argtypes = [ctypes.c_int]
+        lib.kda_status_string.restype = ctypes.c_char_p
+        lib.kda_version.restype = ctypes.c_int32
+        _lib = lib
+        return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _io_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_FP32
+    raise TypeError(f"KDA I/O tensors must be bfloat16 or float32, got {t.dtype}")
+
+
+def _check(t, name, shape, dtype, device):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _require_cuda():
+    if not torch.cuda.is_available():
+        raise RuntimeError("the KDA library needs a CUDA GPU (sm_100a); none is available")
+
+
+def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, scale=None, gate=None,
+              g_floor: float = -5.0, chunk: int = 0, cu_seqlens_host=None,
+              output_final_state: bool = True, out=None, final_state_out=None,
+              workspace=None):
+    """KDA chunked prefill.  Returns ``(o, S_T)`` (``S_T`` None if not requested).
+
+    q, k, g [T,H,dk] (or [B,T,H,dk] with ``cu_seqlens`` None); v, gate
+    [T,H,dv]; beta [T,H]; all bf16 or all fp32 on one GPU.  S0 fp32
+    [N,H,dk,dv] or None.  ``cu_seqlens`` int32 [N+1] on the GPU (None for a
+    single sequence or a fixed-length batch); ``cu_seqlens_host`` an optional
+    host copy (list or CPU tensor) used to validate and plan.
+    """
+    _require_cuda()
+    lib = load_library()
+    batched = q.dim() == 4
+    if batched:
+        if cu_seqlens is not None:
+            raise ValueError("cu_seqlens is for packed [T,H,d] inputs")
+        B, Tb = q.shape[:2]
+        q, k, g = (x.reshape(B * Tb, *x.shape[2:]) for x in (q, k, g))
+        out_shape = v.shape
+        v = v.reshape(B * Tb, *v.shape[2:])
+        beta = beta.reshape(B * Tb, -1)
+        if gate is not None:
+            gate = gate.reshape(B * Tb, *gate.shape[2:])
+        cu_host = [i * Tb for i in range(B + 1)]
+        cu_seqlens = torch.tensor(cu_host, dtype=torch.int32, device=q.device)
+        if cu_seqlens_host is None:
+            cu_seqlens_host = cu_host
+    else:
+        out_shape = v.shape
+        if cu_seqlens is None:
+            cu_host = [0, q.shape[0]]
+            cu_seqlens = torch.tensor(cu_host, dtype=torch.int32, device=q.device)
+            if cu_seqlens_host is None:
+                cu_seqlens_host = cu_host
+    device = q.device
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    dtype = q.dtype
+    N = cu_seqlens.numel() - 1
+    _check(q, "q", (T, H, dk), dtype, device)
+    _check(k, "k", (T, H, dk), dtype, device)
+    _check(g, "g", (T, H, dk), dtype, device)
+    _check(v, "v", (T, H, dv), dtype, device)
+    _check(beta, "beta", (T, H), dtype, device)
+    if gate is not None:
+        _check(gate, "gate", (T, H, dv), dtype, device)
+    if S0 is not None:
+        _check(S0, "S0", (N, H, dk, dv), torch.float32, device)
+    _check(cu_seqlens, "cu_seqlens", (N + 1,), torch.int32, device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(dk)
+    host_arr = None
+    if cu_seqlens_host is not None:
+        vals = [int(x) for x in (cu_seqlens_host.tolist() if hasattr(cu_seqlens_host, "tolist")
+                                 else cu_seqlens_host)]
+        if len(vals) != N + 1:
+            raise ValueError("cu_seqlens_host must have N+1 entries")
+        host_arr = (ctypes.c_int32 * (N + 1))(*vals)
+    desc = FwdDesc(T, N, H, dk, dv, _io_dtype(q), float(scale), float(g_floor), int(chunk), 0)
+    ws_bytes = lib.kda_chunk_fwd_workspace_size(ctypes.byref(desc), host_arr)
+    if ws_bytes == ctypes.c_size_t(-1).value:
+        raise KDAError(1, "kda_chunk_fwd_workspace_size")
+    o = out if out is not None else torch.empty((T, H, dv), dtype=dtype, device=device)
+    _check(o, "out", (T, H, dv), dtype, device)
+    S_T = None
+    if output_final_state:
+        S_T = (final_state_out if final_state_out is not None
+               else torch.empty((N, H, dk, dv), dtype=torch.float32, device=device))
+        _check(S_T, "final_state_out", (N, H, dk, dv), torch.float32, device)
+    if ws_bytes > 0 and (workspace is None or workspace.numel() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+    with torch.cuda.device(device):
+        st = lib.kda_chunk_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                               _ptr(S0), ctypes.cast(ctypes.c_void_p(cu_seqlens.data_ptr()),
+                                                     ctypes.POINTER(ctypes.c_int32)),
+                               host_arr, _ptr(gate), _ptr(o), _ptr(S_T),
+                               _ptr(workspace) if ws_bytes > 0 else None, ws_bytes,
+                               _stream_handle(device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_fwd")
+    return o.view(out_shape), S_T
+
+
+def workspace_size(T, N, H, dk, dv, dtype=torch.bfloat16, chunk=0, g_floor=-5.0,
+                   cu_seqlens_host=None) -> int:
+    """Workspace bytes kda_chunk_fwd needs for this problem."""
+    lib = load_library()
+    desc = FwdDesc(T, N, H, dk, dv, KDA_BF16 if dtype == torch.bfloat16 else KDA_FP32,
+                   1.0 / math.sqrt(dk), float(g_floor), int(chunk), 0)
+    host_arr = None
+    if cu_seqlens_host is not None:
+        host_arr = (ctypes.c_int32 * (N + 1))(*[int(x) for x in cu_seqlens_host])
+    return int(lib.kda_chunk_fwd_workspace_size(ctypes.byref(desc), host_arr))
+
+
+def decode_step(q, k, v, g, beta, S, gate=None, scale=None, g_floor: float = -5.0, out=None):
+    """One decode step; updates ``S`` in place and returns ``o``.
+
+    q, k, g [B,H,dk]; v, gate [B,H,dv]; beta [B,H]; S fp32 [B,H,dk,dv].
+    """
+    _require_cuda()
+    lib = load_library()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    device, dtype = q.device, q.dtype
+    _check(q, "q", (B, H, dk), dtype, device)
+    _check(k, "k", (B, H, dk), dtype, device)
+    _check(g, "g", (B, H, dk), dtype, device)
+    _check(v, "v", (B, H, dv), dtype, device)
+    _check(beta, "beta", (B, H), dtype, device)
+    _check(S, "S", (B, H, dk, dv), torch.float32, device)
+    if gate is not None:
+        _check(gate, "gate", (B, H, dv), dtype, device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(dk)
+    o = out if out is not None else torch.empty((B, H, dv), dtype=dtype, device=device)
+    _check(o, "out", (B, H, dv), dtype, device)
+    desc = DecodeDesc(B, H, dk, dv, _io_dtype(q), float(scale), float(g_floor))
+    with torch.cuda.device(device):
+        st = lib.kda_decode_step(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                 _ptr(beta), _ptr(S), _ptr(gate), _ptr(o), _stream_handle(device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_decode_step")
+    return o
+
+
+def device_status(device=None) -> int:
+    """Synchronise the current stream and read/clear the device error word."""
+    _require_cuda()
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return int(lib.kda_get_device_status(_stream_handle(dev)))

@@ -1,0 +1,173 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention forward library.
+ *
+ * Kimi Delta Attention (KDA) keeps, per head, a fixed-size dk x dv fp32
+ * state S that every token rewrites in place:
+ *
+ *     alpha_t = exp(max(g_t, g_floor))                      (per key channel)
+ *     S_t     = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t     = scale * S_t^T q_t           [* sigmoid(z_t) with an output gate]
+ *
+ * Sources (web pages on Kimi K3, cited by title and section):
+ *   - "Kimi-K3 为什么这么强？", §① ②: per-channel diagonal gate Diag(alpha)
+ *     replacing gated DeltaNet's scalar gate; the three-step update (every row
+ *     forgets at its own rate, the current key's row keeps (1 - beta), the new
+ *     value is written as an interpolation).
+ *   - "Kimi K3 深度拆解", 突破一: the transition is diagonal-plus-low-rank.
+ *   - fupanwang.com Kimi K3 report digest, section
+ *     "KDA：百万上下文先要过「数值 算子」这一关": fixed-size recurrent state; a
+ *     lower bound on the per-step log-decay keeps the cumulative decay of a
+ *     16-token block inside BF16 range so the diagonal block runs on dense
+ *     tensor cores (Fig. 3); the output gate is an input-dependent channel
+ *     switch on the recurrence output.  Section "基础设施": chunked prefill
+ *     (intra-chunk parallel, overlapped with cross-chunk state passing) and
+ *     context parallelism by segment states and a prefix scan.
+ *   - "Kimi K3 技术深度解析", §一: the state is a snapshot updated in place
+ *     during decode.
+ *   The pages do not print the floor formula; here it is max(g, g_floor) with
+ *   g_floor a parameter (default -5).
+ *
+ * Conventions for every entry point
+ *   - Pointers marked "device" are CUDA device pointers on the current device;
+ *     the caller allocates and owns every buffer (inputs, outputs, workspace).
+ *     The library never allocates device memory.
+ *   - Calls are asynchronous and ordered on `stream`; nothing is synchronised
+ *     except in kda_get_device_status.  A call returns before its kernels run.
+ *   - Arguments are validated on the host before anything is launched; a bad
+ *     argument returns an error status and launches nothing.  No exception,
+ *     abort or exit crosses the ABI.
+ *   - Layouts are contiguous row-major:
+ *       q, k, g      [T_tot, H, dk]       v, o, gate   [T_tot, H, dv]
+ *       beta         [T_tot, H]           S0, S_T      [N, H, dk, dv] (fp32)
+ *     A fixed-length batch [B, T, H, d] is the same memory with
+ *     cu_seqlens = {0, T, 2T, ..., BT}.
+ *   - io_dtype KDA_BF16: q, k, v, g, beta, gate and o are bf16; the state is
+ *     always fp32.  KDA_FP32: every tensor is fp32.
+ *   - dk and dv must each be 64 or 128.
+ *   - g is the per-step log-decay (natural log) and must be <= 0 (a
+ *     precondition, not checked); values below g_floor act as g_floor.
+ *     g_floor must lie in [-5.45, 0] so that exp(16 * g_floor) and its inverse
+ *     stay normal fp32/bf16 numbers.
+ */
+#ifndef KDA_B200_KDA_H
+#define KDA_B200_KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, overlap, bad cu_seqlens */
+    KDA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. dk = 96)        */
+    KDA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required       */
+    KDA_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed             */
+    KDA_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up               */
+    KDA_ERR_DEVICE_BOUNDS = 6  /* a device-side bounds check fired                 */
+} kda_status;
+
+typedef enum { KDA_BF16 = 0, KDA_FP32 = 1 } kda_dtype;
+
+/* Description of one chunked prefill call. */
+typedef struct {
+    int64_t total_tokens;  /* T_tot: packed tokens over all sequences (>= 0)           */
+    int32_t num_seqs;      /* N >= 1                                                    */
+    int32_t num_heads;     /* H >= 1                                                    */
+    int32_t dk, dv;        /* 64 or 128 each                                            */
+    kda_dtype io_dtype;
+    float scale;           /* read-out scale; pass 1/sqrt(dk) for the usual choice      */
+    float g_floor;         /* lower bound on the log-decay; -5 is the usual choice      */
+    int32_t chunk;         /* 0 = automatic, 16 or 64: a tiling choice, not semantics  */
+    int32_t max_seqlen;    /* longest sequence if known, else 0                         */
+} kda_fwd_desc;
+
+/*
+ * Bytes of device workspace kda_chunk_fwd needs for `desc` (always a multiple
+ * of 256).  `cu_seqlens_host` (N+1 host int32, nullable) lets the library plan
+ * the long-sequence segment split; the same pointer (or the same values) must
+ * then be passed to kda_chunk_fwd.  Returns 0 when no workspace is needed and
+ * SIZE_MAX when the description itself is invalid.
+ */
+size_t kda_chunk_fwd_workspace_size(const kda_fwd_desc *desc,
+                                    const int32_t *cu_seqlens_host);
+
+/*
+ * Chunked prefill over variable-length packed sequences (the FlashKDA role:
+ * intra-chunk work in parallel, the state carried chunk to chunk).
+ *
+ *   q, k, g, v, beta  device, io_dtype, layouts above (read only)
+ *   S0                device fp32 [N,H,dk,dv] initial states, or NULL = zeros
+ *   cu_seqlens        device int32 [N+1], non-decreasing, cu_seqlens[0] = 0,
+ *                     cu_seqlens[N] = total_tokens.  A length-0 sequence
+ *                     returns S_T = S0 for it and writes no output rows.
+ *   cu_seqlens_host   host copy of cu_seqlens or NULL; when given it is
+ *                     validated (monotone, ends at total_tokens) and used to
+ *                     order work longest-first and to split long sequences.
+ *   gate              device io_dtype [T_tot,H,dv] gate logits z, or NULL;
+ *                     when given o = o * sigmoid(z) elementwise.
+ *   o                 device io_dtype [T_tot,H,dv] output (must not overlap
+ *                     any input)
+ *   S_T               device fp32 [N,H,dk,dv] final states, or NULL; must not
+ *                     overlap S0 or any input.
+ *   workspace         device buffer of at least
+ *                     kda_chunk_fwd_workspace_size(desc, cu_seqlens_host)
+ *                     bytes, 256-byte aligned; may be NULL when that size is 0.
+ *
+ * bf16 outputs are rounded to nearest even from fp32.
+ */
+kda_status kda_chunk_fwd(const kda_fwd_desc *desc,
+                         const void *q, const void *k, const void *v,
+                         const void *g, const void *beta, const float *S0,
+                         const int32_t *cu_seqlens,
+                         const int32_t *cu_seqlens_host,
+                         const void *gate, void *o, float *S_T,
+                         void *workspace, size_t workspace_bytes,
+                         cudaStream_t stream);
+
+/* Description of one decode step: `batch` sequences, one token each. */
+typedef struct {
+    int32_t batch;       /* B >= 1 */
+    int32_t num_heads;   /* H >= 1 */
+    int32_t dk, dv;      /* 64 or 128 each */
+    kda_dtype io_dtype;
+    float scale;
+    float g_floor;
+} kda_decode_desc;
+
+/*
+ * One decode step ("snapshot instead of log": the state is rewritten in place).
+ *
+ *   q, k, g   device io_dtype [B,H,dk];  v device io_dtype [B,H,dv]
+ *   beta      device io_dtype [B,H]
+ *   S         device fp32 [B,H,dk,dv], read and overwritten with the new state
+ *   gate      device io_dtype [B,H,dv] gate logits, or NULL
+ *   o         device io_dtype [B,H,dv] output (must not overlap S or inputs)
+ */
+kda_status kda_decode_step(const kda_decode_desc *desc,
+                           const void *q, const void *k, const void *v,
+                           const void *g, const void *beta, float *S,
+                           const void *gate, void *o, cudaStream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears this device's error word,
+ * which kernels set when a bounded wait gives up (KDA_ERR_TIMEOUT) or a
+ * device-side bounds check fires (KDA_ERR_DEVICE_BOUNDS).  The word is shared
+ * by every call on the device.  Returns KDA_ERR_CUDA if the sync fails.
+ */
+kda_status kda_get_device_status(cudaStream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char *kda_status_string(kda_status status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_B200_KDA_H */

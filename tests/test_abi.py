@@ -1,0 +1,139 @@
+"""The C-ABI library builds, loads and exports every symbol include/kda.h
+declares; host-side validation rejects bad arguments before any launch.
+CPU only: every call here fails validation by construction, so nothing is
+ever launched (the fake pointers below are never dereferenced)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_136_b200 import kda
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "include", "kda.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return kda.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_expected_entry_points():
+    assert set(declared_functions()) == set(kda.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version(lib):
+    for code, name in kda.STATUS_NAMES.items():
+        assert lib.kda_status_string(code).decode() == name
+    assert lib.kda_status_string(99).decode() == "KDA_UNKNOWN_STATUS"
+    assert lib.kda_version() >= 100
+
+
+def _desc(**kw):
+    base = dict(total_tokens=64, num_seqs=1, num_heads=2, dk=128, dv=128, io_dtype=kda.KDA_BF16,
+                scale=0.0883883, g_floor=-5.0, chunk=0, max_seqlen=0)
+    base.update(kw)
+    return kda.FwdDesc(**base)
+
+
+SIZE_MAX = ctypes.c_size_t(-1).value
+
+
+@pytest.mark.parametrize("bad", [dict(num_seqs=0), dict(num_heads=0), dict(total_tokens=-1),
+                                 dict(dk=0), dict(io_dtype=7), dict(g_floor=-6.0),
+                                 dict(g_floor=0.5), dict(chunk=32), dict(scale=float("nan")),
+                                 dict(dk=96), dict(dv=256), dict(max_seqlen=-1)])
+def test_workspace_size_rejects_bad_desc(lib, bad):
+    d = _desc(**bad)
+    assert lib.kda_chunk_fwd_workspace_size(ctypes.byref(d), None) == SIZE_MAX
+
+
+def test_workspace_size_valid_and_aligned(lib):
+    d = _desc(num_seqs=3)
+    n = lib.kda_chunk_fwd_workspace_size(ctypes.byref(d), None)
+    assert n % 256 == 0 and n >= 12
+
+
+def test_workspace_size_checks_host_seqlens(lib):
+    d = _desc(num_seqs=2, total_tokens=10)
+    good = (ctypes.c_int32 * 3)(0, 4, 10)
+    assert lib.kda_chunk_fwd_workspace_size(ctypes.byref(d), good) != SIZE_MAX
+    for vals in ((1, 4, 10), (0, 6, 5), (0, 4, 9)):
+        arr = (ctypes.c_int32 * 3)(*vals)
+        assert lib.kda_chunk_fwd_workspace_size(ctypes.byref(d), arr) == SIZE_MAX
+
+
+# Fake, never-dereferenced device addresses: every call below fails validation.
+A = 0x10000000
+MB = 1 << 20
+
+
+def _fwd(lib, desc, q=A, k=A + 4 * MB, v=A + 8 * MB, g=A + 12 * MB, beta=A + 16 * MB, S0=None,
+         cu=A + 20 * MB, cu_host=None, gate=None, o=A + 24 * MB, S_T=None, ws=A + 64 * MB,
+         ws_bytes=1 << 20):
+    cu_p = ctypes.cast(ctypes.c_void_p(cu), ctypes.POINTER(ctypes.c_int32)) if cu else None
+    return lib.kda_chunk_fwd(ctypes.byref(desc), q, k, v, g, beta, S0, cu_p, cu_host, gate, o,
+                             S_T, ws, ws_bytes, None)
+
+
+def test_fwd_rejects_null_required_pointers(lib):
+    d = _desc()
+    for field in ("q", "k", "v", "g", "beta", "o", "cu"):
+        assert _fwd(lib, d, **{field: None}) == 1, field
+
+
+def test_fwd_rejects_overlapping_output(lib):
+    d = _desc()
+    assert _fwd(lib, d, o=A + 1024) == 1                      # o inside q
+    assert _fwd(lib, d, S_T=A + 12 * MB + 64) == 1            # S_T inside g
+    assert _fwd(lib, d, S0=A + 40 * MB, S_T=A + 40 * MB + 4096) == 1   # S_T overlaps S0
+    assert _fwd(lib, d, ws=A + 8 * MB) == 1                   # workspace inside v
+
+
+def test_fwd_rejects_workspace_problems(lib):
+    d = _desc()
+    assert _fwd(lib, d, ws=None) == 3
+    assert _fwd(lib, d, ws_bytes=16) == 3
+    assert _fwd(lib, d, ws=A + 64 * MB + 8) == 3              # not 256-byte aligned
+
+
+def test_fwd_rejects_bad_host_seqlens(lib):
+    d = _desc(num_seqs=2, total_tokens=10)
+    assert _fwd(lib, d, cu_host=(ctypes.c_int32 * 3)(0, 7, 3)) == 1
+    assert _fwd(lib, d, cu_host=(ctypes.c_int32 * 3)(0, 3, 11)) == 1
+
+
+def test_fwd_unsupported_head_dim(lib):
+    assert _fwd(lib, _desc(dk=96)) == 2
+    assert _fwd(lib, _desc(dv=32)) == 2
+
+
+def _dec(lib, desc, q=A, k=A + MB, v=A + 2 * MB, g=A + 3 * MB, beta=A + 4 * MB, S=A + 8 * MB,
+         gate=None, o=A + 40 * MB):
+    return lib.kda_decode_step(ctypes.byref(desc), q, k, v, g, beta, S, gate, o, None)
+
+
+def test_decode_validation(lib):
+    good = dict(batch=4, num_heads=2, dk=128, dv=128, io_dtype=kda.KDA_BF16, scale=0.09,
+                g_floor=-5.0)
+    for bad in (dict(batch=0), dict(num_heads=0), dict(g_floor=-7.0), dict(io_dtype=3)):
+        assert _dec(lib, kda.DecodeDesc(**{**good, **bad})) == 1, bad
+    assert _dec(lib, kda.DecodeDesc(**{**good, "dk": 80})) == 2
+    d = kda.DecodeDesc(**good)
+    for field in ("q", "k", "v", "g", "beta", "S", "o"):
+        assert _dec(lib, d, **{field: None}) == 1, field
+    assert _dec(lib, d, o=A + 8 * MB + 256) == 1      # o inside S
+    assert _dec(lib, d, S=A + 8 * MB + 4) == 1        # S not 16-byte aligned
+    assert _dec(lib, d, gate=A + 8 * MB) == 1         # gate inside S

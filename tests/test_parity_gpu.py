@@ -1,0 +1,188 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded inputs, plus invariants that hold at any size.
+
+Tolerances: bf16 I/O -- S_T max|d|/RMS <= 2e-2; o the same bound beyond its
+own bf16 storage half-ulp (see tests/parity.py).  fp32 I/O -- 1e-4 plain.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_136_b200 import chunk_fwd, decode_step, device_status, inputs
+from parity import TOL_BF16, TOL_FP32, rel_max, rel_max_beyond_bf16
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _cpu(x):
+    return None if x is None else x.detach().to("cpu")
+
+
+def _oracle_prefill(inp, heads=None, seqs=None):
+    """Oracle on a subset of heads / sequences (units are independent)."""
+    q, k, v, g, beta = (_cpu(inp[n]) for n in ("q", "k", "v", "g", "beta"))
+    gate, S0 = _cpu(inp["gate"]), _cpu(inp["S0"])
+    cu = list(inp["cu_seqlens_host"])
+    if heads is not None:
+        sel = lambda t: None if t is None else t[:, heads].contiguous()
+        q, k, v, g, beta, gate = (sel(t) for t in (q, k, v, g, beta, gate))
+        S0 = None if S0 is None else S0[:, heads].contiguous()
+    if seqs is not None:
+        rows = torch.cat([torch.arange(cu[n], cu[n + 1]) for n in seqs])
+        newcu = [0]
+        for n in seqs:
+            newcu.append(newcu[-1] + cu[n + 1] - cu[n])
+        q, k, v, g, beta = (t[rows] for t in (q, k, v, g, beta))
+        gate = None if gate is None else gate[rows]
+        S0 = None if S0 is None else S0[list(seqs)]
+        cu = newcu
+    return oracle.kda_fwd_ref(q, k, v, g, beta, cu_seqlens=np.array(cu, dtype=np.int64), S0=S0,
+                              scale=inp["scale"], gate=gate)
+
+
+def _assert_close(o, S, o_ref, S_ref, dtype, what=""):
+    assert torch.isfinite(o.float()).all(), f"{what}: non-finite o"
+    if S is not None:
+        assert torch.isfinite(S).all(), f"{what}: non-finite S_T"
+    if dtype == torch.float32:
+        eo, es = rel_max(o, o_ref), (rel_max(S, S_ref) if S is not None else 0.0)
+        assert eo <= TOL_FP32 and es <= TOL_FP32, f"{what}: o {eo:.2e} S {es:.2e}"
+    else:
+        eo, es = rel_max_beyond_bf16(o, o_ref), (rel_max(S, S_ref) if S is not None else 0.0)
+        assert eo <= TOL_BF16 and es <= TOL_BF16, f"{what}: o {eo:.2e} S {es:.2e}"
+    return eo, es
+
+
+def test_config0_fp32_chunk16():
+    """fp32, B=1, H=2, T=256, dk=dv=64, chunk 16, S0 = 0: bound 1e-4."""
+    inp = inputs.prefill_inputs([256], H=2, dk=64, dv=64, dtype=torch.float32, device=DEV, seed=0)
+    o, S = chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                     cu_seqlens=inp["cu_seqlens"], cu_seqlens_host=inp["cu_seqlens_host"],
+                     chunk=16)
+    o_ref, S_ref = _oracle_prefill(inp)
+    _assert_close(o, S, o_ref, S_ref, torch.float32, "config 0")
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (64, 128), (128, 64)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("chunk", [0, 16])
+def test_varlen_ragged_gate_s0(dk, dv, dtype, chunk):
+    lengths = [1, 17, 64, 0, 100, 257, 15]
+    inp = inputs.prefill_inputs(lengths, H=3, dk=dk, dv=dv, dtype=dtype, device=DEV, seed=3,
+                                s0_std=0.02, gate=True)
+    o, S = chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S0=inp["S0"],
+                     cu_seqlens=inp["cu_seqlens"], cu_seqlens_host=inp["cu_seqlens_host"],
+                     gate=inp["gate"], chunk=chunk)
+    o_ref, S_ref = _oracle_prefill(inp)
+    _assert_close(o, S, o_ref, S_ref, dtype, f"varlen {dk}x{dv} {dtype} chunk {chunk}")
+    # the empty sequence keeps its initial state exactly
+    assert torch.equal(S[3], inp["S0"][3])
+
+
+def test_floor_stress_bf16():
+    """Decay drawn near the floor (g ~ -5 U(0.8,1)) with some values below it."""
+    inp = inputs.prefill_inputs([300, 77], H=2, dk=128, dv=128, device=DEV, seed=5,
+                                g_mode="floor_stress", s0_std=0.02)
+    inp["g"][:, 0, :7] = -9.0   # below the floor: acts as the floor
+    o, S = chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S0=inp["S0"],
+                     cu_seqlens=inp["cu_seqlens"], cu_seqlens_host=inp["cu_seqlens_host"])
+    o_ref, S_ref = _oracle_prefill(inp)
+    _assert_close(o, S, o_ref, S_ref, torch.bfloat16, "floor stress")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128)])
+def test_decode_against_oracle(dtype, dk, dv):
+    d = inputs.decode_inputs(batch=16, H=4, dk=dk, dv=dv, steps=3, dtype=dtype, device=DEV, seed=7)
+    S = d["S"].clone()
+    S_ref = _cpu(d["S"]).double().numpy()
+    for t in range(3):
+        o = decode_step(d["q"][t], d["k"][t], d["v"][t], d["g"][t], d["beta"][t], S, gate=d["gate"][t])
+        o_ref, S_ref = oracle.kda_decode_ref(_cpu(d["q"][t]), _cpu(d["k"][t]), _cpu(d["v"][t]),
+                                             _cpu(d["g"][t]), _cpu(d["beta"][t]), S_ref,
+                                             gate=_cpu(d["gate"][t]))
+        _assert_close(o, S, o_ref, S_ref, dtype, f"decode step {t}")
+
+
+def test_decode_steps_equal_prefill_fp32():
+    """T decode steps from S0 give the prefill of the same T tokens."""
+    B, H, T, d = 4, 2, 40, 128
+    inp = inputs.prefill_inputs([T] * B, H=H, dk=d, dv=d, dtype=torch.float32, device=DEV,
+                                seed=11, s0_std=0.05, gate=True)
+    o_p, S_p = chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S0=inp["S0"],
+                         cu_seqlens=inp["cu_seqlens"], gate=inp["gate"])
+    S = inp["S0"].clone()
+    resh = lambda x: x.view(B, T, *x.shape[1:])
+    q, k, v, g, beta, z = (resh(inp[n]) for n in ("q", "k", "v", "g", "beta", "gate"))
+    outs = []
+    for t in range(T):
+        outs.append(decode_step(q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(),
+                                g[:, t].contiguous(), beta[:, t].contiguous(), S,
+                                gate=z[:, t].contiguous()))
+    o_d = torch.stack(outs, 1).reshape(B * T, H, d)
+    assert rel_max(o_d, o_p) <= TOL_FP32 and rel_max(S, S_p) <= TOL_FP32
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_split_invariance(dtype):
+    """prefill(T1) then prefill(T2) from its final state == prefill(T1 + T2):
+    the state is the whole checkpoint (the segment decomposition of context
+    parallelism, fupanwang.com digest, section 基础设施)."""
+    T1, T2 = 130, 190
+    inp = inputs.prefill_inputs([T1 + T2], H=2, dk=128, dv=128, dtype=dtype, device=DEV, seed=13,
+                                s0_std=0.02)
+    full_o, full_S = chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S0=inp["S0"])
+    sl = lambda a, b: [inp[n][a:b].contiguous() for n in ("q", "k", "v", "g", "beta")]
+    o1, S1 = chunk_fwd(*sl(0, T1), S0=inp["S0"])
+    o2, S2 = chunk_fwd(*sl(T1, T1 + T2), S0=S1)
+    tol = TOL_FP32 if dtype == torch.float32 else 1e-2
+    assert rel_max(torch.cat([o1, o2]).float(), full_o.float()) <= tol
+    assert rel_max(S2, full_S) <= tol
+
+
+def test_packing_is_bitwise_invariant():
+    """Packed varlen results equal separate runs exactly (units are independent)."""
+    lengths = [33, 200, 5]
+    inp = inputs.prefill_inputs(lengths, H=2, dk=128, dv=128, device=DEV, seed=17, s0_std=0.02,
+                                gate=True)
+    o, S = chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S0=inp["S0"],
+                     cu_seqlens=inp["cu_seqlens"], gate=inp["gate"])
+    cu = inp["cu_seqlens_host"]
+    for n in range(len(lengths)):
+        a, b = cu[n], cu[n + 1]
+        on, Sn = chunk_fwd(*[inp[x][a:b].contiguous() for x in ("q", "k", "v", "g", "beta")],
+                           S0=inp["S0"][n:n + 1].contiguous(), gate=inp["gate"][a:b].contiguous())
+        assert torch.equal(on, o[a:b]) and torch.equal(Sn[0], S[n])
+
+
+def test_linearity_in_v_and_S0_fp32():
+    T, H, d = 150, 2, 64
+    a = inputs.prefill_inputs([T], H=H, dk=d, dv=d, dtype=torch.float32, device=DEV, seed=19,
+                              s0_std=0.1)
+    b = inputs.prefill_inputs([T], H=H, dk=d, dv=d, dtype=torch.float32, device=DEV, seed=23,
+                              s0_std=0.1)
+    base = [a[n] for n in ("q", "k")]
+    run = lambda v, S0: chunk_fwd(base[0], base[1], v, a["g"], a["beta"], S0=S0)
+    o1, S1 = run(a["v"], a["S0"])
+    o2, S2 = run(b["v"], b["S0"])
+    o3, S3 = run(a["v"] + b["v"], a["S0"] + b["S0"])
+    assert rel_max(o3, o1 + o2) <= TOL_FP32 and rel_max(S3, S1 + S2) <= TOL_FP32
+
+
+def test_config1_full_size_sampled_units():
+    """B=8, H=32, T=4096, dk=dv=128, bf16 in the bench's launch; two
+    (sequence, head) units checked in full against the oracle, every output
+    checked finite."""
+    inp = inputs.prefill_inputs([4096] * 8, H=32, dk=128, dv=128, device=DEV, seed=0)
+    o, S = chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                     cu_seqlens=inp["cu_seqlens"], cu_seqlens_host=inp["cu_seqlens_host"])
+    assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
+    for n, h in ((0, 0), (7, 31)):
+        o_ref, S_ref = _oracle_prefill(inp, heads=[h], seqs=[n])
+        a, b = n * 4096, (n + 1) * 4096
+        _assert_close(o[a:b, h:h + 1], S[n:n + 1, h:h + 1], o_ref, S_ref, torch.bfloat16,
+                      f"config 1 unit ({n},{h})")
+    assert device_status() == 0
