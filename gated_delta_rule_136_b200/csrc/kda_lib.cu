@@ -231,3 +231,82 @@ const char *kda_status_string(kda_status s) {
 int32_t kda_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// kda_chunk_fwd_noalloc: the chunked prefill for callers that cannot give the
+// library any device memory of its own -- for instance a host framework whose
+// plugin interface passes only input and output buffers, or a serving runtime
+// that lays out all device memory before it starts and forbids allocations
+// (and the synchronisation they bring) afterwards.  Instead of a caller
+// workspace, the per-call scratch (the longest-first sequence order) lives in
+// a fixed array compiled into the library.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+
+// One slot per sequence; every device that loads the library holds this
+// array (256 KiB) until the process exits.
+static __device__ __align__(256) int32_t g_noalloc_seq_order[KDA_NOALLOC_MAX_SEQS];
+
+constexpr int kMaxDevices = 128;
+std::mutex g_noalloc_mutex;
+int32_t *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device (the host-side symbol is only a stand-in, not a device address).
+cudaError_t noalloc_scratch(int32_t **out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_seq_order);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = static_cast<int32_t *>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" kda_status kda_chunk_fwd_noalloc(const kda_fwd_desc *desc, const void *q,
+                                            const void *k, const void *v, const void *g,
+                                            const void *beta, const float *S0,
+                                            const int32_t *cu_seqlens, const void *gate, void *o,
+                                            float *S_T, cudaStream_t stream) {
+    kda_status st = validate_fwd_desc(desc);
+    if (st != KDA_OK) return st;
+    const kda_fwd_desc &d = *desc;
+    if (d.num_seqs > KDA_NOALLOC_MAX_SEQS) return KDA_ERR_WORKSPACE;
+    if (!cu_seqlens) return KDA_ERR_INVALID_ARG;
+    if (d.total_tokens > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
+
+    const size_t esz = d.io_dtype == KDA_BF16 ? 2 : 4;
+    const int64_t T = d.total_tokens, H = d.num_heads;
+    const int64_t nk = T * H * d.dk * (int64_t)esz, nv = T * H * d.dv * (int64_t)esz;
+    const int64_t nb = T * H * (int64_t)esz;
+    const int64_t ns = (int64_t)d.num_seqs * H * d.dk * d.dv * 4;
+    const Range ins[] = {range_of(q, nk), range_of(k, nk), range_of(g, nk), range_of(v, nv),
+                         range_of(beta, nb), range_of(gate, gate ? nv : 0), range_of(S0, S0 ? ns : 0),
+                         range_of(cu_seqlens, 4 * (int64_t)(d.num_seqs + 1))};
+    const Range ro = range_of(o, nv), rs = range_of(S_T, S_T ? ns : 0);
+    for (const Range &r : ins)
+        if (overlaps(ro, r) || overlaps(rs, r)) return KDA_ERR_INVALID_ARG;
+    if (overlaps(ro, rs)) return KDA_ERR_INVALID_ARG;
+
+    int32_t *seq_order = nullptr;
+    if (noalloc_scratch(&seq_order) != cudaSuccess) return KDA_ERR_CUDA;
+    // every entry [0, num_seqs) is rewritten by the plan kernel before use,
+    // so the previous call's contents never need clearing
+    cudaError_t e = kda::launch_plan_longest_first(cu_seqlens, d.num_seqs, seq_order, stream);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    SimtParams p{q, k, v, g, beta, gate, S0, cu_seqlens, seq_order, o, S_T,
+                 d.num_heads, d.scale, d.g_floor};
+    e = d.io_dtype == KDA_BF16 ? dispatch_simt<__nv_bfloat16>(d.dk, d.dv, p, d.num_seqs, stream)
+                               : dispatch_simt<float>(d.dk, d.dv, p, d.num_seqs, stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}

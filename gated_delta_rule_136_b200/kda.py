@@ -24,7 +24,9 @@ KDA_BF16, KDA_FP32 = 0, 1
 
 # Every function include/kda.h declares.
 EXPORTED_SYMBOLS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
-                    "kda_get_device_status", "kda_status_string", "kda_version")
+                    "kda_get_device_status", "kda_status_string", "kda_version",
+                    "kda_chunk_fwd_noalloc")
+NOALLOC_MAX_SEQS = 65536   # KDA_NOALLOC_MAX_SEQS in include/kda.h
 
 
 class KDAError(RuntimeError):
@@ -250,3 +252,54 @@ def device_status(device=None) -> int:
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     with torch.cuda.device(dev):
         return int(lib.kda_get_device_status(_stream_handle(dev)))
+
+
+def _noalloc_fn(lib):
+    f = lib.kda_chunk_fwd_noalloc
+    if f.restype is not ctypes.c_int:
+        vp = ctypes.c_void_p
+        f.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, vp, vp, vp,
+                      ctypes.POINTER(ctypes.c_int32), vp, vp, vp, vp]
+        f.restype = ctypes.c_int
+    return f
+
+
+def chunk_fwd_noalloc(q, k, v, g, beta, cu_seqlens, S0=None, scale=None, gate=None,
+                      g_floor: float = -5.0, out=None, final_state_out=None):
+    """``kda_chunk_fwd_noalloc``: the chunked prefill for callers that cannot
+    give the library device memory of its own (its per-call scratch is a fixed
+    array inside the library, for up to ``NOALLOC_MAX_SEQS`` sequences).
+
+    Packed inputs only: q, k, g [T,H,dk]; v, gate [T,H,dv]; beta [T,H];
+    ``cu_seqlens`` int32 [N+1] on the GPU.  ``out`` / ``final_state_out`` may
+    be passed to keep this call free of any allocation; when omitted they are
+    allocated here with PyTorch.  Returns ``(o, S_T)``.
+    """
+    _require_cuda()
+    lib = load_library()
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    device, dtype = q.device, q.dtype
+    N = cu_seqlens.numel() - 1
+    for t, name, shape in ((q, "q", (T, H, dk)), (k, "k", (T, H, dk)), (g, "g", (T, H, dk)),
+                           (v, "v", (T, H, dv)), (beta, "beta", (T, H))):
+        _check(t, name, shape, dtype, device)
+    if gate is not None:
+        _check(gate, "gate", (T, H, dv), dtype, device)
+    if S0 is not None:
+        _check(S0, "S0", (N, H, dk, dv), torch.float32, device)
+    _check(cu_seqlens, "cu_seqlens", (N + 1,), torch.int32, device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(dk)
+    o = out if out is not None else torch.empty((T, H, dv), dtype=dtype, device=device)
+    S_T = (final_state_out if final_state_out is not None
+           else torch.empty((N, H, dk, dv), dtype=torch.float32, device=device))
+    desc = FwdDesc(T, N, H, dk, dv, _io_dtype(q), float(scale), float(g_floor), 0, 0)
+    with torch.cuda.device(device):
+        st = _noalloc_fn(lib)(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                              _ptr(S0), ctypes.cast(ctypes.c_void_p(cu_seqlens.data_ptr()),
+                                                    ctypes.POINTER(ctypes.c_int32)),
+                              _ptr(gate), _ptr(o), _ptr(S_T), _stream_handle(device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_fwd_noalloc")
+    return o, S_T

@@ -153,6 +153,37 @@ kda_status kda_decode_step(const kda_decode_desc *desc,
                            const void *gate, void *o, cudaStream_t stream);
 
 /*
+ * kda_chunk_fwd without any caller-provided device memory.  The pages have
+ * no counterpart to this entry point: it exists for callers that cannot hand
+ * the library a workspace, such as a plugin interface that passes only the
+ * input and output buffers, or a runtime that plans all device memory up
+ * front and allows no allocation once it runs.
+ *
+ * Arguments and results are those of kda_chunk_fwd (same kernels, same
+ * numbers), minus cu_seqlens_host and the workspace.  The scratch it needs
+ * (one int32 per sequence) is a fixed array inside the library, sized for
+ * KDA_NOALLOC_MAX_SEQS sequences; every GPU that loads the library keeps
+ * that array (256 KiB) until the process exits.
+ *   - num_seqs > KDA_NOALLOC_MAX_SEQS returns KDA_ERR_WORKSPACE and launches
+ *     nothing.
+ *   - The call allocates no device or host memory.
+ *   - The first call on each device looks up the array's device address
+ *     (with that device current); make that first call before any stream
+ *     capture begins on the device.
+ *   - All calls on a device share the one array and it keeps the last
+ *     call's contents (each call rewrites the part it reads before reading
+ *     it).  Calls whose kernels can overlap on the GPU -- on different
+ *     streams without ordering between them -- race on the array: order them
+ *     on one stream or with events.
+ */
+#define KDA_NOALLOC_MAX_SEQS 65536
+kda_status kda_chunk_fwd_noalloc(const kda_fwd_desc *desc,
+                                 const void *q, const void *k, const void *v,
+                                 const void *g, const void *beta, const float *S0,
+                                 const int32_t *cu_seqlens, const void *gate,
+                                 void *o, float *S_T, cudaStream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears this device's error word,
  * which kernels set when a bounded wait gives up (KDA_ERR_TIMEOUT) or a
  * device-side bounds check fires (KDA_ERR_DEVICE_BOUNDS).  The word is shared
