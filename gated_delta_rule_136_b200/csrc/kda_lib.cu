@@ -8,8 +8,12 @@
 #include <cstdint>
 #include <cstring>
 
+#include <cudaTypedefs.h>
+#include <mutex>
+
 #include "kda_common.cuh"
 #include "kda_chunk_simt.cuh"
+#include "kda_chunk_tc.cuh"
 #include "kda_decode.cuh"
 #include "kda_plan.cuh"
 
@@ -102,6 +106,81 @@ cudaError_t dispatch_simt(int dk, int dv, const SimtParams &p, int32_t n, cudaSt
     return launch_simt<64, 64, TIO>(p, n, s);
 }
 
+// cuTensorMapEncodeTiled through the runtime, so the library needs no link
+// against the driver library.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 2-D view [rows, cols] of a row-major bf16 tensor, 64 x 64 boxes, 128-byte swizzle.
+bool encode_bf16_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The tensor-core prefill covers bf16 I/O with dk = dv = 128 and 16-byte
+// aligned inputs; chunk = 16 and every other shape use the CUDA-core kernel.
+bool tc_path_applies(const kda_fwd_desc &d, const void *q, const void *k, const void *v,
+                     const void *g) {
+    if (d.io_dtype != KDA_BF16 || d.dk != 128 || d.dv != 128 || d.chunk == 16) return false;
+    if (d.total_tokens <= 0 || d.total_tokens > INT32_MAX - 64) return false;
+    for (const void *ptr : {q, k, v, g})
+        if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return false;
+    return true;
+}
+
+cudaError_t launch_tc(const kda_fwd_desc &d, const void *q, const void *k, const void *v,
+                      const void *g, const kda::tck::TcParams &p, cudaStream_t stream) {
+    CUtensorMap tq, tk, tg, tv;
+    const uint64_t rows = (uint64_t)d.total_tokens, cols = (uint64_t)d.num_heads * 128u;
+    if (!encode_bf16_2d(&tq, q, rows, cols) || !encode_bf16_2d(&tk, k, rows, cols) ||
+        !encode_bf16_2d(&tg, g, rows, cols) || !encode_bf16_2d(&tv, v, rows, cols))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(kda::tck::chunk_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kda::tck::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    const int64_t blocks = (int64_t)d.num_seqs * d.num_heads;
+    if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
+    kda::tck::chunk_tc_kernel<<<(unsigned)blocks, kda::tck::NT, kda::tck::SMEM_ALLOC, stream>>>(
+        tq, tk, tg, tv, p);
+    return cudaGetLastError();
+}
+
+// The prefill kernels after planning: the tensor-core kernel where it applies,
+// else the CUDA-core kernel.  Shared by both prefill entry points.
+cudaError_t launch_prefill(const kda_fwd_desc &d, const void *q, const void *k, const void *v,
+                           const void *g, const void *beta, const float *S0,
+                           const int32_t *cu_seqlens, const int32_t *seq_order, const void *gate,
+                           void *o, float *S_T, cudaStream_t stream) {
+    if (tc_path_applies(d, q, k, v, g)) {
+        kda::tck::TcParams tp{beta, gate, S0, cu_seqlens, seq_order, o, S_T, d.num_heads, d.scale,
+                              d.g_floor};
+        return launch_tc(d, q, k, v, g, tp, stream);
+    }
+    SimtParams p{q, k, v, g, beta, gate, S0, cu_seqlens, seq_order, o, S_T,
+                 d.num_heads, d.scale, d.g_floor};
+    return d.io_dtype == KDA_BF16 ? dispatch_simt<__nv_bfloat16>(d.dk, d.dv, p, d.num_seqs, stream)
+                                  : dispatch_simt<float>(d.dk, d.dv, p, d.num_seqs, stream);
+}
+
 template <int DK, int DV, typename TIO>
 cudaError_t launch_decode(const DecodeParams &p, int64_t units, cudaStream_t stream) {
     if (units > INT32_MAX) return cudaErrorInvalidConfiguration;
@@ -168,10 +247,7 @@ kda_status kda_chunk_fwd(const kda_fwd_desc *desc, const void *q, const void *k,
     cudaError_t e = kda::launch_plan_longest_first(cu_seqlens, d.num_seqs, seq_order, stream);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
 
-    SimtParams p{q, k, v, g, beta, gate, S0, cu_seqlens, seq_order, o, S_T,
-                 d.num_heads, d.scale, d.g_floor};
-    e = d.io_dtype == KDA_BF16 ? dispatch_simt<__nv_bfloat16>(d.dk, d.dv, p, d.num_seqs, stream)
-                               : dispatch_simt<float>(d.dk, d.dv, p, d.num_seqs, stream);
+    e = launch_prefill(d, q, k, v, g, beta, S0, cu_seqlens, seq_order, gate, o, S_T, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -304,9 +380,6 @@ extern "C" kda_status kda_chunk_fwd_noalloc(const kda_fwd_desc *desc, const void
     // so the previous call's contents never need clearing
     cudaError_t e = kda::launch_plan_longest_first(cu_seqlens, d.num_seqs, seq_order, stream);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
-    SimtParams p{q, k, v, g, beta, gate, S0, cu_seqlens, seq_order, o, S_T,
-                 d.num_heads, d.scale, d.g_floor};
-    e = d.io_dtype == KDA_BF16 ? dispatch_simt<__nv_bfloat16>(d.dk, d.dv, p, d.num_seqs, stream)
-                               : dispatch_simt<float>(d.dk, d.dv, p, d.num_seqs, stream);
+    e = launch_prefill(d, q, k, v, g, beta, S0, cu_seqlens, seq_order, gate, o, S_T, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

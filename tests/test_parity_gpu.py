@@ -138,9 +138,12 @@ def test_split_invariance(dtype):
     sl = lambda a, b: [inp[n][a:b].contiguous() for n in ("q", "k", "v", "g", "beta")]
     o1, S1 = chunk_fwd(*sl(0, T1), S0=inp["S0"])
     o2, S2 = chunk_fwd(*sl(T1, T1 + T2), S0=S1)
-    tol = TOL_FP32 if dtype == torch.float32 else 1e-2
-    assert rel_max(torch.cat([o1, o2]).float(), full_o.float()) <= tol
-    assert rel_max(S2, full_S) <= tol
+    o_split = torch.cat([o1, o2])
+    if dtype == torch.float32:
+        assert rel_max(o_split, full_o) <= TOL_FP32 and rel_max(S2, full_S) <= TOL_FP32
+    else:   # different chunk boundaries round differently: the bf16 bar applies
+        assert rel_max_beyond_bf16(o_split, full_o) <= TOL_BF16
+        assert rel_max(S2, full_S) <= TOL_BF16
 
 
 def test_packing_is_bitwise_invariant():
