@@ -203,6 +203,7 @@ def reference_arm(args):
 
 
 def main():
+    global B, T, H
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
@@ -213,8 +214,13 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    # smaller workloads for profiling runs only (a reported bench line uses the defaults)
+    ap.add_argument("--batch", type=int, default=B)
+    ap.add_argument("--seqlen", type=int, default=T)
+    ap.add_argument("--heads", type=int, default=H)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    B, T, H = args.batch, args.seqlen, args.heads
     if args.impl == "reference":
         return reference_arm(args)
 

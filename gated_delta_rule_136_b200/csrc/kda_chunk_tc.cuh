@@ -60,8 +60,8 @@ constexpr uint32_t OFF_INTRA = 65536;     // 72 KB, reused after the A MMAs
 constexpr uint32_t OFF_XT = OFF_INTRA;             // X~ [128 rows x 64 ch] tf32 K-major: 2 x 16 KB
 constexpr uint32_t OFF_KB = OFF_INTRA + 32768;     // K^(b), b = 0..3, packed rows 16(b+1): 40 KB
 //   after the A MMAs:
-constexpr uint32_t OFF_SCR = OFF_INTRA;            // A_kk -> T, fp32 [64][65]
-constexpr uint32_t SCR_LD = 65;
+constexpr uint32_t OFF_SCR = OFF_INTRA;            // A_kk -> T, fp32 [64][68]
+constexpr uint32_t SCR_LD = 68;                    // 16-byte aligned rows
 constexpr uint32_t OFF_TP = OFF_INTRA + 17408;     // T' bf16 K-major [64 i x 64 j]: 8 KB
 constexpr uint32_t OFF_AQK = OFF_INTRA + 25600;    // A_qk tf32 K-major [64 i x 64 j]: 16 KB
 constexpr uint32_t OFF_W = OFF_INTRA + 41984;      // W bf16 MN-major [128 c x 64 j]: 16 KB
@@ -81,9 +81,9 @@ static_assert(SMEM_ALLOC <= 232448, "fits in 227 KB");
 // K-block start; rows past the valid ones read neighbouring bytes of this
 // area, which only feed accumulator rows that are never used.
 __host__ __device__ constexpr uint32_t kb_rows(int b) { return 16u * (b + 1); }
-__host__ __device__ constexpr uint32_t kb_base(int b) {
-    return b == 0 ? 0u : kb_base(b - 1) + 2u * kb_rows(b - 1) * 128u;
-}
+// start of tile b: sum over b' < b of 2 K-blocks x 16(b'+1) rows x 128 B
+__host__ __device__ constexpr uint32_t kb_base(int b) { return 2048u * (uint32_t)b * (uint32_t)(b + 1); }
+static_assert(kb_base(1) == 4096u && kb_base(2) == 12288u && kb_base(3) == 24576u, "packing");
 static_assert(kb_base(3) + 128u * 64u + 64u * 128u <= 40960u, "K^(b) reads stay in the area");
 
 // ---- TMEM columns
@@ -112,10 +112,12 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t kbyte) {
     return row * 128u + ((((kbyte >> 4) & 7u) ^ (row & 7u)) << 4) + (kbyte & 15u);
 }
 
+// fp32 -> tf32, round to nearest with ties away from zero, on the integer
+// pipe: adding half a tf32 ulp to the magnitude bits and truncating the low
+// 13 bits gives that rounding for every finite value (a carry into the
+// exponent is the correct round-up).
 __device__ __forceinline__ float to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
+    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 }
 
 __device__ __forceinline__ float bf16_at(const unsigned char *tile, uint32_t row, uint32_t col) {
@@ -141,9 +143,10 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
 // results are used at tf32 / bf16 operand precision or as decay factors).
 __device__ __forceinline__ float fexp(float x) { return __expf(x); }
 
+// two fp32 -> one 32-bit word of bf16 (round to nearest even), lo in the low half
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
-           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
 }
 
 __global__ void __launch_bounds__(NT, 1)
@@ -251,9 +254,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     uint32_t mma_phase = 0, mma_issued = 0;
     bool failed = false;
+    // One thread polls the barrier while the others block in bar.sync (which
+    // costs no issue slots); afterwards every thread observes the completed
+    // phase once, which acquires the TMA / MMA results for it.
     auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
-        bool ok = mbar_wait(bar, parity);
-        return __syncthreads_and(ok) != 0;
+        const bool ok = tid == 0 ? mbar_wait(bar, parity) : true;
+        const bool all = __syncthreads_and(ok) != 0;
+        if (all && tid != 0) (void)mbar_try_wait(bar, parity);
+        return all;
     };
     auto wait_mma = [&]() -> bool {
         bool ok = wait_all(bar_mma, mma_phase & 1);
@@ -451,58 +459,50 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int i = 0; i < 16; ++i) Tb[i * SCR_LD + jj] = t[i];
             }
             __syncthreads();
-            // (2) 16 -> 32: T10 = -T11 (A10 T00) for the block pairs (0,1), (2,3); one element per thread
+            // Off-diagonal blocks by block products, each thread one row i x 4 columns
+            // (16-byte loads of T rows).  C = D E over an n-wide inner range:
+            auto rowx4 = [&](const float *Drow, const float *Ecol4, int n) -> float4 {
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int m = 0; m < 32; ++m) {
+                    if (m < n) {
+                        const float dv = Drow[m];
+                        const float4 e = *reinterpret_cast<const float4 *>(Ecol4 + m * SCR_LD);
+                        acc.x = fmaf(dv, e.x, acc.x); acc.y = fmaf(dv, e.y, acc.y);
+                        acc.z = fmaf(dv, e.z, acc.z); acc.w = fmaf(dv, e.w, acc.w);
+                    }
+                }
+                return acc;
+            };
+            // (2) 16 -> 32 for the pairs (0,1), (2,3): T10 = -T11 (A10 T00)
             {
-                const int o0 = 32 * (tid >> 8), e = tid & 255, i = e >> 4, j2 = e & 15;
-                float x = 0.0f;
-#pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    x = fmaf(scr[(o0 + 16 + i) * SCR_LD + o0 + m], scr[(o0 + m) * SCR_LD + o0 + j2], x);
+                const bool act2 = tid < 128;
+                const int o0 = 32 * (tid >> 6), i = (tid >> 2) & 15, j0 = (tid & 3) * 4;
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (act2) x = rowx4(scr + (o0 + 16 + i) * SCR_LD + o0, scr + o0 * SCR_LD + o0 + j0, 16);
                 __syncthreads();
-                scr[(o0 + 16 + i) * SCR_LD + o0 + j2] = x;
+                if (act2) *reinterpret_cast<float4 *>(scr + (o0 + 16 + i) * SCR_LD + o0 + j0) = x;
                 __syncthreads();
-                float y = 0.0f;
-#pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    if (m <= i) y = fmaf(scr[(o0 + 16 + i) * SCR_LD + o0 + 16 + m], scr[(o0 + 16 + m) * SCR_LD + o0 + j2], y);
+                if (act2) x = rowx4(scr + (o0 + 16 + i) * SCR_LD + o0 + 16, scr + (o0 + 16) * SCR_LD + o0 + j0, 16);
                 __syncthreads();
-                scr[(o0 + 16 + i) * SCR_LD + o0 + j2] = -y;
+                if (act2)
+                    *reinterpret_cast<float4 *>(scr + (o0 + 16 + i) * SCR_LD + o0 + j0) =
+                        make_float4(-x.x, -x.y, -x.z, -x.w);
                 __syncthreads();
             }
-            // (3) 32 -> 64: T[32:, :32] = -T[32:, 32:] (A[32:, :32] T[:32, :32]); two elements per thread
+            // (3) 32 -> 64: T[32:, :32] = -T[32:, 32:] (A[32:, :32] T[:32, :32])
             {
-                float x[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int idx = tid * 2 + u, i = idx >> 5, j2 = idx & 31;
-                    float acc = 0.0f;
-#pragma unroll
-                    for (int m = 0; m < 32; ++m)
-                        acc = fmaf(scr[(32 + i) * SCR_LD + m], scr[m * SCR_LD + j2], acc);
-                    x[u] = acc;
-                }
+                const bool act3 = tid < 256;
+                const int i = tid >> 3, j0 = (tid & 7) * 4;
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (act3) x = rowx4(scr + (32 + i) * SCR_LD, scr + j0, 32);
                 __syncthreads();
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int idx = tid * 2 + u, i = idx >> 5, j2 = idx & 31;
-                    scr[(32 + i) * SCR_LD + j2] = x[u];
-                }
+                if (act3) *reinterpret_cast<float4 *>(scr + (32 + i) * SCR_LD + j0) = x;
                 __syncthreads();
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int idx = tid * 2 + u, i = idx >> 5, j2 = idx & 31;
-                    float acc = 0.0f;
-#pragma unroll
-                    for (int m = 0; m < 32; ++m)
-                        if (m <= i) acc = fmaf(scr[(32 + i) * SCR_LD + 32 + m], scr[(32 + m) * SCR_LD + j2], acc);
-                    x[u] = -acc;
-                }
+                if (act3) x = rowx4(scr + (32 + i) * SCR_LD + 32, scr + 32 * SCR_LD + j0, 32);
                 __syncthreads();
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int idx = tid * 2 + u, i = idx >> 5, j2 = idx & 31;
-                    scr[(32 + i) * SCR_LD + j2] = x[u];
-                }
+                if (act3)
+                    *reinterpret_cast<float4 *>(scr + (32 + i) * SCR_LD + j0) = make_float4(-x.x, -x.y, -x.z, -x.w);
                 __syncthreads();
             }
             // (4) T' = T Diag(beta) as bf16, K-major [i x j], zero above the diagonal; 8 per thread
