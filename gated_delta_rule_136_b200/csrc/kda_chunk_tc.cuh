@@ -63,16 +63,21 @@ constexpr uint32_t OFF_KB = OFF_INTRA + 32768;     // K^(b), b = 0..3, packed ro
 constexpr uint32_t OFF_SCR = OFF_INTRA;            // A_kk -> T, fp32 [64][68]
 constexpr uint32_t SCR_LD = 68;                    // 16-byte aligned rows
 constexpr uint32_t OFF_TP = OFF_INTRA + 17408;     // T' bf16 K-major [64 i x 64 j]: 8 KB
-constexpr uint32_t OFF_AQK = OFF_INTRA + 25600;    // A_qk tf32 K-major [64 i x 64 j]: 16 KB
 constexpr uint32_t OFF_W = OFF_INTRA + 41984;      // W bf16 MN-major [128 c x 64 j]: 16 KB
 constexpr uint32_t OFF_QG = OFF_INTRA + 73728;     // Q e^G bf16 MN-major [128 c x 64 i]: 16 KB
 constexpr uint32_t OFF_KG = OFF_QG + 16384;        // K e^G bf16 K-major [128 c x 64 j]: 16 KB
-constexpr uint32_t OFF_KHT = OFF_KG + 16384;       // K^(4)^T tf32 K-major [128 c x 64 j]: 32 KB
-constexpr uint32_t OFF_SMALL = OFF_KHT + 32768;    // beta[64], gamma[128], barriers, tmem base
+// B operand of the second state MMA: rows 0-63 = A_qk [i x j], rows 64-191 =
+// K^(4)^T [c x j]; tf32 K-major with two 128-byte K-blocks of 192 rows each
+constexpr uint32_t OFF_AK = OFF_KG + 16384;
+constexpr uint32_t AK_KBLK = 192u * 128u;          // 24 KB per K-block
+constexpr uint32_t OFF_AQK = OFF_AK;               // + kb * AK_KBLK + row * 128
+constexpr uint32_t OFF_KHT = OFF_AK + 64u * 128u;  // + kb * AK_KBLK + row * 128
+constexpr uint32_t OFF_SMALL = OFF_AK + 2u * AK_KBLK;  // beta[64], gamma[128], barriers, tmem base
 constexpr uint32_t OFF_TOT = OFF_SMALL + 1024;     // per-row-group decay totals [8][64] fp32
 constexpr uint32_t SMEM_BYTES = OFF_TOT + 2048;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024; // slack for aligning the base
 static_assert(OFF_W + 16384 <= OFF_INTRA + 73728, "post-MMA tiles fit the intra region");
+static_assert(OFF_QG - OFF_W < (1u << 18) && (OFF_QG - OFF_W) % 16 == 0, "W | Q e^G as one MN-major operand");
 static_assert(OFF_KB + 40960 <= OFF_INTRA + 73728, "intra tiles fit");
 static_assert(SMEM_ALLOC <= 232448, "fits in 227 KB");
 
@@ -87,13 +92,14 @@ static_assert(kb_base(1) == 4096u && kb_base(2) == 12288u && kb_base(3) == 24576
 static_assert(kb_base(3) + 128u * 64u + 64u * 128u <= 40960u, "K^(b) reads stay in the area");
 
 // ---- TMEM columns
-constexpr uint32_t T_DB = 0;      // A MMAs: 4 x 32 columns (M = 64 layout); later dS^T (128)
+constexpr uint32_t T_DB = 0;      // A MMAs: 4 x 32 columns (M = 64 layout)
+constexpr uint32_t T_O2 = 0;      // (A_qk Vn)^T   [v x i]   } one MMA (N = 192), after the
+constexpr uint32_t T_DS = 64;     // dS^T          [v x c]   } A readout and the Vn step
 constexpr uint32_t T_U = 128;     // U^T     [v x i]
 constexpr uint32_t T_W = 192;     // W^T     [c x i]
-constexpr uint32_t T_P = 256;     // P^T = (W S)^T, then Vn^T (tf32 A operand)
-constexpr uint32_t T_O1 = 320;    // ((Q e^G) S)^T
+constexpr uint32_t T_P = 256;     // P^T = (W S)^T, then Vn^T (tf32 A operand)  } one MMA
+constexpr uint32_t T_O1 = 320;    // ((Q e^G) S)^T                              } (N = 128)
 constexpr uint32_t T_S = 384;     // S^T bf16 A operand (2 per column)
-constexpr uint32_t T_O2 = 448;    // (A_qk Vn)^T
 constexpr uint32_t TMEM_COLS = 512;
 
 struct TcParams {
@@ -124,6 +130,17 @@ __device__ __forceinline__ float bf16_at(const unsigned char *tile, uint32_t row
     // element (row, col) of a [64 x 64] bf16 TMA tile (128-byte swizzle)
     const __nv_bfloat16 *p = reinterpret_cast<const __nv_bfloat16 *>(tile + sw128(row, col * 2));
     return __bfloat162float(*p);
+}
+
+// D[16x8] += A[16x8] B[8x8] on the warp-level tensor-core path (tf32 inputs,
+// fp32 accumulation); fragments: g = lane / 4, t = lane % 4,
+//   a = {A[g][t], A[g+8][t], A[g][t+4], A[g+8][t+4]},  b = {B[t][g], B[t+4][g]},
+//   d = {D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1]}.
+__device__ __forceinline__ void mma_16x8x8_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+                 "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
@@ -254,6 +271,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     uint32_t mma_phase = 0, mma_issued = 0;
     bool failed = false;
+    // beta of the next chunk, loaded one chunk ahead (64 strided values)
+    auto load_beta = [&](int ci) -> float {
+        const int64_t tb = t_begin + (int64_t)ci * C + tid;
+        return (tid < C && ci < nchunks && tb < t_end) ? __bfloat162float(beta[tb * H + hh]) : 0.0f;
+    };
+    float beta_next = load_beta(0);
     // One thread polls the barrier while the others block in bar.sync (which
     // costs no issue slots); afterwards every thread observes the completed
     // phase once, which acquires the TMA / MMA results for it.
@@ -280,12 +303,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t id_a = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 64, 32);
     const uint32_t id_w = instr_desc(FMT_BF16, K_MAJOR, K_MAJOR, 128, 64);
     const uint32_t id_u = instr_desc(FMT_BF16, MN_MAJOR, K_MAJOR, 128, 64);
-    const uint32_t id_1 = instr_desc(FMT_BF16, K_MAJOR, MN_MAJOR, 128, 64);
-    const uint32_t id_o = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 128, 64);
-    const uint32_t id_s = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 128, 128);
+    const uint32_t id_1 = instr_desc(FMT_BF16, K_MAJOR, MN_MAJOR, 128, 128);
+    const uint32_t id_2 = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 128, 192);
     const uint64_t d_k16 = smem_desc_sw128(smb, 16, 1024);          // K-major template
     const uint64_t d_mnv = smem_desc_sw128(smb, 8192, 1024);        // v: MN blocks 8 KB apart
-    const uint64_t d_mnc = smem_desc_sw128(smb, 16384, 1024);       // [128 c x 64] MN-major
+    const uint64_t d_wq = smem_desc_sw128(smb, OFF_QG - OFF_W, 1024);  // [W | Q e^G] MN-major
     auto at = [](uint64_t tmpl, uint32_t byte_off) -> uint64_t {     // same descriptor, moved start
         return tmpl + (uint64_t)(byte_off >> 4);
     };
@@ -300,13 +322,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t ld_par = (uint32_t)(ci & 1);
 
         // ================================================= prep + A MMAs, 2 passes of 64 key channels
+        bool loads_ok = true;
         for (int pass = 0; pass < 2 && !failed; ++pass) {
-            if (!wait_all(&bar_qkg[pass], ld_par)) { failed = true; break; }
+            // every thread observes the TMA barrier itself (no block barrier here, so
+            // this pass's first part overlaps the previous pass's MMA issue); a
+            // timeout is folded into the next block-wide barrier
+            loads_ok = mbar_wait(&bar_qkg[pass], ld_par) && loads_ok;
             ++qkg_done[pass];
             const unsigned char *raw = sm + (pass ? OFF_QKG1 : OFF_QKG0);
             const int c = pass * 64 + cl;
-            if (pass == 0 && tid < C)
-                s_beta[tid] = tid < L ? __bfloat162float(beta[(t0 + tid) * H + hh]) : 0.0f;
+            if (pass == 0) {
+                if (tid < C) s_beta[tid] = beta_next;
+                beta_next = load_beta(ci + 1);
+            }
             // local inclusive cumulative decay over this thread's 8 rows
             float G[8];
             {
@@ -327,8 +355,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 qv[r] = bf16_at(raw + QKG_Q, rg * 8 + r, cl);
                 kv[r] = bf16_at(raw + QKG_K, rg * 8 + r, cl);
             }
-            if (pass == 1 && !wait_mma()) { failed = true; break; }   // pass-0 A MMAs done (also syncs s_tot)
-            if (pass == 0) __syncthreads();
+            if (pass == 1) {                       // pass-0 A MMAs done (also syncs s_tot)
+                const bool ok = tid == 0 ? mbar_wait(bar_mma, mma_phase & 1) : true;
+                const bool all = __syncthreads_and(ok && loads_ok) != 0;
+                if (all && tid != 0) (void)mbar_try_wait(bar_mma, mma_phase & 1);
+                ++mma_phase;
+                tc_fence_after();
+                if (!all) { failed = true; break; }
+            } else if (!__syncthreads_and(loads_ok)) {
+                failed = true;
+                break;
+            }
             // prefix over row groups: P[k] = sum of the first k group totals
             float P[9];
             P[0] = 0.0f;
@@ -382,7 +419,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // K^(4)^T (K-major [c x j], tf32): 8 tokens = 32 bytes
             {
                 const uint32_t jb = (uint32_t)rg * 32u;
-                unsigned char *dst = sm + OFF_KHT + (jb >> 7) * 16384u;
+                unsigned char *dst = sm + OFF_KHT + (jb >> 7) * AK_KBLK;
                 *reinterpret_cast<float4 *>(dst + sw128(c, jb & 127u)) =
                     make_float4(to_tf32(kh[0]), to_tf32(kh[1]), to_tf32(kh[2]), to_tf32(kh[3]));
                 *reinterpret_cast<float4 *>(dst + sw128(c, (jb & 127u) + 16u)) =
@@ -419,7 +456,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (lane < 16) {
                 const int j = lq * 16 + lane;
                 const uint32_t kbj = (uint32_t)j * 4u;
-                unsigned char *aqk = sm + OFF_AQK + (kbj >> 7) * 8192u;
+                unsigned char *aqk = sm + OFF_AQK + (kbj >> 7) * AK_KBLK;
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int i = 16 * cq + e;
@@ -459,50 +496,53 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int i = 0; i < 16; ++i) Tb[i * SCR_LD + jj] = t[i];
             }
             __syncthreads();
-            // Off-diagonal blocks by block products, each thread one row i x 4 columns
-            // (16-byte loads of T rows).  C = D E over an n-wide inner range:
-            auto rowx4 = [&](const float *Drow, const float *Ecol4, int n) -> float4 {
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int m = 0; m < 32; ++m) {
-                    if (m < n) {
-                        const float dv = Drow[m];
-                        const float4 e = *reinterpret_cast<const float4 *>(Ecol4 + m * SCR_LD);
-                        acc.x = fmaf(dv, e.x, acc.x); acc.y = fmaf(dv, e.y, acc.y);
-                        acc.z = fmaf(dv, e.z, acc.z); acc.w = fmaf(dv, e.w, acc.w);
-                    }
+            // Off-diagonal blocks by block products on the warp-level tensor cores
+            // (tf32; T' only needs bf16 precision).  tile(...) returns one 16x8
+            // tile of D[dr0.., dc0..] E[er0.., ec0..] over a K-wide inner range.
+            const int gq = lane >> 2, tq = lane & 3;
+            auto tile = [&](int dr0, int dc0, int er0, int ec0, int K, float (&acc)[4]) {
+                acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
+                for (int k0 = 0; k0 < K; k0 += 8) {
+                    uint32_t a[4], b[2];
+                    a[0] = __float_as_uint(scr[(dr0 + gq) * SCR_LD + dc0 + k0 + tq]);
+                    a[1] = __float_as_uint(scr[(dr0 + gq + 8) * SCR_LD + dc0 + k0 + tq]);
+                    a[2] = __float_as_uint(scr[(dr0 + gq) * SCR_LD + dc0 + k0 + tq + 4]);
+                    a[3] = __float_as_uint(scr[(dr0 + gq + 8) * SCR_LD + dc0 + k0 + tq + 4]);
+                    b[0] = __float_as_uint(scr[(er0 + k0 + tq) * SCR_LD + ec0 + gq]);
+                    b[1] = __float_as_uint(scr[(er0 + k0 + tq + 4) * SCR_LD + ec0 + gq]);
+                    mma_16x8x8_tf32(acc, a, b);
                 }
-                return acc;
             };
-            // (2) 16 -> 32 for the pairs (0,1), (2,3): T10 = -T11 (A10 T00)
+            auto put = [&](int r0, int c0, const float (&acc)[4], float sign) {
+                scr[(r0 + gq) * SCR_LD + c0 + 2 * tq] = sign * acc[0];
+                scr[(r0 + gq) * SCR_LD + c0 + 2 * tq + 1] = sign * acc[1];
+                scr[(r0 + gq + 8) * SCR_LD + c0 + 2 * tq] = sign * acc[2];
+                scr[(r0 + gq + 8) * SCR_LD + c0 + 2 * tq + 1] = sign * acc[3];
+            };
+            // (2) 16 -> 32 for the pairs (0,1), (2,3): T10 = -T11 (A10 T00); warps 0-3
             {
-                const bool act2 = tid < 128;
-                const int o0 = 32 * (tid >> 6), i = (tid >> 2) & 15, j0 = (tid & 3) * 4;
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (act2) x = rowx4(scr + (o0 + 16 + i) * SCR_LD + o0, scr + o0 * SCR_LD + o0 + j0, 16);
+                const int o0 = 32 * (warp >> 1), n0 = o0 + 8 * (warp & 1);
+                float acc[4];
+                if (warp < 4) tile(o0 + 16, o0, o0, n0, 16, acc);
                 __syncthreads();
-                if (act2) *reinterpret_cast<float4 *>(scr + (o0 + 16 + i) * SCR_LD + o0 + j0) = x;
+                if (warp < 4) put(o0 + 16, n0, acc, 1.0f);
                 __syncthreads();
-                if (act2) x = rowx4(scr + (o0 + 16 + i) * SCR_LD + o0 + 16, scr + (o0 + 16) * SCR_LD + o0 + j0, 16);
+                if (warp < 4) tile(o0 + 16, o0 + 16, o0 + 16, n0, 16, acc);
                 __syncthreads();
-                if (act2)
-                    *reinterpret_cast<float4 *>(scr + (o0 + 16 + i) * SCR_LD + o0 + j0) =
-                        make_float4(-x.x, -x.y, -x.z, -x.w);
+                if (warp < 4) put(o0 + 16, n0, acc, -1.0f);
                 __syncthreads();
             }
-            // (3) 32 -> 64: T[32:, :32] = -T[32:, 32:] (A[32:, :32] T[:32, :32])
+            // (3) 32 -> 64: T[32:, :32] = -T[32:, 32:] (A[32:, :32] T[:32, :32]); warps 0-7
             {
-                const bool act3 = tid < 256;
-                const int i = tid >> 3, j0 = (tid & 7) * 4;
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (act3) x = rowx4(scr + (32 + i) * SCR_LD, scr + j0, 32);
+                const int r0 = 32 + 16 * (warp >> 2), n0 = 8 * (warp & 3);
+                float acc[4];
+                if (warp < 8) tile(r0, 0, 0, n0, 32, acc);
                 __syncthreads();
-                if (act3) *reinterpret_cast<float4 *>(scr + (32 + i) * SCR_LD + j0) = x;
+                if (warp < 8) put(r0, n0, acc, 1.0f);
                 __syncthreads();
-                if (act3) x = rowx4(scr + (32 + i) * SCR_LD + 32, scr + 32 * SCR_LD + j0, 32);
+                if (warp < 8) tile(r0, 32, 32, n0, 32, acc);
                 __syncthreads();
-                if (act3)
-                    *reinterpret_cast<float4 *>(scr + (32 + i) * SCR_LD + j0) = make_float4(-x.x, -x.y, -x.z, -x.w);
+                if (warp < 8) put(r0, n0, acc, -1.0f);
                 __syncthreads();
             }
             // (4) T' = T Diag(beta) as bf16, K-major [i x j], zero above the diagonal; 8 per thread
@@ -557,11 +597,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ++mma_issued;
         if (tid == 0) {
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {          // K = 128 key channels in steps of 16
-                const uint32_t a_t = tbase + T_S + 8u * s;
-                mma_bf16_ts(tbase + T_P, a_t, at(d_mnc, OFF_W + 2048u * s), id_1, s > 0);
-                mma_bf16_ts(tbase + T_O1, a_t, at(d_mnc, OFF_QG + 2048u * s), id_1, s > 0);
-            }
+            for (int s = 0; s < 8; ++s)            // K = 128 key channels in steps of 16
+                mma_bf16_ts(tbase + T_P, tbase + T_S + 8u * s, at(d_wq, OFF_W + 2048u * s), id_1, s > 0);
             mma_commit(bar_mma);
         }
         if (!wait_mma()) { failed = true; break; }
@@ -588,9 +625,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
             for (int s = 0; s < 8; ++s) {          // K = 64 tokens in steps of 8
                 const uint32_t kb = (uint32_t)(s >> 2), koff = (uint32_t)(s & 3) * 32u;
-                const uint32_t a_t = tbase + T_P + 8u * s;
-                mma_tf32_ts(tbase + T_O2, a_t, at(d_k16, OFF_AQK + kb * 8192u + koff), id_o, s > 0);
-                mma_tf32_ts(tbase + T_DB, a_t, at(d_k16, OFF_KHT + kb * 16384u + koff), id_s, s > 0);
+                mma_tf32_ts(tbase + T_O2, tbase + T_P + 8u * s, at(d_k16, OFF_AK + kb * AK_KBLK + koff), id_2, s > 0);
             }
             mma_commit(bar_mma);
         }
@@ -598,18 +633,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
         // ================================================= state update and outputs
         {
-            uint32_t rd0[16], rd1[16], r1[16], r2[16];
-            tmem_ld16(tbase + lane_base + T_DB + cq * 32, rd0);
-            tmem_ld16(tbase + lane_base + T_DB + cq * 32 + 16, rd1);
+#pragma unroll
+            for (int hq = 0; hq < 2; ++hq) {       // dS^T rows c in [32 cq + 16 hq, +16)
+                uint32_t rd[16];
+                tmem_ld16(tbase + lane_base + T_DS + cq * 32 + hq * 16, rd);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    S[hq * 16 + e] = fmaf(s_gam[cq * 32 + hq * 16 + e], S[hq * 16 + e], __uint_as_float(rd[e]));
+            }
+            store_state_bf16();
+            uint32_t r1[16], r2[16];
             tmem_ld16(tbase + lane_base + T_O1 + cq * 16, r1);
             tmem_ld16(tbase + lane_base + T_O2 + cq * 16, r2);
             tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                S[e] = fmaf(s_gam[cq * 32 + e], S[e], __uint_as_float(rd0[e]));
-                S[16 + e] = fmaf(s_gam[cq * 32 + 16 + e], S[16 + e], __uint_as_float(rd1[e]));
-            }
-            store_state_bf16();
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int i = cq * 16 + e;
