@@ -102,6 +102,20 @@ constexpr uint32_t T_O1 = 320;    // ((Q e^G) S)^T                              
 constexpr uint32_t T_S = 384;     // S^T bf16 A operand (2 per column)
 constexpr uint32_t TMEM_COLS = 512;
 
+// One explicit work unit (used by the long-sequence segment split): a token
+// range of one head, where its state starts and ends, and what to produce.
+enum : int32_t {
+    UNIT_STORE_O = 1,      // write the outputs of the range
+    UNIT_ZERO_V = 2,       // treat v as zero (U = 0): the run then maps S0 -> M S0
+    UNIT_S0_IDENTITY = 4,  // start from S0 = I (with UNIT_ZERO_V: the final state is M)
+};
+struct TcUnit {
+    int64_t t_begin, t_end;
+    const float *S0;       // [dk x dv] start state or nullptr (zeros / identity)
+    float *S_out;          // [dk x dv] final state or nullptr
+    int32_t head, flags;
+};
+
 struct TcParams {
     const void *beta, *gate;
     const float *S0;
@@ -111,6 +125,7 @@ struct TcParams {
     float *S_T;
     int32_t num_heads;
     float scale, g_floor;
+    const TcUnit *units;   // when set, block b runs units[b] instead of a (sequence, head)
 };
 
 // byte offset of (row, byte kb within a 128-byte K-block row) in a swizzled block
@@ -184,11 +199,27 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.num_heads;
-    const int n_slot = blockIdx.x / H;
-    const int hh = blockIdx.x % H;
-    const int n = p.seq_order ? p.seq_order[n_slot] : n_slot;
-    const int64_t t_begin = p.cu_seqlens[n], t_end = p.cu_seqlens[n + 1];
-    const int64_t unit = (int64_t)n * H + hh;
+    int hh;
+    int64_t t_begin, t_end;
+    const float *S0p;
+    float *S_outp;
+    int32_t flags;
+    if (p.units) {
+        const TcUnit u = p.units[blockIdx.x];
+        hh = u.head; t_begin = u.t_begin; t_end = u.t_end;
+        S0p = u.S0; S_outp = u.S_out; flags = u.flags;
+    } else {
+        const int n_slot = blockIdx.x / H;
+        hh = blockIdx.x % H;
+        const int n = p.seq_order ? p.seq_order[n_slot] : n_slot;
+        t_begin = p.cu_seqlens[n]; t_end = p.cu_seqlens[n + 1];
+        const int64_t unit = (int64_t)n * H + hh;
+        S0p = p.S0 ? p.S0 + unit * D * D : nullptr;
+        S_outp = p.S_T ? p.S_T + unit * D * D : nullptr;
+        flags = UNIT_STORE_O;
+    }
+    const bool store_o = (flags & UNIT_STORE_O) != 0;
+    const bool zero_v = (flags & UNIT_ZERO_V) != 0;
     const int nchunks = (int)((t_end - t_begin + C - 1) / C);
     const __nv_bfloat16 *beta = static_cast<const __nv_bfloat16 *>(p.beta);
     const __nv_bfloat16 *gate = static_cast<const __nv_bfloat16 *>(p.gate);
@@ -246,7 +277,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float S[32];
 #pragma unroll
     for (int r = 0; r < 32; ++r)
-        S[r] = p.S0 ? p.S0[(unit * D + cq * 32 + r) * D + vlane] : 0.0f;
+        S[r] = S0p ? S0p[(cq * 32 + r) * D + vlane]
+                   : ((flags & UNIT_S0_IDENTITY) && cq * 32 + r == vlane ? 1.0f : 0.0f);
     auto store_state_bf16 = [&]() {        // S^T as the bf16 A operand (2 rows c per column)
         uint32_t r16[16];
 #pragma unroll
@@ -611,7 +643,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 16; ++e)
-                rp[e] = __float_as_uint(to_tf32(__uint_as_float(ru[e]) - __uint_as_float(rp[e])));
+                rp[e] = __float_as_uint(to_tf32((zero_v ? 0.0f : __uint_as_float(ru[e])) - __uint_as_float(rp[e])));
             tmem_st16(tbase + lane_base + T_P + cq * 16, rp);
             tmem_wait_st();
         }
@@ -650,7 +682,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int i = cq * 16 + e;
-                if (i < L) {
+                if (store_o && i < L) {
                     const int64_t off = ((t0 + i) * H + hh) * D + vlane;
                     float x = p.scale * (__uint_as_float(r1[e]) + __uint_as_float(r2[e]));
                     if (gate) x *= sigmoidf(__bfloat162float(gate[off]));
@@ -663,9 +695,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
     }
 
-    if (!failed && p.S_T) {
+    if (!failed && S_outp) {
 #pragma unroll
-        for (int r = 0; r < 32; ++r) p.S_T[(unit * D + cq * 32 + r) * D + vlane] = S[r];
+        for (int r = 0; r < 32; ++r) S_outp[(cq * 32 + r) * D + vlane] = S[r];
     }
     if (failed && tid == 0) {
         // drain what is still in flight (bounded) before TMEM and shared memory go away

@@ -9,13 +9,17 @@
 #include <cstring>
 
 #include <cudaTypedefs.h>
+#include <algorithm>
+#include <cstdlib>
 #include <mutex>
+#include <vector>
 
 #include "kda_common.cuh"
 #include "kda_chunk_simt.cuh"
 #include "kda_chunk_tc.cuh"
 #include "kda_decode.cuh"
 #include "kda_plan.cuh"
+#include "kda_segment.cuh"
 
 namespace {
 
@@ -80,10 +84,96 @@ kda_status validate_host_seqlens(const kda_fwd_desc *d, const int32_t *cu) {
     return KDA_OK;
 }
 
+// ---------------------------------------------------------------- long-sequence split
+// When there are fewer (sequence, head) units than SMs, long sequences are cut
+// into segments so that the tensor-core prefill still fills the GPU (needs
+// cu_seqlens_host).  KDA_SEGMENTS=<P> forces P segments per sequence (tuning
+// and tests).
+constexpr int64_t kMinSegTokens = 1024;
+
+int device_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        (void)cudaGetLastError();
+        return 148;
+    }
+    return n;
+}
+
+struct SegPlan {
+    bool active = false;
+    std::vector<int32_t> nseg;      // segments per sequence (1: not split)
+    std::vector<int64_t> seglen;    // tokens per segment (multiple of 64)
+    int64_t pass1_units = 0, pass2_units = 0, jobs = 0, mat_blocks = 0;
+};
+
+bool tc_shape(const kda_fwd_desc &d) {
+    return d.io_dtype == KDA_BF16 && d.dk == 128 && d.dv == 128 && d.chunk != 16 &&
+           d.total_tokens > 0 && d.total_tokens <= INT32_MAX - 64;
+}
+
+SegPlan plan_segments(const kda_fwd_desc &d, const int32_t *cu) {
+    SegPlan pl;
+    const int32_t N = d.num_seqs, H = d.num_heads;
+    pl.nseg.assign(N, 1);
+    pl.seglen.assign(N, 0);
+    if (!cu || !tc_shape(d)) {
+        pl.pass2_units = (int64_t)N * H;
+        return pl;
+    }
+    const char *env = std::getenv("KDA_SEGMENTS");
+    const int forced = env ? std::atoi(env) : 0;
+    const int64_t units = (int64_t)N * H;
+    const int sms = device_sm_count();
+    for (int32_t n = 0; n < N; ++n) {
+        const int64_t L = (int64_t)cu[n + 1] - cu[n];
+        int64_t P = 1;
+        if (forced > 1)
+            P = std::min<int64_t>(forced, L / 128);
+        else if (units < sms)
+            P = std::min<int64_t>((2 * sms + units - 1) / units, L / kMinSegTokens);
+        if (P >= 2) {
+            const int64_t seg = ((L + P - 1) / P + 63) / 64 * 64;
+            P = (L + seg - 1) / seg;
+        }
+        if (P >= 2) {
+            pl.active = true;
+            pl.nseg[n] = (int32_t)P;
+            pl.seglen[n] = ((L + P - 1) / P + 63) / 64 * 64;
+            pl.pass1_units += (int64_t)H * ((P - 1) + (P - 2));
+            pl.jobs += H;
+            pl.mat_blocks += (int64_t)H * P;
+        }
+        pl.pass2_units += (int64_t)H * pl.nseg[n];
+    }
+    return pl;
+}
+
 // Workspace layout (each region 256-byte aligned):
-//   [0]  int32 seq_order[N]       sequences longest-first
-size_t fwd_workspace_bytes(const kda_fwd_desc *d, const int32_t *) {
-    return align256(sizeof(int32_t) * (size_t)d->num_seqs);
+//   int32 seq_order[N]                       sequences longest-first
+//   with a segment split (cu_seqlens_host given, see plan_segments):
+//   TcUnit pass1[...], TcUnit pass2[...], ScanJob jobs[...],
+//   fp32 matrices: per split (sequence, head), per segment: S_loc, M, S_in
+struct WsLayout {
+    size_t order = 0, pass1 = 0, pass2 = 0, jobs = 0, mats = 0, total = 0;
+};
+
+WsLayout ws_layout(const kda_fwd_desc *d, const SegPlan &pl) {
+    WsLayout w;
+    size_t off = align256(sizeof(int32_t) * (size_t)d->num_seqs);
+    if (pl.active) {
+        w.pass1 = off; off += align256(sizeof(kda::tck::TcUnit) * (size_t)pl.pass1_units);
+        w.pass2 = off; off += align256(sizeof(kda::tck::TcUnit) * (size_t)pl.pass2_units);
+        w.jobs = off;  off += align256(sizeof(kda::ScanJob) * (size_t)pl.jobs);
+        w.mats = off;  off += align256((size_t)pl.mat_blocks * 3u * 128u * 128u * sizeof(float));
+    }
+    w.total = off;
+    return w;
+}
+
+size_t fwd_workspace_bytes(const kda_fwd_desc *d, const int32_t *cu_host) {
+    return ws_layout(d, plan_segments(*d, cu_host)).total;
 }
 
 template <int DK, int DV, typename TIO>
@@ -139,15 +229,24 @@ bool encode_bf16_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t 
 // aligned inputs; chunk = 16 and every other shape use the CUDA-core kernel.
 bool tc_path_applies(const kda_fwd_desc &d, const void *q, const void *k, const void *v,
                      const void *g) {
-    if (d.io_dtype != KDA_BF16 || d.dk != 128 || d.dv != 128 || d.chunk == 16) return false;
-    if (d.total_tokens <= 0 || d.total_tokens > INT32_MAX - 64) return false;
+    if (!tc_shape(d)) return false;
     for (const void *ptr : {q, k, v, g})
         if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return false;
     return true;
 }
 
+cudaError_t launch_tc_units(const kda_fwd_desc &d, const void *q, const void *k, const void *v,
+                            const void *g, const kda::tck::TcParams &p, int64_t blocks,
+                            cudaStream_t stream);
+
 cudaError_t launch_tc(const kda_fwd_desc &d, const void *q, const void *k, const void *v,
                       const void *g, const kda::tck::TcParams &p, cudaStream_t stream) {
+    return launch_tc_units(d, q, k, v, g, p, (int64_t)d.num_seqs * d.num_heads, stream);
+}
+
+cudaError_t launch_tc_units(const kda_fwd_desc &d, const void *q, const void *k, const void *v,
+                            const void *g, const kda::tck::TcParams &p, int64_t blocks,
+                            cudaStream_t stream) {
     CUtensorMap tq, tk, tg, tv;
     const uint64_t rows = (uint64_t)d.total_tokens, cols = (uint64_t)d.num_heads * 128u;
     if (!encode_bf16_2d(&tq, q, rows, cols) || !encode_bf16_2d(&tk, k, rows, cols) ||
@@ -157,8 +256,8 @@ cudaError_t launch_tc(const kda_fwd_desc &d, const void *q, const void *k, const
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kda::tck::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    const int64_t blocks = (int64_t)d.num_seqs * d.num_heads;
     if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
+    if (blocks == 0) return cudaSuccess;
     kda::tck::chunk_tc_kernel<<<(unsigned)blocks, kda::tck::NT, kda::tck::SMEM_ALLOC, stream>>>(
         tq, tk, tg, tv, p);
     return cudaGetLastError();
@@ -172,13 +271,89 @@ cudaError_t launch_prefill(const kda_fwd_desc &d, const void *q, const void *k, 
                            void *o, float *S_T, cudaStream_t stream) {
     if (tc_path_applies(d, q, k, v, g)) {
         kda::tck::TcParams tp{beta, gate, S0, cu_seqlens, seq_order, o, S_T, d.num_heads, d.scale,
-                              d.g_floor};
+                              d.g_floor, nullptr};
         return launch_tc(d, q, k, v, g, tp, stream);
     }
     SimtParams p{q, k, v, g, beta, gate, S0, cu_seqlens, seq_order, o, S_T,
                  d.num_heads, d.scale, d.g_floor};
     return d.io_dtype == KDA_BF16 ? dispatch_simt<__nv_bfloat16>(d.dk, d.dv, p, d.num_seqs, stream)
                                   : dispatch_simt<float>(d.dk, d.dv, p, d.num_seqs, stream);
+}
+
+// Segment split: pass 1 (S_loc and M per segment), scan, pass 2 (outputs).
+cudaError_t launch_split(const kda_fwd_desc &d, const SegPlan &pl, const int32_t *cu,
+                         const void *q, const void *k, const void *v, const void *g,
+                         const void *beta, const float *S0, const void *gate, void *o, float *S_T,
+                         unsigned char *ws, cudaStream_t stream) {
+    using kda::tck::TcUnit;
+    const WsLayout w = ws_layout(&d, pl);
+    const int32_t N = d.num_seqs, H = d.num_heads;
+    const size_t DD = 128u * 128u;
+    float *mats = reinterpret_cast<float *>(ws + w.mats);
+    std::vector<TcUnit> p1, p2;
+    std::vector<kda::ScanJob> jobs;
+    p1.reserve((size_t)pl.pass1_units);
+    p2.reserve((size_t)pl.pass2_units);
+    size_t blk = 0;   // next (sequence, head) matrix block, each P x 3 x D^2 floats
+    for (int32_t n = 0; n < N; ++n) {
+        const int64_t t0 = cu[n], t1 = cu[n + 1];
+        const int32_t P = pl.nseg[n];
+        for (int32_t h = 0; h < H; ++h) {
+            const size_t unit = (size_t)n * H + h;
+            const float *s0 = S0 ? S0 + unit * DD : nullptr;
+            float *st = S_T ? S_T + unit * DD : nullptr;
+            if (P == 1) {
+                p2.push_back(TcUnit{t0, t1, s0, st, h, kda::tck::UNIT_STORE_O});
+                continue;
+            }
+            float *base = mats + blk * (size_t)P * 3u * DD;
+            ++blk;
+            auto Sloc = [&](int32_t sp) { return base + ((size_t)sp * 3u + 0u) * DD; };
+            auto Mp = [&](int32_t sp) { return base + ((size_t)sp * 3u + 1u) * DD; };
+            auto Sin = [&](int32_t sp) { return base + ((size_t)sp * 3u + 2u) * DD; };
+            for (int32_t sp = 0; sp < P; ++sp) {
+                const int64_t a = t0 + (int64_t)sp * pl.seglen[n];
+                const int64_t b = std::min<int64_t>(t1, a + pl.seglen[n]);
+                if (sp + 1 < P) p1.push_back(TcUnit{a, b, sp == 0 ? s0 : nullptr, Sloc(sp), h, 0});
+                if (sp >= 1 && sp + 1 < P)
+                    p1.push_back(TcUnit{a, b, nullptr, Mp(sp), h,
+                                        kda::tck::UNIT_ZERO_V | kda::tck::UNIT_S0_IDENTITY});
+                p2.push_back(TcUnit{a, b, sp == 0 ? s0 : Sin(sp), sp + 1 == P ? st : nullptr, h,
+                                    kda::tck::UNIT_STORE_O});
+            }
+            jobs.push_back(kda::ScanJob{Sloc(0), Mp(0), Sin(0), (int64_t)(3u * DD), P});
+        }
+    }
+    auto longest_first = [](const TcUnit &x, const TcUnit &y) {
+        return (x.t_end - x.t_begin) > (y.t_end - y.t_begin);
+    };
+    std::stable_sort(p1.begin(), p1.end(), longest_first);
+    std::stable_sort(p2.begin(), p2.end(), longest_first);
+    TcUnit *d1 = reinterpret_cast<TcUnit *>(ws + w.pass1);
+    TcUnit *d2 = reinterpret_cast<TcUnit *>(ws + w.pass2);
+    kda::ScanJob *dj = reinterpret_cast<kda::ScanJob *>(ws + w.jobs);
+    cudaError_t e;
+    if (!p1.empty() &&
+        (e = cudaMemcpyAsync(d1, p1.data(), p1.size() * sizeof(TcUnit), cudaMemcpyHostToDevice, stream)) != cudaSuccess)
+        return e;
+    if ((e = cudaMemcpyAsync(d2, p2.data(), p2.size() * sizeof(TcUnit), cudaMemcpyHostToDevice, stream)) != cudaSuccess)
+        return e;
+    if ((e = cudaMemcpyAsync(dj, jobs.data(), jobs.size() * sizeof(kda::ScanJob), cudaMemcpyHostToDevice,
+                             stream)) != cudaSuccess)
+        return e;
+    kda::tck::TcParams tp{beta, gate, nullptr, nullptr, nullptr, o, nullptr, H, d.scale, d.g_floor, d1};
+    if (!p1.empty()) {
+        tp.units = d1;
+        if ((e = launch_tc_units(d, q, k, v, g, tp, (int64_t)p1.size(), stream)) != cudaSuccess) return e;
+    }
+    const size_t scan_smem = 2u * DD * sizeof(float);
+    if ((e = cudaFuncSetAttribute(kda::segment_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)scan_smem)) != cudaSuccess)
+        return e;
+    kda::segment_scan_kernel<<<(unsigned)jobs.size(), 256, scan_smem, stream>>>(dj);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    tp.units = d2;
+    return launch_tc_units(d, q, k, v, g, tp, (int64_t)p2.size(), stream);
 }
 
 template <int DK, int DV, typename TIO>
@@ -241,6 +416,13 @@ kda_status kda_chunk_fwd(const kda_fwd_desc *desc, const void *q, const void *k,
         for (const Range &r : ins)
             if (overlaps(rw, r)) return KDA_ERR_INVALID_ARG;
         if (overlaps(rw, ro) || overlaps(rw, rs)) return KDA_ERR_INVALID_ARG;
+    }
+
+    const SegPlan pl = plan_segments(d, cu_seqlens_host);
+    if (pl.active && tc_path_applies(d, q, k, v, g)) {
+        const cudaError_t e = launch_split(d, pl, cu_seqlens_host, q, k, v, g, beta, S0, gate, o, S_T,
+                                           static_cast<unsigned char *>(workspace), stream);
+        return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     }
 
     int32_t *seq_order = static_cast<int32_t *>(workspace);
