@@ -53,6 +53,28 @@ def bytes_per_token_head(dk=DK, dv=DV, esz=2):
     return esz * (3 * dk + dv + 1) + esz * dv
 
 
+# DRAM traffic per unit from the ncu captures under profiles/ (bytes), valid only
+# for the kernel source they were taken from (sha1 prefix); otherwise null.
+PROFILED_TRAFFIC = {
+    "csrc/kda_chunk_tc.cuh": {"sha1": "4b144001c6b5", "bytes_per_token_head": (281.834240e6 + 54.751488e6) / 262144,
+                              "profile": "profiles/chunk_tc_kernel_prefill_4x4096x16.md"},
+    "csrc/kda_decode.cuh": {"sha1": "8e75484b34f3", "bytes_per_head_step": (273.707520e6 + 212.401408e6) / 4096,
+                            "profile": "profiles/decode_kernel_64x64.md"},
+}
+
+
+def profiled_traffic(src: str, key: str, units: float):
+    """Traffic per launch scaled from the capture, or None if the kernel changed."""
+    import hashlib
+    rec = PROFILED_TRAFFIC[src]
+    path = os.path.join(ROOT, "gated_delta_rule_136_b200", src)
+    try:
+        digest = hashlib.sha1(open(path, "rb").read()).hexdigest()[:12]
+    except OSError:
+        return None
+    return rec[key] * units if digest == rec["sha1"] else None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -203,7 +225,7 @@ def reference_arm(args):
 
 
 def main():
-    global B, T, H
+    global B, T, H, DEC_B, DEC_STEPS
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
@@ -218,9 +240,15 @@ def main():
     ap.add_argument("--batch", type=int, default=B)
     ap.add_argument("--seqlen", type=int, default=T)
     ap.add_argument("--heads", type=int, default=H)
+    ap.add_argument("--decode-batch", type=int, default=DEC_B)
+    ap.add_argument("--decode-steps", type=int, default=DEC_STEPS)
+    ap.add_argument("--all-workloads", action="store_true",
+                    help="also time the varlen (64 x [512, 32768] x 64 heads) and the "
+                         "1M-token x 32-head floor-stress prefill")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     B, T, H = args.batch, args.seqlen, args.heads
+    DEC_B, DEC_STEPS = args.decode_batch, args.decode_steps
     if args.impl == "reference":
         return reference_arm(args)
 
@@ -375,10 +403,55 @@ def main():
                   "state_hbm_gbs": dec_gbs,
                   "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"],
                                "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"],
-                               "traffic": None},
+                               "traffic": profiled_traffic("csrc/kda_decode.cuh",
+                                                           "bytes_per_head_step", units)},
                   "bytes_per_step": dec_bytes, "gpu_launches": DEC_STEPS}
         del d, S, od
         torch.cuda.empty_cache()
+
+    others = None
+    if args.all_workloads:
+        others = {}
+        cases = {
+            "varlen 64 sequences, lengths U[512, 32768], H=64, S0 ~ N(0, 0.02)":
+                dict(lengths=inputs.varlen_lengths(64, 512, 32768, seed=0), H=64, s0_std=0.02,
+                     g_mode="softplus"),
+            "1 sequence x 2^20 tokens, H=32, g ~ -5 U(0.8, 1)":
+                dict(lengths=[1 << 20], H=32, s0_std=None, g_mode="floor_stress"),
+        }
+        for name, c in cases.items():
+            w = inputs.prefill_inputs(c["lengths"], H=c["H"], dk=DK, dv=DV, device=dev, seed=rank,
+                                      s0_std=c["s0_std"], g_mode=c["g_mode"])
+            ow = torch.empty_like(w["v"])
+            Sw = torch.empty((len(c["lengths"]), c["H"], DK, DV), device=dev, dtype=torch.float32)
+            wsz = kbind.workspace_size(w["q"].shape[0], len(c["lengths"]), c["H"], DK, DV,
+                                       cu_seqlens_host=w["cu_seqlens_host"])
+            wsw = torch.empty(max(256, wsz), dtype=torch.uint8, device=dev)
+            run = lambda: chunk_fwd(w["q"], w["k"], w["v"], w["g"], w["beta"], S0=w["S0"],
+                                    cu_seqlens=w["cu_seqlens"], cu_seqlens_host=w["cu_seqlens_host"],
+                                    out=ow, final_state_out=Sw, workspace=wsw)
+            for _ in range(2):
+                run()
+            barrier()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 3
+            tw0 = time.time()
+            a.record(stream)
+            for _ in range(reps):
+                run()
+            b.record(stream)
+            barrier()
+            if sampler:
+                sampler.mark(tw0, time.time())
+            ms = max_over_ranks(a.elapsed_time(b)) / reps
+            ttok = int(w["q"].shape[0])
+            byts = ttok * c["H"] * bytes_per_token_head() + len(c["lengths"]) * c["H"] * DK * DV * 4 * (
+                2 if c["s0_std"] is not None else 1)
+            others[name] = {"tokens": ttok, "ms": ms, "tokens_per_s": world * ttok / (ms / 1e3),
+                            "alg_gbs": byts / (ms / 1e3) / 1e9,
+                            "roofline_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+            del w, ow, Sw, wsw
+            torch.cuda.empty_cache()
 
     if sampler:
         sampler.stop()
@@ -405,11 +478,13 @@ def main():
                        "l2": "inputs (1.36 GB per step) larger than L2; no flush"},
             "tflops": tflops, "pct_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": None,
+                         "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
+                         "traffic": profiled_traffic("csrc/kda_chunk_tc.cuh", "bytes_per_token_head", th),
                          "kernel": "kda_chunk_fwd (plan + chunk kernel)",
                          "alg_bytes_per_launch": alg_bytes, "alg_flops_per_launch": alg_flops,
                          "peak_source": peaks["source"]},
             "e2e": e2e, "decode": decode, "cpu_baseline": cpu_baseline,
+            "other_workloads": others,
             "gpu_launches": 2 * args.steps, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

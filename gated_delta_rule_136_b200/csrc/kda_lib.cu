@@ -126,13 +126,30 @@ SegPlan plan_segments(const kda_fwd_desc &d, const int32_t *cu) {
     const int forced = env ? std::atoi(env) : 0;
     const int64_t units = (int64_t)N * H;
     const int sms = device_sm_count();
+    // Wave model with the longest sequence's chunk count C: unsplit time ~
+    // ceil(U / SMs) * C; with P segments pass 1 runs U (2P - 3) units and pass 2
+    // U P units, each of ceil(C / P) chunks.  Take the best P, and split only
+    // if it saves at least 10 %.
+    int64_t best_p = 1;
+    if (forced <= 1 && units < sms) {
+        int64_t cmax = 0;
+        for (int32_t n = 0; n < N; ++n) cmax = std::max<int64_t>(cmax, ((int64_t)cu[n + 1] - cu[n] + 63) / 64);
+        auto waves = [&](int64_t x) { return (x + sms - 1) / sms; };
+        const int64_t t1 = waves(units) * cmax;
+        int64_t best_t = t1;
+        for (int64_t P = 2; P <= 64 && P * kMinSegTokens / 64 <= cmax; ++P) {
+            const int64_t t = (waves(units * (2 * P - 3)) + waves(units * P)) * ((cmax + P - 1) / P);
+            if (t < best_t) { best_t = t; best_p = P; }
+        }
+        if (best_t * 10 > t1 * 9) best_p = 1;
+    }
     for (int32_t n = 0; n < N; ++n) {
         const int64_t L = (int64_t)cu[n + 1] - cu[n];
         int64_t P = 1;
         if (forced > 1)
             P = std::min<int64_t>(forced, L / 128);
-        else if (units < sms)
-            P = std::min<int64_t>((2 * sms + units - 1) / units, L / kMinSegTokens);
+        else if (best_p > 1)
+            P = std::min<int64_t>(best_p, L / kMinSegTokens);
         if (P >= 2) {
             const int64_t seg = ((L + P - 1) / P + 63) / 64 * 64;
             P = (L + seg - 1) / seg;
