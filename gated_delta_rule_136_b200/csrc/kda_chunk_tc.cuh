@@ -63,6 +63,8 @@ constexpr uint32_t OFF_KB = OFF_INTRA + 32768;     // K^(b), b = 0..3, packed ro
 constexpr uint32_t OFF_SCR = OFF_INTRA;            // A_kk -> T, fp32 [64][68]
 constexpr uint32_t SCR_LD = 68;                    // 16-byte aligned rows
 constexpr uint32_t OFF_TP = OFF_INTRA + 17408;     // T' bf16 K-major [64 i x 64 j]: 8 KB
+constexpr uint32_t OFF_XS = OFF_INTRA + 25600;     // inverse scratch: 4 warps x [32 x 8] fp32: 4 KB
+constexpr uint32_t XS_LD = 8;
 constexpr uint32_t OFF_W = OFF_INTRA + 41984;      // W bf16 MN-major [128 c x 64 j]: 16 KB
 constexpr uint32_t OFF_QG = OFF_INTRA + 73728;     // Q e^G bf16 MN-major [128 c x 64 i]: 16 KB
 constexpr uint32_t OFF_KG = OFF_QG + 16384;        // K e^G bf16 K-major [128 c x 64 j]: 16 KB
@@ -71,12 +73,16 @@ constexpr uint32_t OFF_KG = OFF_QG + 16384;        // K e^G bf16 K-major [128 c 
 constexpr uint32_t OFF_AK = OFF_KG + 16384;
 constexpr uint32_t AK_KBLK = 192u * 128u;          // 24 KB per K-block
 constexpr uint32_t OFF_AQK = OFF_AK;               // + kb * AK_KBLK + row * 128
+// Between the second state MMA and the next A readout the A_qk rows are free:
+// the output tile waits there for its TMA store, bf16 [64 tokens x 64 v] per
+// K-block (v in [0, 64) at OFF_AK, [64, 128) at OFF_AK + AK_KBLK).
+constexpr uint32_t OFF_OST = OFF_AK;
 constexpr uint32_t OFF_KHT = OFF_AK + 64u * 128u;  // + kb * AK_KBLK + row * 128
-constexpr uint32_t OFF_SMALL = OFF_AK + 2u * AK_KBLK;  // beta[64], gamma[128], barriers, tmem base
-constexpr uint32_t OFF_TOT = OFF_SMALL + 1024;     // per-row-group decay totals [8][64] fp32
-constexpr uint32_t SMEM_BYTES = OFF_TOT + 2048;
+constexpr uint32_t OFF_SMALL = OFF_AK + 2u * AK_KBLK;  // beta[64], gamma[2][128], barriers, tmem base
+constexpr uint32_t SMEM_BYTES = OFF_SMALL + 2048;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024; // slack for aligning the base
 static_assert(OFF_W + 16384 <= OFF_INTRA + 73728, "post-MMA tiles fit the intra region");
+static_assert(OFF_TP + 8192 <= OFF_XS && OFF_XS + 4096 <= OFF_W, "inverse scratch between T' and W");
 static_assert(OFF_QG - OFF_W < (1u << 18) && (OFF_QG - OFF_W) % 16 == 0, "W | Q e^G as one MN-major operand");
 static_assert(OFF_KB + 40960 <= OFF_INTRA + 73728, "intra tiles fit");
 static_assert(SMEM_ALLOC <= 232448, "fits in 227 KB");
@@ -158,6 +164,59 @@ __device__ __forceinline__ void mma_16x8x8_tf32(float (&d)[4], const uint32_t (&
                  : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+// D[16x8] += A[16x16] B[16x8], bf16 inputs, fp32 accumulation; fragments:
+//   a = {A[g][2t..2t+1], A[g+8][2t..], A[g][2t+8..], A[g+8][2t+8..]},
+//   b = {B[2t..2t+1][g], B[2t+8..2t+9][g]},  d as for the tf32 form above.
+__device__ __forceinline__ void mma_16x8x16_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+                 "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// four 8x8 b16 matrices, transposed on the way in: lane l gives the address
+// of row l % 8 of matrix l / 8 (16 contiguous bytes); lane (g, t) receives
+// elements (2t, g) and (2t + 1, g) of each matrix
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr) : "memory");
+}
+
+// two 8x8 b16 matrices from the fragment layout (lane (g, t) holds elements
+// (g, 2t) and (g, 2t + 1)), stored transposed: lane l (< 16) gives the address
+// of stored row l % 8 of matrix l / 8
+__device__ __forceinline__ void stsm_x2_trans(uint32_t addr, uint32_t r0, uint32_t r1) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x2.trans.shared.b16 [%0], {%1, %2};"
+                 :: "r"(addr), "r"(r0), "r"(r1) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// bf16 pair in one 32-bit word -> two floats (low half first)
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// 2^x on the special-function unit (approximate; denormal results flush to zero)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// waits (bounded) for the barrier phases [done, issued) of `bar` to complete
+__device__ __noinline__ void drain_phases(uint64_t *bar, uint32_t done, uint32_t issued) {
+    for (uint32_t k = done; k < issued; ++k) mbar_wait(bar, k & 1u, 1u << 20);
+}
+
+// sigmoid on the special-function unit (relative error a few fp32 ulp, far
+// below the bf16 rounding of the gated output)
+__device__ __forceinline__ float sigmoid_fast(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
                                             uint64_t *bar) {
     asm volatile(
@@ -165,6 +224,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         "[%0], [%1, {%2, %3}], [%4];"
         ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar)) : "memory");
 }
+
+// TMA tile store from shared memory (bulk-group completion)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+                 ::"l"(map), "r"(x), "r"(y), "r"(src) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the shared-memory sources of this thread's committed stores may be reused
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// this thread's committed stores are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
@@ -184,17 +254,16 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __global__ void __launch_bounds__(NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
-                TcParams p)
+                const __grid_constant__ CUtensorMap tm_o, TcParams p)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float *s_beta = reinterpret_cast<float *>(sm + OFF_SMALL);          // [64]
-    float *s_gam = s_beta + 64;                                          // [128]
-    uint64_t *bar_qkg = reinterpret_cast<uint64_t *>(sm + OFF_SMALL + 768);   // [2]
+    float *s_gam = s_beta + 64;                                          // [2][128], by chunk parity
+    uint64_t *bar_qkg = reinterpret_cast<uint64_t *>(sm + OFF_SMALL + 1280);  // [2]
     uint64_t *bar_v = bar_qkg + 2;
     uint64_t *bar_mma = bar_qkg + 3;
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + OFF_SMALL + 832);
-    float *s_tot = reinterpret_cast<float *>(sm + OFF_TOT);              // [8][64]
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + OFF_SMALL + 1344);
     float *scr = reinterpret_cast<float *>(sm + OFF_SCR);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -232,9 +301,36 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int cq = warp >> 2;
     const int vlane = lq * 32 + lane;
     const uint32_t lane_base = (uint32_t)(lq * 32) << 16;
-    // Prep coordinates: 8-row group and 32-channel half of the pass.
-    const int rg = warp & 7;
-    const int cl = (warp >> 3) * 32 + lane;        // channel within the pass, 0..63
+    // Prep coordinates (mma fragment layout): channel tile nt, block pair mp,
+    // lane (gq, tq); channels cA, cA + 1 of the pass.
+    const int nt = warp & 7, mp = warp >> 3;
+    const int gq = lane >> 2, tq = lane & 3;
+    const int cA = nt * 8 + 2 * tq;
+    // swizzled byte offset of (a row r with r % 8 == gq, channel cA) in the tf32
+    // K-major operand tiles, and the K-block of cA
+    const uint32_t kblk = (uint32_t)(cA >> 5);
+    const uint32_t kbyte = (uint32_t)(cA & 31) * 4u;
+    const uint32_t sw_lane = ((((kbyte >> 4) & 7u) ^ (uint32_t)gq) << 4) + (kbyte & 15u);
+    const uint32_t xt_lane = OFF_XT + kblk * 16384u + sw_lane;
+    const uint32_t kb_lane = OFF_KB + sw_lane;
+    // constant A fragments of the prefix-sum products (bf16 1.0 = 0x3F80):
+    //   a_blk: 16x16 lower triangle with diagonal;  a_ref[kb]: rows m < 4 select block kb <= m
+    uint32_t a_blk[4];
+    a_blk[0] = (2 * tq <= gq ? 0x3F80u : 0u) | (2 * tq + 1 <= gq ? 0x3F800000u : 0u);
+    a_blk[1] = 0x3F803F80u;
+    a_blk[2] = 0u;
+    a_blk[3] = a_blk[0];
+    uint32_t a_ref[NB][4];
+#pragma unroll
+    for (int kb = 0; kb < NB; ++kb) {
+        const uint32_t v = (gq < NB && kb <= gq) ? 0x3F803F80u : 0u;
+        a_ref[kb][0] = v; a_ref[kb][1] = 0u; a_ref[kb][2] = v; a_ref[kb][3] = 0u;
+    }
+    // floor: the largest bf16 fb <= floor; max(g, floor) = max(g, fb) + (g <= fb) (floor - fb)
+    const __nv_bfloat16 fb = __float2bfloat16_rd(p.g_floor);
+    const __nv_bfloat162 floor_b2 = __halves2bfloat162(fb, fb);
+    const float floor_gap = p.g_floor - __bfloat162float(fb);
+    const bool floor_inexact = floor_gap != 0.0f;
 
     if (warp == 0) {
         tmem_alloc(s_tmem, TMEM_COLS);
@@ -252,6 +348,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
     const uint32_t tbase = *s_tmem;
     const uint32_t smb = smem_u32(sm);
+    const bool leader = elect_one();       // this warp's MMA-issuing lane (used in warp 0)
 
     // issue the TMA loads of chunk `ci` (mask bit 0: pass 0, bit 1: pass 1, bit 2: v)
     auto issue_loads = [&](int ci, int mask) {
@@ -303,6 +400,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     uint32_t mma_phase = 0, mma_issued = 0;
     bool failed = false;
+    // first token of the output tile waiting in the staging area (-1: none);
+    // tid 0 issues its TMA store after the next block barrier
+    int64_t o_row = -1;
+    auto store_o_tile = [&]() {            // tid 0; the staging tile is complete and fenced
+        const int x = hh * D;
+        tma_store_2d(&tm_o, smb + OFF_OST, x, (int)o_row);
+        tma_store_2d(&tm_o, smb + OFF_OST + AK_KBLK, x + 64, (int)o_row);
+        bulk_commit();
+    };
     // beta of the next chunk, loaded one chunk ahead (64 strided values)
     auto load_beta = [&](int ci) -> float {
         const int64_t tb = t_begin + (int64_t)ci * C + tid;
@@ -344,9 +450,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         return tmpl + (uint64_t)(byte_off >> 4);
     };
 
-    const float g_floor = p.g_floor;
     const float L2E = 1.4426950408889634f;
-    (void)L2E;
 
     for (int ci = 0; ci < nchunks && !failed; ++ci) {
         const int64_t t0 = t_begin + (int64_t)ci * C;
@@ -354,115 +458,186 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t ld_par = (uint32_t)(ci & 1);
 
         // ================================================= prep + A MMAs, 2 passes of 64 key channels
+        // Warp (nt, mp) of a pass owns channels 8 nt .. 8 nt + 7 of the pass and the
+        // 16-token blocks 2 mp, 2 mp + 1; lane (gq, tq) holds channels cA = 8 nt + 2 tq,
+        // cA + 1 of tokens 16 b + gq and 16 b + gq + 8 (mma fragment layout).
         bool loads_ok = true;
-        for (int pass = 0; pass < 2 && !failed; ++pass) {
-            // every thread observes the TMA barrier itself (no block barrier here, so
-            // this pass's first part overlaps the previous pass's MMA issue); a
-            // timeout is folded into the next block-wide barrier
+        const bool ragged = L < C;
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
             loads_ok = mbar_wait(&bar_qkg[pass], ld_par) && loads_ok;
             ++qkg_done[pass];
-            const unsigned char *raw = sm + (pass ? OFF_QKG1 : OFF_QKG0);
-            const int c = pass * 64 + cl;
+            const uint32_t raw = smb + (pass ? OFF_QKG1 : OFF_QKG0);
             if (pass == 0) {
                 if (tid < C) s_beta[tid] = beta_next;
                 beta_next = load_beta(ci + 1);
             }
-            // local inclusive cumulative decay over this thread's 8 rows
-            float G[8];
-            {
-                float acc = 0.0f;
+            // (1) decay prefix sums on the warp-level tensor cores: with
+            //     gc = max(g, floor) (zero past the chunk's end),
+            //       x_i   = sum of gc over block b(i) up to i      = G_i - r_b(i)
+            //       r_b+1 = sum of gc over blocks 0..b
+            //     as products of 0/1 matrices with gc (bf16 operands, fp32 sums:
+            //     exact up to the fp32 rounding of the sums)
+            uint32_t gf[2][4];                     // [tokens 32h..][block 2h + (j>>1), half j&1]
+            ldsm_x4_trans(gf[0], raw + QKG_G + sw128((uint32_t)lane, (uint32_t)nt * 16u));
+            ldsm_x4_trans(gf[1], raw + QKG_G + sw128((uint32_t)(32 + lane), (uint32_t)nt * 16u));
+            uint32_t gi[2][4];                     // indicator g <= fb (floor not a bf16 value)
 #pragma unroll
-                for (int r = 0; r < 8; ++r) {
-                    const int i = rg * 8 + r;
-                    const float gi = i < L ? fmaxf(bf16_at(raw + QKG_G, i, cl), g_floor) : 0.0f;
-                    acc += gi;
-                    G[r] = acc;
+            for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const __nv_bfloat162 gv = *reinterpret_cast<const __nv_bfloat162 *>(&gf[h][j]);
+                    __nv_bfloat162 gc = __hmax2(gv, floor_b2);
+                    __nv_bfloat162 ind = __hle2(gv, floor_b2);
+                    if (ragged) {                  // tokens past the chunk's end contribute nothing
+                        const int tok = 32 * h + 8 * j + 2 * tq;
+                        const uint32_t keep = (tok < L ? 0x0000FFFFu : 0u) | (tok + 1 < L ? 0xFFFF0000u : 0u);
+                        gf[h][j] = *reinterpret_cast<uint32_t *>(&gc) & keep;
+                        gi[h][j] = *reinterpret_cast<uint32_t *>(&ind) & keep;
+                    } else {
+                        gf[h][j] = *reinterpret_cast<uint32_t *>(&gc);
+                        gi[h][j] = *reinterpret_cast<uint32_t *>(&ind);
+                    }
                 }
-                s_tot[rg * 64 + cl] = acc;
             }
-            // q, k of the 8 rows (issued before the barrier to overlap its latency)
-            float qv[8], kv[8];
+            float xs[2][4], rr[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                qv[r] = bf16_at(raw + QKG_Q, rg * 8 + r, cl);
-                kv[r] = bf16_at(raw + QKG_K, rg * 8 + r, cl);
+            for (int bb = 0; bb < 2; ++bb) {
+                const uint32_t b0 = mp ? gf[1][2 * bb] : gf[0][2 * bb];
+                const uint32_t b1 = mp ? gf[1][2 * bb + 1] : gf[0][2 * bb + 1];
+                xs[bb][0] = xs[bb][1] = xs[bb][2] = xs[bb][3] = 0.0f;
+                mma_16x8x16_bf16(xs[bb], a_blk, b0, b1);
             }
-            if (pass == 1) {                       // pass-0 A MMAs done (also syncs s_tot)
-                const bool ok = tid == 0 ? mbar_wait(bar_mma, mma_phase & 1) : true;
-                const bool all = __syncthreads_and(ok && loads_ok) != 0;
-                if (all && tid != 0) (void)mbar_try_wait(bar_mma, mma_phase & 1);
+#pragma unroll
+            for (int kb = 0; kb < NB; ++kb) mma_16x8x16_bf16(rr, a_ref[kb], gf[kb >> 1][2 * (kb & 1)], gf[kb >> 1][2 * (kb & 1) + 1]);
+            if (floor_inexact) {                   // + (floor - fb) x (the same sums of the indicator)
+                float xi[2][4], ri[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                for (int bb = 0; bb < 2; ++bb) {
+                    const uint32_t b0 = mp ? gi[1][2 * bb] : gi[0][2 * bb];
+                    const uint32_t b1 = mp ? gi[1][2 * bb + 1] : gi[0][2 * bb + 1];
+                    xi[bb][0] = xi[bb][1] = xi[bb][2] = xi[bb][3] = 0.0f;
+                    mma_16x8x16_bf16(xi[bb], a_blk, b0, b1);
+                }
+#pragma unroll
+                for (int kb = 0; kb < NB; ++kb) mma_16x8x16_bf16(ri, a_ref[kb], gi[kb >> 1][2 * (kb & 1)], gi[kb >> 1][2 * (kb & 1) + 1]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    xs[0][e] = fmaf(floor_gap, xi[0][e], xs[0][e]);
+                    xs[1][e] = fmaf(floor_gap, xi[1][e], xs[1][e]);
+                    rr[e] = fmaf(floor_gap, ri[e], rr[e]);
+                }
+            }
+            // (2) block decay factors eT_b = e^{r_b+1 - r_b} for this lane's two channels
+            //     (rows 0..3 of the r tile sit in lanes 4 m + tq)
+            float2 eT[NB];
+            {
+                float pa = 0.0f, pb = 0.0f;
+#pragma unroll
+                for (int m = 0; m < NB; ++m) {
+                    const float ra = __shfl_sync(0xffffffffu, rr[0], 4 * m + tq);
+                    const float rb2 = __shfl_sync(0xffffffffu, rr[1], 4 * m + tq);
+                    eT[m] = make_float2(fexp(ra - pa), fexp(rb2 - pb));
+                    pa = ra; pb = rb2;
+                }
+            }
+            if (mp == 0 && gq == 0) {              // gamma = e^{r_4} for the state update
+                const float2 g4 = __fmul2_rn(__fmul2_rn(eT[0], eT[1]), __fmul2_rn(eT[2], eT[3]));
+                *reinterpret_cast<float2 *>(s_gam + (ci & 1) * D + pass * 64 + cA) = g4;
+            }
+            // (3) per-element factors; the stores that no MMA in flight reads go first
+            float2 qt[2][2], kt[2][2], kbar[2][2];
+            const float2 l2e = make_float2(L2E, L2E), nl2e = make_float2(-L2E, -L2E);
+            const uint32_t kh_col = OFF_KHT;       // + (i >> 5) * AK_KBLK + sw128(c, (i & 31) * 4)
+#pragma unroll
+            for (int bb = 0; bb < 2; ++bb) {
+                const int b = 2 * mp + bb;
+                float2 Eb = make_float2(1.0f, 1.0f), eK = make_float2(1.0f, 1.0f);
+#pragma unroll
+                for (int m = 0; m < NB; ++m) {
+                    if (m < b) Eb = __fmul2_rn(Eb, eT[m]);
+                    else eK = __fmul2_rn(eK, eT[m]);
+                }
+                uint32_t pq[2], pk[2];
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int i = 16 * b + gq + 8 * hr;
+                    const float2 x2 = make_float2(xs[bb][2 * hr], xs[bb][2 * hr + 1]);
+                    const float2 t2 = __fmul2_rn(x2, l2e), u2 = __fmul2_rn(x2, nl2e);
+                    const float2 gt = make_float2(ex2_approx(t2.x), ex2_approx(t2.y));       // Gt_i
+                    const float2 ig = make_float2(ex2_approx(u2.x), ex2_approx(u2.y));       // 1 / Gt_i
+                    const uint32_t qoff = raw + QKG_Q + sw128((uint32_t)i, (uint32_t)cA * 2u);
+                    const float2 q2 = unpack_bf16x2(ld_shared_u32(qoff));
+                    const float2 k2 = unpack_bf16x2(ld_shared_u32(qoff + (QKG_K - QKG_Q)));
+                    qt[bb][hr] = __fmul2_rn(q2, gt);
+                    kt[bb][hr] = __fmul2_rn(k2, gt);
+                    kbar[bb][hr] = __fmul2_rn(k2, ig);                                        // Kbar_i
+                    const float2 qg = __fmul2_rn(qt[bb][hr], Eb), kg = __fmul2_rn(kt[bb][hr], Eb);
+                    pq[hr] = pack_bf16(qg.x, qg.y);
+                    pk[hr] = pack_bf16(kg.x, kg.y);
+                    // K^(4)^T [c x j] tf32: two channels of token i
+                    const float2 kh = __fmul2_rn(kbar[bb][hr], eK);
+                    const uint32_t cg = (uint32_t)(pass * 64 + cA);
+                    const uint32_t kho = kh_col + (uint32_t)(i >> 5) * AK_KBLK;
+                    *reinterpret_cast<float *>(sm + kho + sw128(cg, (uint32_t)(i & 31) * 4u)) = to_tf32(kh.x);
+                    *reinterpret_cast<float *>(sm + kho + sw128(cg + 1u, (uint32_t)(i & 31) * 4u)) = to_tf32(kh.y);
+                }
+                // Q e^G and K e^G (bf16 [c x i], tokens contiguous): transposing matrix stores
+                {
+                    const uint32_t row = (uint32_t)(pass * 64 + nt * 8 + (lane & 7));
+                    const uint32_t tb2 = (uint32_t)(16 * b + 8 * ((lane >> 3) & 1)) * 2u;
+                    stsm_x2_trans(smb + OFF_QG + sw128(row, tb2), pq[0], pq[1]);
+                    stsm_x2_trans(smb + OFF_KG + sw128(row, tb2), pk[0], pk[1]);
+                }
+            }
+            if (pass == 1) {                       // pass-0 A MMAs must be done with X~ and K^(b)
+                loads_ok = mbar_wait(bar_mma, mma_phase & 1) && loads_ok;
                 ++mma_phase;
                 tc_fence_after();
-                if (!all) { failed = true; break; }
-            } else if (!__syncthreads_and(loads_ok)) {
-                failed = true;
-                break;
             }
-            // prefix over row groups: P[k] = sum of the first k group totals
-            float P[9];
-            P[0] = 0.0f;
+            // (4) the A-MMA operands: X~ rows (q~ at 32 b + r, k~ at 32 b + 16 + r) and the
+            //     K^(b') copies, b' >= b (tf32 operands: the MMA reads the leading 19 bits)
 #pragma unroll
-            for (int k = 0; k < 8; ++k) P[k + 1] = P[k] + s_tot[k * 64 + cl];
-            const int b = rg >> 1;                 // 16-token block of these rows
-            float rg_pre = 0.0f;                   // P[rg]
+            for (int bb = 0; bb < 2; ++bb) {
+                const int b = 2 * mp + bb;
+                float2 dfac[NB];                   // e^{r_b' - r_b} for b' > b
+                {
+                    float2 run = make_float2(1.0f, 1.0f);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) rg_pre = (k == rg) ? P[k] : rg_pre;
-            float rb = 0.0f;                       // r_b = P[2b]
+                    for (int m = 0; m < NB; ++m) {
+                        if (m > b) run = __fmul2_rn(run, eT[m - 1]);
+                        dfac[m] = run;
+                    }
+                }
 #pragma unroll
-            for (int k = 0; k < 4; ++k) rb = (k == b) ? P[2 * k] : rb;
-            const float r4 = P[8];
-            float dfac[NB];                        // e^{r_b' - r_b}, b' >= b
+                for (int hr = 0; hr < 2; ++hr) {
+                    const uint32_t i = (uint32_t)(16 * b + 8 * hr) + (uint32_t)gq;
+                    const uint32_t xrow = (uint32_t)(32 * b + 8 * hr) + (uint32_t)gq;
+                    *reinterpret_cast<float2 *>(sm + xt_lane + xrow * 128u) = qt[bb][hr];
+                    *reinterpret_cast<float2 *>(sm + xt_lane + (xrow + 16u) * 128u) = kt[bb][hr];
 #pragma unroll
-            for (int k = 0; k < NB; ++k) dfac[k] = k >= b ? fexp(P[2 * k] - rb) : 0.0f;
-            const float eb = fexp(rb);             // e^{r_b}: rebases Gt to the chunk start
-            const float e4 = fexp(r4 - rb);        // e^{r_4 - r_b}
-            if (rg == 0) s_gam[c] = fexp(r4);
-            const uint32_t kbyte = (uint32_t)(cl & 31) * 4u;
-            const uint32_t kblk = (uint32_t)(cl >> 5);
-            unsigned char *xt = sm + OFF_XT + kblk * 16384u;
-            float qg[8], kg[8], kh[8];
-#pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                const int i = rg * 8 + r;
-                const float Gi = rg_pre + G[r];
-                const float gt = fexp(Gi - rb);            // Gt_i
-                const float kbar = kv[r] * fexp(rb - Gi);   // Kbar_i
-                const float qt = qv[r] * gt, kt = kv[r] * gt;
-                const uint32_t row = 32u * b + (uint32_t)(i & 15);
-                *reinterpret_cast<float *>(xt + sw128(row, kbyte)) = to_tf32(qt);
-                *reinterpret_cast<float *>(xt + sw128(row + 16, kbyte)) = to_tf32(kt);
-                qg[r] = qt * eb;
-                kg[r] = kt * eb;
-                kh[r] = kbar * e4;
-#pragma unroll
-                for (int bp = 0; bp < NB; ++bp) {
-                    if (bp < b) continue;
-                    unsigned char *tile = sm + OFF_KB + kb_base(bp) + kblk * kb_rows(bp) * 128u;
-                    *reinterpret_cast<float *>(tile + sw128(i, kbyte)) = to_tf32(kbar * dfac[bp]);
+                    for (int m = 0; m < NB; ++m) {
+                        if (m < b) continue;
+                        const float2 v = m == b ? kbar[bb][hr] : __fmul2_rn(kbar[bb][hr], dfac[m]);
+                        *reinterpret_cast<float2 *>(sm + kb_lane + kb_base(m) + kblk * kb_rows(m) * 128u + i * 128u) = v;
+                    }
                 }
             }
-            // Q e^G (MN-major [c x i]) and K e^G (K-major [c x j]): 8 tokens = one 16-byte chunk
-            *reinterpret_cast<uint4 *>(sm + OFF_QG + sw128(c, rg * 16)) =
-                make_uint4(pack_bf16(qg[0], qg[1]), pack_bf16(qg[2], qg[3]), pack_bf16(qg[4], qg[5]),
-                           pack_bf16(qg[6], qg[7]));
-            *reinterpret_cast<uint4 *>(sm + OFF_KG + sw128(c, rg * 16)) =
-                make_uint4(pack_bf16(kg[0], kg[1]), pack_bf16(kg[2], kg[3]), pack_bf16(kg[4], kg[5]),
-                           pack_bf16(kg[6], kg[7]));
-            // K^(4)^T (K-major [c x j], tf32): 8 tokens = 32 bytes
-            {
-                const uint32_t jb = (uint32_t)rg * 32u;
-                unsigned char *dst = sm + OFF_KHT + (jb >> 7) * AK_KBLK;
-                *reinterpret_cast<float4 *>(dst + sw128(c, jb & 127u)) =
-                    make_float4(to_tf32(kh[0]), to_tf32(kh[1]), to_tf32(kh[2]), to_tf32(kh[3]));
-                *reinterpret_cast<float4 *>(dst + sw128(c, (jb & 127u) + 16u)) =
-                    make_float4(to_tf32(kh[4]), to_tf32(kh[5]), to_tf32(kh[6]), to_tf32(kh[7]));
-            }
-            sync_for_mma();
+            // block barrier: the MMA issue needs every thread's operands (and the waits' outcome)
+            fence_async_smem();
+            tc_fence_before();
+            if (!__syncthreads_and(loads_ok)) { failed = true; break; }
+            tc_fence_after();
             if (ci + 1 < nchunks) note_loads(1 << pass);
             ++mma_issued;
-            if (tid == 0) {
-                // q, k, g of this pass are consumed: prefetch the next chunk's
-                if (ci + 1 < nchunks) issue_loads(ci + 1, 1 << pass);
+            if (warp == 0) {
+                // q, k, g of this pass are consumed: prefetch the next chunk's; the
+                // previous chunk's output tile is complete: store it
+                if (lane == 0) {
+                    if (ci + 1 < nchunks) issue_loads(ci + 1, 1 << pass);
+                    if (pass == 0 && o_row >= 0) store_o_tile();
+                }
+                __syncwarp();
 #pragma unroll
                 for (int bb = 0; bb < NB; ++bb) {
 #pragma unroll
@@ -470,13 +645,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         const uint32_t kb = (uint32_t)(s >> 2), koff = (uint32_t)(s & 3) * 32u;
                         const uint64_t ad = at(d_k16, OFF_KB + kb_base(bb) + kb * kb_rows(bb) * 128u + koff);
                         const uint64_t bd = at(d_k16, OFF_XT + kb * 16384u + 32u * bb * 128u + koff);
-                        mma_tf32_ss(tbase + T_DB + 32 * bb, ad, bd, id_a, (pass > 0 || s > 0) ? 1u : 0u);
+                        if (leader) mma_tf32_ss(tbase + T_DB + 32 * bb, ad, bd, id_a, (pass > 0 || s > 0) ? 1u : 0u);
                     }
                 }
-                mma_commit(bar_mma);
+                if (leader) mma_commit(bar_mma);
             }
+            if (pass == 0) o_row = -1;
         }
         if (failed) break;
+        if (tid == 0) bulk_wait_read();        // the staged output tile has been read
         if (!wait_mma()) { failed = true; break; }
 
         // ================================================= A readout: warp (lq, cq): rows j, row block b = cq
@@ -502,93 +679,117 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_before();
         __syncthreads();
 
-        // ================================================= T = (I + A_kk)^-1 in place, blocked
+        // ================================================= T = (I + A_kk)^-1, then T' = T Diag(beta) in bf16
+        // Blocked inverse of the unit lower-triangular 64x64 matrix: 16x16
+        // diagonal blocks by forward substitution, then the block merges
+        //   [[T11, 0], [T21, T22]]:  T21 = -T22 (A21 T11)
+        // for 16 -> 32 and 32 -> 64.  Each warp owns what it merges, so only one
+        // barrier (among warps 0-3) separates the two merge levels.
         {
-            // (1) 16x16 diagonal blocks by forward substitution: thread (block, column)
-            float t[16];
-            const bool act = tid < 64;
-            const int bb = tid >> 4, jj = tid & 15;
-            if (act) {
-                const float *A = scr + (16 * bb) * SCR_LD + 16 * bb;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) t[i] = (i == jj) ? 1.0f : 0.0f;
-#pragma unroll
-                for (int i = 1; i < 16; ++i) {
-                    float acc = 0.0f;
-#pragma unroll
-                    for (int m = 0; m < 15; ++m)
-                        if (m < i) acc = fmaf(A[i * SCR_LD + m], t[m], acc);
-                    if (i > jj) t[i] = -acc;
-                }
-            }
-            __syncthreads();
-            if (act) {
-                float *Tb = scr + (16 * bb) * SCR_LD + 16 * bb;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) Tb[i * SCR_LD + jj] = t[i];
-            }
-            __syncthreads();
-            // Off-diagonal blocks by block products on the warp-level tensor cores
-            // (tf32; T' only needs bf16 precision).  tile(...) returns one 16x8
-            // tile of D[dr0.., dc0..] E[er0.., ec0..] over a K-wide inner range.
             const int gq = lane >> 2, tq = lane & 3;
-            auto tile = [&](int dr0, int dc0, int er0, int ec0, int K, float (&acc)[4]) {
-                acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
+            // acc[16 x 8] += X[16 x K] Y[K x 8] on the warp-level tensor cores
+            // (tf32; T' only needs bf16 precision); ldx / ldy in floats
+            auto mma_tile = [&](float (&acc)[4], const float *X, int ldx, const float *Y, int ldy, int K) {
                 for (int k0 = 0; k0 < K; k0 += 8) {
-                    uint32_t a[4], b[2];
-                    a[0] = __float_as_uint(scr[(dr0 + gq) * SCR_LD + dc0 + k0 + tq]);
-                    a[1] = __float_as_uint(scr[(dr0 + gq + 8) * SCR_LD + dc0 + k0 + tq]);
-                    a[2] = __float_as_uint(scr[(dr0 + gq) * SCR_LD + dc0 + k0 + tq + 4]);
-                    a[3] = __float_as_uint(scr[(dr0 + gq + 8) * SCR_LD + dc0 + k0 + tq + 4]);
-                    b[0] = __float_as_uint(scr[(er0 + k0 + tq) * SCR_LD + ec0 + gq]);
-                    b[1] = __float_as_uint(scr[(er0 + k0 + tq + 4) * SCR_LD + ec0 + gq]);
-                    mma_16x8x8_tf32(acc, a, b);
+                    uint32_t a[4], bb[2];
+                    a[0] = __float_as_uint(X[gq * ldx + k0 + tq]);
+                    a[1] = __float_as_uint(X[(gq + 8) * ldx + k0 + tq]);
+                    a[2] = __float_as_uint(X[gq * ldx + k0 + tq + 4]);
+                    a[3] = __float_as_uint(X[(gq + 8) * ldx + k0 + tq + 4]);
+                    bb[0] = __float_as_uint(Y[(k0 + tq) * ldy + gq]);
+                    bb[1] = __float_as_uint(Y[(k0 + tq + 4) * ldy + gq]);
+                    mma_16x8x8_tf32(acc, a, bb);
                 }
             };
-            auto put = [&](int r0, int c0, const float (&acc)[4], float sign) {
-                scr[(r0 + gq) * SCR_LD + c0 + 2 * tq] = sign * acc[0];
-                scr[(r0 + gq) * SCR_LD + c0 + 2 * tq + 1] = sign * acc[1];
-                scr[(r0 + gq + 8) * SCR_LD + c0 + 2 * tq] = sign * acc[2];
-                scr[(r0 + gq + 8) * SCR_LD + c0 + 2 * tq + 1] = sign * acc[3];
+            // store a 16x8 accumulator tile (times `sign`) at D (leading dimension ld)
+            auto put_tile = [&](float *D, int ld, const float (&acc)[4], float sign) {
+                *reinterpret_cast<float2 *>(D + gq * ld + 2 * tq) = make_float2(sign * acc[0], sign * acc[1]);
+                *reinterpret_cast<float2 *>(D + (gq + 8) * ld + 2 * tq) = make_float2(sign * acc[2], sign * acc[3]);
             };
-            // (2) 16 -> 32 for the pairs (0,1), (2,3): T10 = -T11 (A10 T00); warps 0-3
-            {
-                const int o0 = 32 * (warp >> 1), n0 = o0 + 8 * (warp & 1);
-                float acc[4];
-                if (warp < 4) tile(o0 + 16, o0, o0, n0, 16, acc);
-                __syncthreads();
-                if (warp < 4) put(o0 + 16, n0, acc, 1.0f);
-                __syncthreads();
-                if (warp < 4) tile(o0 + 16, o0 + 16, o0 + 16, n0, 16, acc);
-                __syncthreads();
-                if (warp < 4) put(o0 + 16, n0, acc, -1.0f);
-                __syncthreads();
-            }
-            // (3) 32 -> 64: T[32:, :32] = -T[32:, 32:] (A[32:, :32] T[:32, :32]); warps 0-7
-            {
-                const int r0 = 32 + 16 * (warp >> 2), n0 = 8 * (warp & 3);
-                float acc[4];
-                if (warp < 8) tile(r0, 0, 0, n0, 32, acc);
-                __syncthreads();
-                if (warp < 8) put(r0, n0, acc, 1.0f);
-                __syncthreads();
-                if (warp < 8) tile(r0, 32, 32, n0, 32, acc);
-                __syncthreads();
-                if (warp < 8) put(r0, n0, acc, -1.0f);
-                __syncthreads();
-            }
-            // (4) T' = T Diag(beta) as bf16, K-major [i x j], zero above the diagonal; 8 per thread
-            {
-                const int i = tid >> 3, j0 = (tid & 7) * 8;
-                uint32_t pk[4];
+            if (warp < 2) {
+                const int o = 32 * warp;                       // blocks o/16 and o/16 + 1
+                {   // diagonal blocks: lane = (block, column jj)
+                    const int d0 = o + 16 * (lane >> 4), jj = lane & 15;
+                    const float *A = scr + d0 * SCR_LD + d0;
+                    float t[16];
 #pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                    const int j = j0 + e;
-                    const float a = j <= i ? scr[i * SCR_LD + j] * s_beta[j] : 0.0f;
-                    const float a2 = j + 1 <= i ? scr[i * SCR_LD + j + 1] * s_beta[j + 1] : 0.0f;
-                    pk[e / 2] = pack_bf16(a, a2);
+                    for (int i = 0; i < 16; ++i) t[i] = (i == jj) ? 1.0f : 0.0f;
+#pragma unroll
+                    for (int i = 1; i < 16; ++i) {
+                        float acc = 0.0f;
+#pragma unroll
+                        for (int m = 0; m < 15; ++m)
+                            if (m < i) acc = fmaf(A[i * SCR_LD + m], t[m], acc);
+                        if (i > jj) t[i] = -acc;
+                    }
+                    __syncwarp();
+                    float *Tb = scr + d0 * SCR_LD + d0;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) Tb[i * SCR_LD + jj] = t[i];
+                    __syncwarp();
                 }
-                *reinterpret_cast<uint4 *>(sm + OFF_TP + sw128(i, j0 * 2)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                // 16 -> 32: X = A[o+16.., o..] T[o.., o..] over A's block, then T21 = -T22 X
+                float x[2][4];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    x[nt][0] = x[nt][1] = x[nt][2] = x[nt][3] = 0.0f;
+                    mma_tile(x[nt], scr + (o + 16) * SCR_LD + o, SCR_LD, scr + o * SCR_LD + o + 8 * nt, SCR_LD, 16);
+                }
+                float *blk21 = scr + (o + 16) * SCR_LD + o;
+                __syncwarp();
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) put_tile(blk21 + 8 * nt, SCR_LD, x[nt], 1.0f);
+                __syncwarp();
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    x[nt][0] = x[nt][1] = x[nt][2] = x[nt][3] = 0.0f;
+                    mma_tile(x[nt], scr + (o + 16) * SCR_LD + o + 16, SCR_LD, blk21 + 8 * nt, SCR_LD, 16);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) put_tile(blk21 + 8 * nt, SCR_LD, x[nt], -1.0f);
+                __syncwarp();
+                // T' rows o..o+31 (lane = row): columns o..o+31 from T, the upper 32 zero;
+                // rows 32-63, columns 0-31 are written by the 32 -> 64 step
+                const int i = o + lane;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const int j0 = 8 * ch;
+                    if (warp == 1 && j0 < 32) continue;
+                    uint32_t pk[4] = {0u, 0u, 0u, 0u};
+                    if (j0 >= o && j0 < o + 32) {
+#pragma unroll
+                        for (int e = 0; e < 8; e += 2)
+                            pk[e / 2] = pack_bf16(scr[i * SCR_LD + j0 + e] * s_beta[j0 + e],
+                                                  scr[i * SCR_LD + j0 + e + 1] * s_beta[j0 + e + 1]);
+                    }
+                    *reinterpret_cast<uint4 *>(sm + OFF_TP + sw128(i, j0 * 2)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+            if (warp < 4) {
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                // 32 -> 64 for columns 8 warp .. 8 warp + 7:
+                //   X = A[32:64, 0:32] T[0:32, cols],  T[32:64, cols] = -T[32:64, 32:64] X
+                float *xs = reinterpret_cast<float *>(sm + OFF_XS) + warp * 32 * XS_LD;
+                const int n0 = 8 * warp;
+                float x[2][4];
+#pragma unroll
+                for (int rt = 0; rt < 2; ++rt) {
+                    x[rt][0] = x[rt][1] = x[rt][2] = x[rt][3] = 0.0f;
+                    mma_tile(x[rt], scr + (32 + 16 * rt) * SCR_LD, SCR_LD, scr + n0, SCR_LD, 32);
+                    put_tile(xs + 16 * rt * XS_LD, XS_LD, x[rt], 1.0f);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int rt = 0; rt < 2; ++rt) {
+                    x[rt][0] = x[rt][1] = x[rt][2] = x[rt][3] = 0.0f;
+                    mma_tile(x[rt], scr + (32 + 16 * rt) * SCR_LD + 32, SCR_LD, xs, XS_LD, 32);
+                    const int j = n0 + 2 * tq;
+                    const float b0 = -s_beta[j], b1 = -s_beta[j + 1];
+                    const int i0 = 32 + 16 * rt + gq;
+                    *reinterpret_cast<uint32_t *>(sm + OFF_TP + sw128(i0, 2 * j)) = pack_bf16(x[rt][0] * b0, x[rt][1] * b1);
+                    *reinterpret_cast<uint32_t *>(sm + OFF_TP + sw128(i0 + 8, 2 * j)) = pack_bf16(x[rt][2] * b0, x[rt][3] * b1);
+                }
             }
         }
         sync_for_mma();
@@ -597,14 +798,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!wait_all(bar_v, ld_par)) { failed = true; break; }
         ++v_done;
         ++mma_issued;
-        if (tid == 0) {
+        if (warp == 0) {
 #pragma unroll
             for (int s = 0; s < 4; ++s) {          // K = 64 tokens in steps of 16
                 const uint64_t bd = at(d_k16, OFF_TP + 32u * s);
-                mma_bf16_ss(tbase + T_W, at(d_k16, OFF_KG + 32u * s), bd, id_w, s > 0);
-                mma_bf16_ss(tbase + T_U, at(d_mnv, OFF_V + 2048u * s), bd, id_u, s > 0);
+                if (leader) mma_bf16_ss(tbase + T_W, at(d_k16, OFF_KG + 32u * s), bd, id_w, s > 0);
+                if (leader) mma_bf16_ss(tbase + T_U, at(d_mnv, OFF_V + 2048u * s), bd, id_u, s > 0);
             }
-            mma_commit(bar_mma);
+            if (leader) mma_commit(bar_mma);
         }
         if (!wait_mma()) { failed = true; break; }
         if (ci + 1 < nchunks) {                      // v consumed: prefetch the next chunk's
@@ -627,11 +828,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
         // ================================================= P^T = S^T W^T, O1^T = S^T (Q e^G)^T (bf16, A from TMEM)
         ++mma_issued;
-        if (tid == 0) {
+        if (warp == 0) {
 #pragma unroll
             for (int s = 0; s < 8; ++s)            // K = 128 key channels in steps of 16
-                mma_bf16_ts(tbase + T_P, tbase + T_S + 8u * s, at(d_wq, OFF_W + 2048u * s), id_1, s > 0);
-            mma_commit(bar_mma);
+                if (leader) mma_bf16_ts(tbase + T_P, tbase + T_S + 8u * s, at(d_wq, OFF_W + 2048u * s), id_1, s > 0);
+            if (leader) mma_commit(bar_mma);
         }
         if (!wait_mma()) { failed = true; break; }
 
@@ -653,18 +854,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
         // ================================================= O2^T = Vn^T A_qk^T, dS^T = Vn^T K^(4) (tf32)
         ++mma_issued;
-        if (tid == 0) {
+        if (warp == 0) {
 #pragma unroll
             for (int s = 0; s < 8; ++s) {          // K = 64 tokens in steps of 8
                 const uint32_t kb = (uint32_t)(s >> 2), koff = (uint32_t)(s & 3) * 32u;
-                mma_tf32_ts(tbase + T_O2, tbase + T_P + 8u * s, at(d_k16, OFF_AK + kb * AK_KBLK + koff), id_2, s > 0);
+                if (leader) mma_tf32_ts(tbase + T_O2, tbase + T_P + 8u * s, at(d_k16, OFF_AK + kb * AK_KBLK + koff), id_2, s > 0);
             }
-            mma_commit(bar_mma);
+            if (leader) mma_commit(bar_mma);
         }
         if (!wait_mma()) { failed = true; break; }
 
         // ================================================= state update and outputs
+        // (no block barrier after this phase: the next chunk's prep touches none
+        // of what it reads -- gamma is double-buffered -- and the next MMA that
+        // overwrites these TMEM columns is issued after a block barrier)
         {
+            const float *gam = s_gam + (ci & 1) * D;
 #pragma unroll
             for (int hq = 0; hq < 2; ++hq) {       // dS^T rows c in [32 cq + 16 hq, +16)
                 uint32_t rd[16];
@@ -672,39 +877,57 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    S[hq * 16 + e] = fmaf(s_gam[cq * 32 + hq * 16 + e], S[hq * 16 + e], __uint_as_float(rd[e]));
+                    S[hq * 16 + e] = fmaf(gam[cq * 32 + hq * 16 + e], S[hq * 16 + e], __uint_as_float(rd[e]));
             }
             store_state_bf16();
             uint32_t r1[16], r2[16];
             tmem_ld16(tbase + lane_base + T_O1 + cq * 16, r1);
             tmem_ld16(tbase + lane_base + T_O2 + cq * 16, r2);
             tmem_wait_ld();
+            if (store_o) {
+                float x[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int i = cq * 16 + e;
-                if (store_o && i < L) {
-                    const int64_t off = ((t0 + i) * H + hh) * D + vlane;
-                    float x = p.scale * (__uint_as_float(r1[e]) + __uint_as_float(r2[e]));
-                    if (gate) x *= sigmoidf(__bfloat162float(gate[off]));
-                    o[off] = __float2bfloat16_rn(x);
+                for (int e = 0; e < 16; ++e) x[e] = p.scale * (__uint_as_float(r1[e]) + __uint_as_float(r2[e]));
+                const int nv = min(16, L - cq * 16);   // tokens of this thread inside the chunk
+                const int64_t off0 = ((t0 + cq * 16) * H + hh) * D + vlane;
+                if (gate) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        if (e < nv) x[e] *= sigmoid_fast(__bfloat162float(gate[off0 + (int64_t)e * H * D]));
+                }
+                if (L == C) {
+                    // full chunk: into the staging tile, stored by TMA after the next block barrier
+                    unsigned char *ost = sm + OFF_OST + (uint32_t)(vlane >> 6) * AK_KBLK;
+                    const uint32_t vb = (uint32_t)(vlane & 63) * 2u;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        *reinterpret_cast<__nv_bfloat16 *>(ost + sw128((uint32_t)(cq * 16 + e), vb)) = __float2bfloat16_rn(x[e]);
+                    o_row = t0;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        if (e < nv) o[off0 + (int64_t)e * H * D] = __float2bfloat16_rn(x[e]);
                 }
             }
         }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
     }
 
     if (!failed && S_outp) {
 #pragma unroll
         for (int r = 0; r < 32; ++r) S_outp[(cq * 32 + r) * D + vlane] = S[r];
     }
+    if (!failed && o_row >= 0) {           // the last chunk's output tile
+        fence_async_smem();
+        __syncthreads();
+        if (tid == 0) store_o_tile();
+    }
+    if (tid == 0) bulk_wait_all();         // every TMA store has completed
     if (failed && tid == 0) {
         // drain what is still in flight (bounded) before TMEM and shared memory go away
-        for (int pp = 0; pp < 2; ++pp)
-            for (uint32_t k2 = qkg_done[pp]; k2 < qkg_issued[pp]; ++k2) mbar_wait(&bar_qkg[pp], k2 & 1u, 1u << 20);
-        for (uint32_t k2 = v_done; k2 < v_issued; ++k2) mbar_wait(bar_v, k2 & 1u, 1u << 20);
-        for (uint32_t k2 = mma_phase; k2 < mma_issued; ++k2) mbar_wait(bar_mma, k2 & 1u, 1u << 20);
+        drain_phases(&bar_qkg[0], qkg_done[0], qkg_issued[0]);
+        drain_phases(&bar_qkg[1], qkg_done[1], qkg_issued[1]);
+        drain_phases(bar_v, v_done, v_issued);
+        drain_phases(bar_mma, mma_phase, mma_issued);
     }
     tc_fence_before();
     __syncthreads();

@@ -243,11 +243,12 @@ bool encode_bf16_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t 
 }
 
 // The tensor-core prefill covers bf16 I/O with dk = dv = 128 and 16-byte
-// aligned inputs; chunk = 16 and every other shape use the CUDA-core kernel.
+// aligned q, k, v, g and o (all moved by TMA); chunk = 16 and every other
+// shape use the CUDA-core kernel.
 bool tc_path_applies(const kda_fwd_desc &d, const void *q, const void *k, const void *v,
-                     const void *g) {
+                     const void *g, const void *o) {
     if (!tc_shape(d)) return false;
-    for (const void *ptr : {q, k, v, g})
+    for (const void *ptr : {q, k, v, g, o})
         if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return false;
     return true;
 }
@@ -264,10 +265,11 @@ cudaError_t launch_tc(const kda_fwd_desc &d, const void *q, const void *k, const
 cudaError_t launch_tc_units(const kda_fwd_desc &d, const void *q, const void *k, const void *v,
                             const void *g, const kda::tck::TcParams &p, int64_t blocks,
                             cudaStream_t stream) {
-    CUtensorMap tq, tk, tg, tv;
+    CUtensorMap tq, tk, tg, tv, to;
     const uint64_t rows = (uint64_t)d.total_tokens, cols = (uint64_t)d.num_heads * 128u;
     if (!encode_bf16_2d(&tq, q, rows, cols) || !encode_bf16_2d(&tk, k, rows, cols) ||
-        !encode_bf16_2d(&tg, g, rows, cols) || !encode_bf16_2d(&tv, v, rows, cols))
+        !encode_bf16_2d(&tg, g, rows, cols) || !encode_bf16_2d(&tv, v, rows, cols) ||
+        !encode_bf16_2d(&to, p.o, rows, cols))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(kda::tck::chunk_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -276,7 +278,7 @@ cudaError_t launch_tc_units(const kda_fwd_desc &d, const void *q, const void *k,
     if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
     if (blocks == 0) return cudaSuccess;
     kda::tck::chunk_tc_kernel<<<(unsigned)blocks, kda::tck::NT, kda::tck::SMEM_ALLOC, stream>>>(
-        tq, tk, tg, tv, p);
+        tq, tk, tg, tv, to, p);
     return cudaGetLastError();
 }
 
@@ -286,7 +288,7 @@ cudaError_t launch_prefill(const kda_fwd_desc &d, const void *q, const void *k, 
                            const void *g, const void *beta, const float *S0,
                            const int32_t *cu_seqlens, const int32_t *seq_order, const void *gate,
                            void *o, float *S_T, cudaStream_t stream) {
-    if (tc_path_applies(d, q, k, v, g)) {
+    if (tc_path_applies(d, q, k, v, g, o)) {
         kda::tck::TcParams tp{beta, gate, S0, cu_seqlens, seq_order, o, S_T, d.num_heads, d.scale,
                               d.g_floor, nullptr};
         return launch_tc(d, q, k, v, g, tp, stream);
@@ -436,7 +438,7 @@ kda_status kda_chunk_fwd(const kda_fwd_desc *desc, const void *q, const void *k,
     }
 
     const SegPlan pl = plan_segments(d, cu_seqlens_host);
-    if (pl.active && tc_path_applies(d, q, k, v, g)) {
+    if (pl.active && tc_path_applies(d, q, k, v, g, o)) {
         const cudaError_t e = launch_split(d, pl, cu_seqlens_host, q, k, v, g, beta, S0, gate, o, S_T,
                                            static_cast<unsigned char *>(workspace), stream);
         return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;

@@ -42,14 +42,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete; gives up after
-// `max_iters` polls (each try_wait itself blocks for a bounded time slice).
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
-                                          uint32_t max_iters = (1u << 22)) {
+// The polling loop of mbar_wait, kept out of line: waits are many and their
+// slow path is rare, so inlining it would only grow the kernels' code.
+__device__ __noinline__ bool mbar_wait_poll(uint64_t *bar, uint32_t parity, uint32_t max_iters) {
     for (uint32_t i = 0; i < max_iters; ++i)
         if (mbar_try_wait(bar, parity)) return true;
     raise_error(ERR_TIMEOUT);
     return false;
+}
+
+// Waits for the phase with the given parity to complete; gives up after
+// `max_iters` polls (each try_wait itself blocks for a bounded time slice).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
+                                          uint32_t max_iters = (1u << 22)) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_poll(bar, parity, max_iters);
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
@@ -150,6 +157,20 @@ __device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}"
         ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
+// One lane of a converged warp, the same on every call with all lanes
+// active.  MMA issue runs warp-wide (descriptor arithmetic stays uniform)
+// with only the elected lane executing the tcgen05 instructions; this keeps
+// the issue sequence short in both instructions and code size.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t e;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(e));
+    return e != 0;
+}
+
 // Arrive on `bar` once every MMA this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
