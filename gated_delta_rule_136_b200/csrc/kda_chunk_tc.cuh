@@ -11,15 +11,16 @@
 //                                                Fig. 3)
 //   K^(b)_j = Kbar_j e^{r_b - r_{b(j)}}  for b(j) <= b   ( = k_j e^{r_b - G_j} )
 //   A_qk[i,j] = (q_i Gt_i) . K^(b(i))_j   (j <= i),   A_kk[i,j] = beta_i (k_i Gt_i) . K^(b(i))_j  (j < i)
-//   T' = (I + A_kk)^-1 Diag(beta);  W = T' (k Gt e^{r_b}),  U = T' V
-//   Vn = U - W S;   O = scale ((q Gt e^{r_b}) S + A_qk Vn) [* sigmoid(z)]
+//   T' = (I + A_kk)^-1 Diag(beta)
+//   Vn = T' (V - (k Gt e^{r_b}) S)   (= U - W S of the WY form, U = T' V, W = T' K e^G)
+//   O  = scale ((q Gt e^{r_b}) S + A_qk Vn) [* sigmoid(z)]
 //   S  = Diag(e^{r_4}) S + K^(4)^T Vn
 // which equals the token recurrence in real arithmetic (the intra-chunk part
 // in parallel, then the state carried to the next chunk: fupanwang.com digest,
 // section 基础设施, FlashKDA).
 //
 // Precision: the products the outputs are sensitive to run in tf32 (A_qk /
-// A_kk operands, A_qk Vn, K^(4)^T Vn); W S, (Q e^G) S, W and U run in bf16.
+// A_kk operands, T' Z, A_qk Vn, K^(4)^T Vn); (K e^G) S and (Q e^G) S run in bf16.
 //
 // Orientation: the state products are computed transposed so that the value
 // channel v is the TMEM lane (M = 128): S^T and Vn^T live in TMEM as the A
@@ -28,8 +29,9 @@
 // One CTA (512 threads) carries one (sequence, head) unit; its phases per
 // chunk run in order:
 //   prep (2 passes of 64 key channels; TMA tiles of q, k, g)  ->  A MMAs (tf32)
-//   -> A readout + block-triangular inverse (CUDA cores)  ->  W, U MMAs (bf16)
-//   -> W readout  ->  W S, (Q e^G) S MMAs  ->  Vn  ->  A_qk Vn, K^T Vn MMAs (tf32)
+//   -> A readout -> block-triangular inverse (warps 0-3), while warps 4-15 form
+//      Z = V - (K e^G) S from a (Q e^G | K e^G) S MMA issued after the readout
+//   -> Vn = T' Z MMA (tf32)  ->  A_qk Vn, K^T Vn MMAs (tf32)
 //   -> state update + output epilogue.
 // The next chunk's q, k, g, v tiles are loaded by TMA while the current
 // chunk's later phases run.
@@ -62,10 +64,9 @@ constexpr uint32_t OFF_KB = OFF_INTRA + 32768;     // K^(b), b = 0..3, packed ro
 //   after the A MMAs:
 constexpr uint32_t OFF_SCR = OFF_INTRA;            // A_kk -> T, fp32 [64][68]
 constexpr uint32_t SCR_LD = 68;                    // 16-byte aligned rows
-constexpr uint32_t OFF_TP = OFF_INTRA + 17408;     // T' bf16 K-major [64 i x 64 j]: 8 KB
-constexpr uint32_t OFF_XS = OFF_INTRA + 25600;     // inverse scratch: 4 warps x [32 x 8] fp32: 4 KB
+constexpr uint32_t OFF_TP = OFF_INTRA + 17408;     // T' tf32 K-major [64 i x 64 j]: 2 x 8 KB
+constexpr uint32_t OFF_XS = OFF_INTRA + 33792;     // inverse scratch: 4 warps x [32 x 8] fp32: 4 KB
 constexpr uint32_t XS_LD = 8;
-constexpr uint32_t OFF_W = OFF_INTRA + 41984;      // W bf16 MN-major [128 c x 64 j]: 16 KB
 constexpr uint32_t OFF_QG = OFF_INTRA + 73728;     // Q e^G bf16 MN-major [128 c x 64 i]: 16 KB
 constexpr uint32_t OFF_KG = OFF_QG + 16384;        // K e^G bf16 K-major [128 c x 64 j]: 16 KB
 // B operand of the second state MMA: rows 0-63 = A_qk [i x j], rows 64-191 =
@@ -81,9 +82,9 @@ constexpr uint32_t OFF_KHT = OFF_AK + 64u * 128u;  // + kb * AK_KBLK + row * 128
 constexpr uint32_t OFF_SMALL = OFF_AK + 2u * AK_KBLK;  // beta[64], gamma[2][128], barriers, tmem base
 constexpr uint32_t SMEM_BYTES = OFF_SMALL + 2048;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024; // slack for aligning the base
-static_assert(OFF_W + 16384 <= OFF_INTRA + 73728, "post-MMA tiles fit the intra region");
-static_assert(OFF_TP + 8192 <= OFF_XS && OFF_XS + 4096 <= OFF_W, "inverse scratch between T' and W");
-static_assert(OFF_QG - OFF_W < (1u << 18) && (OFF_QG - OFF_W) % 16 == 0, "W | Q e^G as one MN-major operand");
+static_assert(OFF_TP % 1024 == 0 && OFF_TP + 16384 <= OFF_XS && OFF_XS + 4096 <= OFF_INTRA + 73728,
+              "post-MMA tiles fit the intra region");
+static_assert((OFF_KG - OFF_QG) % 16 == 0, "Q e^G | K e^G as one MN-major operand");
 static_assert(OFF_KB + 40960 <= OFF_INTRA + 73728, "intra tiles fit");
 static_assert(SMEM_ALLOC <= 232448, "fits in 227 KB");
 
@@ -100,11 +101,10 @@ static_assert(kb_base(3) + 128u * 64u + 64u * 128u <= 40960u, "K^(b) reads stay 
 // ---- TMEM columns
 constexpr uint32_t T_DB = 0;      // A MMAs: 4 x 32 columns (M = 64 layout)
 constexpr uint32_t T_O2 = 0;      // (A_qk Vn)^T   [v x i]   } one MMA (N = 192), after the
-constexpr uint32_t T_DS = 64;     // dS^T          [v x c]   } A readout and the Vn step
-constexpr uint32_t T_U = 128;     // U^T     [v x i]
-constexpr uint32_t T_W = 192;     // W^T     [c x i]
-constexpr uint32_t T_P = 256;     // P^T = (W S)^T, then Vn^T (tf32 A operand)  } one MMA
-constexpr uint32_t T_O1 = 320;    // ((Q e^G) S)^T                              } (N = 128)
+constexpr uint32_t T_DS = 64;     // dS^T          [v x c]   } A readout and Vn
+constexpr uint32_t T_VN = 192;    // Vn^T = Z^T T'^T, then its tf32 copy (A operand)
+constexpr uint32_t T_O1 = 256;    // ((Q e^G) S)^T  [v x i]  } one MMA (N = 128)
+constexpr uint32_t T_Z = 320;     // ((K e^G) S)^T  [v x j], then Z^T (tf32 A operand)
 constexpr uint32_t T_S = 384;     // S^T bf16 A operand (2 per column)
 constexpr uint32_t TMEM_COLS = 512;
 
@@ -263,6 +263,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t *bar_qkg = reinterpret_cast<uint64_t *>(sm + OFF_SMALL + 1280);  // [2]
     uint64_t *bar_v = bar_qkg + 2;
     uint64_t *bar_mma = bar_qkg + 3;
+    uint64_t *bar_y = bar_qkg + 4;       // the (Q e^G | K e^G) S MMA
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + OFF_SMALL + 1344);
     float *scr = reinterpret_cast<float *>(sm + OFF_SCR);
 
@@ -341,6 +342,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(&bar_qkg[1], 1);
         mbar_init(bar_v, 1);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_y, 1);
         mbar_fence_init();
     }
     tc_fence_before();
@@ -398,7 +400,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         note_loads(7);
     }
 
-    uint32_t mma_phase = 0, mma_issued = 0;
+    uint32_t mma_phase = 0, mma_issued = 0, y_phase = 0, y_issued = 0;
     bool failed = false;
     // first token of the output tile waiting in the staging area (-1: none);
     // tid 0 issues its TMA store after the next block barrier
@@ -430,22 +432,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
         return ok;
     };
-    auto sync_for_mma = [&]() {            // generic smem / TMEM writes -> MMA issue
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-    };
 
     // MMA descriptors that do not depend on the chunk (start addresses advance per K-step)
     const uint32_t id_a = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 64, 32);
-    const uint32_t id_w = instr_desc(FMT_BF16, K_MAJOR, K_MAJOR, 128, 64);
-    const uint32_t id_u = instr_desc(FMT_BF16, MN_MAJOR, K_MAJOR, 128, 64);
     const uint32_t id_1 = instr_desc(FMT_BF16, K_MAJOR, MN_MAJOR, 128, 128);
+    const uint32_t id_vn = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 128, 64);
     const uint32_t id_2 = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 128, 192);
     const uint64_t d_k16 = smem_desc_sw128(smb, 16, 1024);          // K-major template
-    const uint64_t d_mnv = smem_desc_sw128(smb, 8192, 1024);        // v: MN blocks 8 KB apart
-    const uint64_t d_wq = smem_desc_sw128(smb, OFF_QG - OFF_W, 1024);  // [W | Q e^G] MN-major
+    const uint64_t d_qk = smem_desc_sw128(smb, OFF_KG - OFF_QG, 1024);  // [Q e^G | K e^G] MN-major
     auto at = [](uint64_t tmpl, uint32_t byte_off) -> uint64_t {     // same descriptor, moved start
         return tmpl + (uint64_t)(byte_off >> 4);
     };
@@ -649,6 +643,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
                 if (leader) mma_commit(bar_mma);
+                // [O1 | Y]^T = S^T [Q e^G | K e^G]^T (bf16, A = S^T from TMEM), this pass's
+                // 64 key channels; it runs behind the A MMAs, off the critical path
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const uint32_t ks = (uint32_t)(4 * pass + s);   // K = 128 key channels in steps of 16
+                    if (leader) mma_bf16_ts(tbase + T_O1, tbase + T_S + 8u * ks, at(d_qk, OFF_QG + 2048u * ks), id_1, ks > 0);
+                }
+                if (pass == 1 && leader) mma_commit(bar_y);
             }
             if (pass == 0) o_row = -1;
         }
@@ -678,8 +680,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         tc_fence_before();
         __syncthreads();
+        tc_fence_after();
 
-        // ================================================= T = (I + A_kk)^-1, then T' = T Diag(beta) in bf16
+        bool z_ok = true;
+        ++y_issued;
+        // ================================================= T = (I + A_kk)^-1, then T' = T Diag(beta) (warps 0-3)
+        // and, concurrently, Z = V - (K e^G) S (warps 4-15)
         // Blocked inverse of the unit lower-triangular 64x64 matrix: 16x16
         // diagonal blocks by forward substitution, then the block merges
         //   [[T11, 0], [T21, T22]]:  T21 = -T22 (A21 T11)
@@ -749,25 +755,28 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) put_tile(blk21 + 8 * nt, SCR_LD, x[nt], -1.0f);
                 __syncwarp();
-                // T' rows o..o+31 (lane = row): columns o..o+31 from T, the upper 32 zero;
+                // T' rows o..o+31 (lane = row), tf32 K-major [i x j] in two 32-column
+                // K-blocks: columns o..o+31 from T, the other 32 zero for rows 0-31;
                 // rows 32-63, columns 0-31 are written by the 32 -> 64 step
                 const int i = o + lane;
+                unsigned char *tpr = sm + OFF_TP + (uint32_t)warp * 8192u;   // K-block of columns o..o+31
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const int j0 = 8 * ch;
-                    if (warp == 1 && j0 < 32) continue;
-                    uint32_t pk[4] = {0u, 0u, 0u, 0u};
-                    if (j0 >= o && j0 < o + 32) {
+                for (int c4 = 0; c4 < 8; ++c4) {
+                    const int j0 = o + 4 * c4;
+                    const float4 t4 = *reinterpret_cast<const float4 *>(scr + i * SCR_LD + j0);
+                    const float4 b4 = *reinterpret_cast<const float4 *>(s_beta + j0);
+                    *reinterpret_cast<float4 *>(tpr + sw128((uint32_t)i, (uint32_t)c4 * 16u)) =
+                        make_float4(t4.x * b4.x, t4.y * b4.y, t4.z * b4.z, t4.w * b4.w);
+                }
+                if (warp == 0) {
 #pragma unroll
-                        for (int e = 0; e < 8; e += 2)
-                            pk[e / 2] = pack_bf16(scr[i * SCR_LD + j0 + e] * s_beta[j0 + e],
-                                                  scr[i * SCR_LD + j0 + e + 1] * s_beta[j0 + e + 1]);
-                    }
-                    *reinterpret_cast<uint4 *>(sm + OFF_TP + sw128(i, j0 * 2)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    for (int c4 = 0; c4 < 8; ++c4)
+                        *reinterpret_cast<float4 *>(sm + OFF_TP + 8192u + sw128((uint32_t)i, (uint32_t)c4 * 16u)) =
+                            make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                 }
             }
             if (warp < 4) {
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                asm volatile("bar.sync 1, 128;" ::: "memory");   // warps 0-3 only
                 // 32 -> 64 for columns 8 warp .. 8 warp + 7:
                 //   X = A[32:64, 0:32] T[0:32, cols],  T[32:64, cols] = -T[32:64, 32:64] X
                 float *xs = reinterpret_cast<float *>(sm + OFF_XS) + warp * 32 * XS_LD;
@@ -784,68 +793,67 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int rt = 0; rt < 2; ++rt) {
                     x[rt][0] = x[rt][1] = x[rt][2] = x[rt][3] = 0.0f;
                     mma_tile(x[rt], scr + (32 + 16 * rt) * SCR_LD + 32, SCR_LD, xs, XS_LD, 32);
-                    const int j = n0 + 2 * tq;
+                    const int j = n0 + 2 * tq;            // columns 0-31: K-block 0
                     const float b0 = -s_beta[j], b1 = -s_beta[j + 1];
                     const int i0 = 32 + 16 * rt + gq;
-                    *reinterpret_cast<uint32_t *>(sm + OFF_TP + sw128(i0, 2 * j)) = pack_bf16(x[rt][0] * b0, x[rt][1] * b1);
-                    *reinterpret_cast<uint32_t *>(sm + OFF_TP + sw128(i0 + 8, 2 * j)) = pack_bf16(x[rt][2] * b0, x[rt][3] * b1);
+                    *reinterpret_cast<float2 *>(sm + OFF_TP + sw128((uint32_t)i0, (uint32_t)j * 4u)) =
+                        make_float2(x[rt][0] * b0, x[rt][1] * b1);
+                    *reinterpret_cast<float2 *>(sm + OFF_TP + sw128((uint32_t)i0 + 8u, (uint32_t)j * 4u)) =
+                        make_float2(x[rt][2] * b0, x[rt][3] * b1);
                 }
             }
-        }
-        sync_for_mma();
-
-        // ================================================= W^T = (K e^G)^T T'^T, U^T = V^T T'^T (bf16)
-        if (!wait_all(bar_v, ld_par)) { failed = true; break; }
-        ++v_done;
-        ++mma_issued;
-        if (warp == 0) {
+            if (warp >= 4) {
+                // Z^T[v, j] = V[j, v] - Y^T[v, j], tf32, in place of Y^T: lane quarter
+                // w % 4; the three warps of a quarter share its four 16-token groups
+                z_ok = mbar_wait(bar_v, ld_par) && mbar_wait(bar_y, y_phase & 1);
+                tc_fence_after();
+                const unsigned char *vt = sm + OFF_V + (uint32_t)(vlane >> 6) * 8192u;
+                const uint32_t vb = (uint32_t)(vlane & 63) * 2u;
+                for (int grp = (warp >> 2) - 1; grp < 4; grp += 3) {
+                    uint32_t ry[16];
+                    tmem_ld16(tbase + lane_base + T_Z + 16u * grp, ry);
+                    tmem_wait_ld();
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {          // K = 64 tokens in steps of 16
-                const uint64_t bd = at(d_k16, OFF_TP + 32u * s);
-                if (leader) mma_bf16_ss(tbase + T_W, at(d_k16, OFF_KG + 32u * s), bd, id_w, s > 0);
-                if (leader) mma_bf16_ss(tbase + T_U, at(d_mnv, OFF_V + 2048u * s), bd, id_u, s > 0);
+                    for (int e = 0; e < 16; ++e) {
+                        const float vv = zero_v ? 0.0f
+                                                : __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
+                                                      vt + sw128((uint32_t)(16 * grp + e), vb)));
+                        ry[e] = __float_as_uint(to_tf32(vv - __uint_as_float(ry[e])));
+                    }
+                    tmem_st16(tbase + lane_base + T_Z + 16u * grp, ry);
+                }
+                tmem_wait_st();
             }
-            if (leader) mma_commit(bar_mma);
         }
-        if (!wait_mma()) { failed = true; break; }
+        ++v_done;
+        ++y_phase;
+        fence_async_smem();
+        tc_fence_before();
+        if (!__syncthreads_and(z_ok)) { failed = true; break; }
+        tc_fence_after();
         if (ci + 1 < nchunks) {                      // v consumed: prefetch the next chunk's
             if (tid == 0) issue_loads(ci + 1, 4);
             note_loads(4);
         }
 
-        // ================================================= W readout: lane c, tokens j in [16 cq, 16 cq + 16)
-        {
-            uint32_t rw[16];
-            tmem_ld16(tbase + lane_base + T_W + cq * 16, rw);
-            tmem_wait_ld();
-            uint32_t pk[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(__uint_as_float(rw[2 * e]), __uint_as_float(rw[2 * e + 1]));
-            *reinterpret_cast<uint4 *>(sm + OFF_W + sw128(vlane, cq * 32)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            *reinterpret_cast<uint4 *>(sm + OFF_W + sw128(vlane, cq * 32 + 16)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
-        sync_for_mma();
-
-        // ================================================= P^T = S^T W^T, O1^T = S^T (Q e^G)^T (bf16, A from TMEM)
+        // ================================================= Vn^T = Z^T T'^T (tf32, A from TMEM), then rounded to tf32
         ++mma_issued;
         if (warp == 0) {
 #pragma unroll
-            for (int s = 0; s < 8; ++s)            // K = 128 key channels in steps of 16
-                if (leader) mma_bf16_ts(tbase + T_P, tbase + T_S + 8u * s, at(d_wq, OFF_W + 2048u * s), id_1, s > 0);
+            for (int s = 0; s < 8; ++s) {          // K = 64 tokens in steps of 8
+                const uint32_t kb = (uint32_t)(s >> 2), koff = (uint32_t)(s & 3) * 32u;
+                if (leader) mma_tf32_ts(tbase + T_VN, tbase + T_Z + 8u * s, at(d_k16, OFF_TP + kb * 8192u + koff), id_vn, s > 0);
+            }
             if (leader) mma_commit(bar_mma);
         }
         if (!wait_mma()) { failed = true; break; }
-
-        // ================================================= Vn^T = U^T - P^T (tf32, in place of P^T)
         {
-            uint32_t rp[16], ru[16];
-            tmem_ld16(tbase + lane_base + T_P + cq * 16, rp);
-            tmem_ld16(tbase + lane_base + T_U + cq * 16, ru);
+            uint32_t rv[16];
+            tmem_ld16(tbase + lane_base + T_VN + cq * 16, rv);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                rp[e] = __float_as_uint(to_tf32((zero_v ? 0.0f : __uint_as_float(ru[e])) - __uint_as_float(rp[e])));
-            tmem_st16(tbase + lane_base + T_P + cq * 16, rp);
+            for (int e = 0; e < 16; ++e) rv[e] = __float_as_uint(to_tf32(__uint_as_float(rv[e])));
+            tmem_st16(tbase + lane_base + T_VN + cq * 16, rv);
             tmem_wait_st();
         }
         tc_fence_before();
@@ -858,7 +866,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
             for (int s = 0; s < 8; ++s) {          // K = 64 tokens in steps of 8
                 const uint32_t kb = (uint32_t)(s >> 2), koff = (uint32_t)(s & 3) * 32u;
-                if (leader) mma_tf32_ts(tbase + T_O2, tbase + T_P + 8u * s, at(d_k16, OFF_AK + kb * AK_KBLK + koff), id_2, s > 0);
+                if (leader) mma_tf32_ts(tbase + T_O2, tbase + T_VN + 8u * s, at(d_k16, OFF_AK + kb * AK_KBLK + koff), id_2, s > 0);
             }
             if (leader) mma_commit(bar_mma);
         }
@@ -928,6 +936,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         drain_phases(&bar_qkg[1], qkg_done[1], qkg_issued[1]);
         drain_phases(bar_v, v_done, v_issued);
         drain_phases(bar_mma, mma_phase, mma_issued);
+        drain_phases(bar_y, y_phase, y_issued);
     }
     tc_fence_before();
     __syncthreads();
