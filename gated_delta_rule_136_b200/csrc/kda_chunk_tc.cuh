@@ -443,6 +443,32 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     auto at = [](uint64_t tmpl, uint32_t byte_off) -> uint64_t {     // same descriptor, moved start
         return tmpl + (uint64_t)(byte_off >> 4);
     };
+    // Warp 0: the A MMAs of blocks [b0, b1) of a prep pass (tf32, 8 K-steps of 8
+    // channels each); when the pass's last block is issued: commit, then this
+    // pass's half of [O1 | Y]^T = S^T [Q e^G | K e^G]^T (bf16, A = S^T from TMEM),
+    // which runs behind the A MMAs, off the critical path.
+    auto issue_a = [&](int pass_, int b0, int b1) {
+#pragma unroll
+        for (int bb = 0; bb < NB; ++bb) {
+            if (bb < b0 || bb >= b1) continue;
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const uint32_t kb = (uint32_t)(s >> 2), koff = (uint32_t)(s & 3) * 32u;
+                const uint64_t ad = at(d_k16, OFF_KB + kb_base(bb) + kb * kb_rows(bb) * 128u + koff);
+                const uint64_t bd = at(d_k16, OFF_XT + kb * 16384u + 32u * bb * 128u + koff);
+                if (leader) mma_tf32_ss(tbase + T_DB + 32 * bb, ad, bd, id_a, (pass_ > 0 || s > 0) ? 1u : 0u);
+            }
+        }
+        if (b1 == NB) {
+            if (leader) mma_commit(bar_mma);
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                const uint32_t ks = (uint32_t)(4 * pass_ + s);   // K = 128 key channels in steps of 16
+                if (leader) mma_bf16_ts(tbase + T_O1, tbase + T_S + 8u * ks, at(d_qk, OFF_QG + 2048u * ks), id_1, ks > 0);
+            }
+            if (pass_ == 1 && leader) mma_commit(bar_y);
+        }
+    };
 
     const float L2E = 1.4426950408889634f;
 
@@ -475,6 +501,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             uint32_t gf[2][4];                     // [tokens 32h..][block 2h + (j>>1), half j&1]
             ldsm_x4_trans(gf[0], raw + QKG_G + sw128((uint32_t)lane, (uint32_t)nt * 16u));
             ldsm_x4_trans(gf[1], raw + QKG_G + sw128((uint32_t)(32 + lane), (uint32_t)nt * 16u));
+            if (pass == 1 && warp == 0) {          // the rest of the pass-0 A MMAs
+                __syncwarp();
+                issue_a(0, 2, NB);
+                __syncwarp();
+            }
             uint32_t gi[2][4];                     // indicator g <= fb (floor not a bf16 value)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -632,25 +663,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (pass == 0 && o_row >= 0) store_o_tile();
                 }
                 __syncwarp();
-#pragma unroll
-                for (int bb = 0; bb < NB; ++bb) {
-#pragma unroll
-                    for (int s = 0; s < 8; ++s) {      // 8 tf32 K-steps of 8 channels
-                        const uint32_t kb = (uint32_t)(s >> 2), koff = (uint32_t)(s & 3) * 32u;
-                        const uint64_t ad = at(d_k16, OFF_KB + kb_base(bb) + kb * kb_rows(bb) * 128u + koff);
-                        const uint64_t bd = at(d_k16, OFF_XT + kb * 16384u + 32u * bb * 128u + koff);
-                        if (leader) mma_tf32_ss(tbase + T_DB + 32 * bb, ad, bd, id_a, (pass > 0 || s > 0) ? 1u : 0u);
-                    }
-                }
-                if (leader) mma_commit(bar_mma);
-                // [O1 | Y]^T = S^T [Q e^G | K e^G]^T (bf16, A = S^T from TMEM), this pass's
-                // 64 key channels; it runs behind the A MMAs, off the critical path
-#pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    const uint32_t ks = (uint32_t)(4 * pass + s);   // K = 128 key channels in steps of 16
-                    if (leader) mma_bf16_ts(tbase + T_O1, tbase + T_S + 8u * ks, at(d_qk, OFF_QG + 2048u * ks), id_1, ks > 0);
-                }
-                if (pass == 1 && leader) mma_commit(bar_y);
+                // pass 0: blocks 0-1 now, blocks 2-3 early in warp 0's pass-1 prep (a long
+                // run of issues stalls the issuing warp); pass 1: everything now
+                issue_a(pass, 0, pass == 0 ? 2 : NB);
             }
             if (pass == 0) o_row = -1;
         }

@@ -21,7 +21,7 @@ def _cpu(x):
     return None if x is None else x.detach().to("cpu")
 
 
-def _oracle_prefill(inp, heads=None, seqs=None):
+def _oracle_prefill(inp, heads=None, seqs=None, g_floor=-5.0):
     """Oracle on a subset of heads / sequences (units are independent)."""
     q, k, v, g, beta = (_cpu(inp[n]) for n in ("q", "k", "v", "g", "beta"))
     gate, S0 = _cpu(inp["gate"]), _cpu(inp["S0"])
@@ -40,7 +40,7 @@ def _oracle_prefill(inp, heads=None, seqs=None):
         S0 = None if S0 is None else S0[list(seqs)]
         cu = newcu
     return oracle.kda_fwd_ref(q, k, v, g, beta, cu_seqlens=np.array(cu, dtype=np.int64), S0=S0,
-                              scale=inp["scale"], gate=gate)
+                              scale=inp["scale"], gate=gate, g_floor=g_floor)
 
 
 def _all_finite(t, rows_per_slab=1 << 16):
@@ -98,6 +98,24 @@ def test_floor_stress_bf16():
                      cu_seqlens=inp["cu_seqlens"], cu_seqlens_host=inp["cu_seqlens_host"])
     o_ref, S_ref = _oracle_prefill(inp)
     _assert_close(o, S, o_ref, S_ref, torch.bfloat16, "floor stress")
+
+
+@pytest.mark.parametrize("g_floor", [-4.7, -5.45, -0.3])
+def test_floor_not_a_bf16_value(g_floor):
+    """A floor that bf16 cannot represent: the tensor-core prefill clamps with
+    the nearest bf16 below it and adds the exact remainder for every clamped
+    token, so the result must still match max(g, floor) in the oracle.  At
+    -0.3 every token is clamped; at -5.45 (the lowest floor) a third are."""
+    assert float(torch.tensor(g_floor, dtype=torch.bfloat16)) != float(np.float32(g_floor))
+    inp = inputs.prefill_inputs([300, 77], H=2, dk=128, dv=128, device=DEV, seed=7,
+                                g_mode="floor_stress", s0_std=0.02, gate=True)
+    inp["g"][::3] = -6.0
+    o, S = chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S0=inp["S0"],
+                     cu_seqlens=inp["cu_seqlens"], cu_seqlens_host=inp["cu_seqlens_host"],
+                     gate=inp["gate"], g_floor=g_floor)
+    o_ref, S_ref = _oracle_prefill(inp, g_floor=g_floor)
+    _assert_close(o, S, o_ref, S_ref, torch.bfloat16, f"floor {g_floor}")
+    assert device_status() == 0
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
