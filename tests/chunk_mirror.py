@@ -18,7 +18,9 @@ which is exact: g = 0, beta = 0, k = 0 make a padded token the identity):
   T = (I + A_kk)^-1   (16x16 diagonal blocks by substitution, then block merges)
   W = T (beta * k * Gt * D[b(i),0]),   U = T (beta * v)
   per chunk, with the carried state S:
-     Vn = U - W S
+     Vn = U - W S                       (form "wy")
+        = T' (V - (k Gt D[b(i),0]) S)   (form "z", T' = T Diag(beta): what the
+                                         tensor-core kernel computes)
      O  = scale ((q * Gt * D[b(i),0]) S + A_qk Vn)
      S  = Diag(D[nb,0]) S + K^(nb)^T Vn        (K^(nb) = k_j exp(G_{C-1} - G_j))
 
@@ -26,12 +28,13 @@ The 16-token blocks are where the per-step floor matters: within a block
 every factor is bounded by e^{-16 floor}, inside bf16/fp32 range for floor >= -5.45
 (fupanwang.com Kimi K3 report digest, KDA section, Fig. 3).
 
-``prec`` (a dict operand -> "bf16" | "tf32") rounds the tensor-core
-operands the way a kernel stores them; ``KERNEL_PREC`` is the mixed plan of
-the tcgen05 kernel: tf32 for the operands the output is sensitive to (the
-intra-chunk A operands, A_qk, V_new, K^) and bf16 for the rest.  beta is
-folded into the columns of T (T' = T Diag(beta)) so that U = T' V multiplies
-the exact bf16 input V.
+``prec`` (a dict operand -> "bf16" | "tf32" | "tf32t") rounds the tensor-core
+operands the way a kernel stores them ("tf32t": fp32 stored whole, the MMA
+reading only its leading 19 bits, i.e. truncation); ``KERNEL_PREC`` with
+``KERNEL_FORM`` is the plan of the tcgen05 kernel: tf32 for the operands the
+output is sensitive to (the intra-chunk A operands, A_qk, T', Z, V_new, K^)
+and bf16 for the state and Q e^G / K e^G.  beta is folded into the columns of
+T (T' = T Diag(beta)).
 """
 from __future__ import annotations
 
@@ -56,14 +59,24 @@ def _tf32(x):
     return u.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
-_ROUND = {"bf16": _bf16, "tf32": _tf32, "fp32": lambda x: np.asarray(x, np.float32).astype(np.float64)}
+def _tf32_trunc(x):
+    """fp64 -> fp32, keeping the leading 19 bits (what a tf32 MMA reads of an
+    unrounded fp32 operand) -> fp64."""
+    f = np.asarray(x, dtype=np.float32)
+    u = f.view(np.uint32) & np.uint32(0xFFFFE000)
+    return u.view(np.float32).astype(np.float64)
 
-# operand -> storage precision in the tcgen05 kernel
+
+_ROUND = {"bf16": _bf16, "tf32": _tf32, "tf32t": _tf32_trunc,
+          "fp32": lambda x: np.asarray(x, np.float32).astype(np.float64)}
+
+# operand -> storage precision in the tcgen05 kernel, and the form of its V_new
 KERNEL_PREC = {
-    "Arow": "tf32", "Acol": "tf32",       # q~, k~ and K^(b) for A_qk / A_kk
-    "Aqk": "tf32", "Vn": "tf32", "Khat": "tf32",
-    "T": "bf16", "KG": "bf16", "W": "bf16", "S": "bf16", "QG": "bf16",
+    "Arow": "tf32t", "Acol": "tf32t",     # q~, k~ and K^(b) for A_qk / A_kk
+    "Aqk": "tf32", "T": "tf32t", "Z": "tf32", "Vn": "tf32", "Khat": "tf32",
+    "KG": "bf16", "S": "bf16", "QG": "bf16",
 }
+KERNEL_FORM = "z"
 
 
 def _block_inverse(A, sub=16):
@@ -93,7 +106,7 @@ def _block_inverse(A, sub=16):
 
 
 def chunked_kda(q, k, v, g, beta, S0=None, scale=None, gate=None, g_floor=-5.0,
-                C=64, sub=16, prec=None):
+                C=64, sub=16, prec=None, form="wy"):
     """One sequence, all heads.  q,k,g [T,H,dk]; v [T,H,dv]; beta [T,H];
     S0 [H,dk,dv].  Returns (o [T,H,dv], S_T [H,dk,dv]) in fp64."""
     q, k, v, g, beta = (np.asarray(x, dtype=np.float64) for x in (q, k, v, g, beta))
@@ -140,10 +153,14 @@ def chunked_kda(q, k, v, g, beta, S0=None, scale=None, gate=None, g_floor=-5.0,
             A_kk = np.where(jj < ii, A_kk, 0.0) * bc[:, None]
             Tb = rb("T", _block_inverse(A_kk, sub) * bc[None, :])   # T' = T Diag(beta)
             Dq = D[blk, 0]                                   # exp(r_{b(i)}) = Gamma / Gt
-            W = rb("W", Tb @ rb("KG", kc * Gt * Dq))
-            U = Tb @ vc
             Sb = rb("S", S)
-            Vn = rb("Vn", U - W @ Sb)
+            if form == "z":
+                Z = rb("Z", vc - rb("KG", kc * Gt * Dq) @ Sb)
+                Vn = rb("Vn", Tb @ Z)
+            else:
+                W = rb("W", Tb @ rb("KG", kc * Gt * Dq))
+                U = Tb @ vc
+                Vn = rb("Vn", U - W @ Sb)
             O = scale * (rb("QG", qc * Gt * Dq) @ Sb + rb("Aqk", A_qk) @ Vn)
             S = D[nb, 0][:, None] * S + rb("Khat", Kb[nb]).T @ Vn
             o[c0:c0 + L, h] = O[:L]

@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 
 import oracle
-from chunk_mirror import KERNEL_PREC, chunked_kda, _bf16
+from chunk_mirror import KERNEL_FORM, KERNEL_PREC, chunked_kda, _bf16
 from parity import TOL_BF16, rel_max, rel_max_beyond_bf16
 
 
@@ -22,16 +22,17 @@ def _inputs(rng, T, H, d, g_mode="softplus"):
     return q, k, v, g, beta
 
 
+@pytest.mark.parametrize("form", ["wy", "z"])
 @pytest.mark.parametrize("C", [16, 32, 64])
 @pytest.mark.parametrize("g_mode", ["softplus", "floor"])
-def test_mirror_matches_oracle_fp64(C, g_mode):
+def test_mirror_matches_oracle_fp64(C, g_mode, form):
     rng = np.random.default_rng(C)
     T, H, d = 200, 2, 32          # several chunks and a ragged tail
     q, k, v, g, beta = _inputs(rng, T, H, d, g_mode)
     S0 = rng.standard_normal((H, d, d)) * 0.02
     z = rng.standard_normal((T, H, d))
     o_ref, S_ref = oracle.kda_fwd_ref(q, k, v, g, beta, S0=S0[None], gate=z)
-    o, S = chunked_kda(q, k, v, g, beta, S0=S0, gate=z, C=C)
+    o, S = chunked_kda(q, k, v, g, beta, S0=S0, gate=z, C=C, form=form)
     assert oracle.rel_err(o, o_ref) < 1e-10
     assert oracle.rel_err(S, S_ref[0]) < 1e-10
 
@@ -54,7 +55,7 @@ def test_mixed_precision_plan_within_tolerance(g_mode):
     T, H, d = 512, 2, 128
     q, k, v, g, beta = (_bf16(x) for x in _inputs(rng, T, H, d, g_mode))
     o_ref, S_ref = oracle.kda_fwd_ref(q, k, v, g, beta)
-    o, S = chunked_kda(q, k, v, g, beta, C=64, prec=KERNEL_PREC)
+    o, S = chunked_kda(q, k, v, g, beta, C=64, prec=KERNEL_PREC, form=KERNEL_FORM)
     eo = rel_max_beyond_bf16(_bf16(o), o_ref)
     es = rel_max(S, S_ref[0])
     assert eo < 0.6 * TOL_BF16 and es < 0.6 * TOL_BF16, (eo, es)
@@ -68,7 +69,7 @@ def test_all_bf16_operands_exceed_tolerance():
     q, k, v, g, beta = (_bf16(x) for x in _inputs(rng, T, H, d, "softplus"))
     o_ref, S_ref = oracle.kda_fwd_ref(q, k, v, g, beta)
     allbf = {name: "bf16" for name in KERNEL_PREC}
-    o, S = chunked_kda(q, k, v, g, beta, C=64, prec=allbf)
+    o, S = chunked_kda(q, k, v, g, beta, C=64, prec=allbf, form=KERNEL_FORM)
     assert max(rel_max_beyond_bf16(_bf16(o), o_ref), rel_max(S, S_ref[0])) > TOL_BF16
 
 
