@@ -472,204 +472,284 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const float L2E = 1.4426950408889634f;
 
-    for (int ci = 0; ci < nchunks && !failed; ++ci) {
-        const int64_t t0 = t_begin + (int64_t)ci * C;
-        const int L = (int)min((int64_t)C, t_end - t0);
+    // The loop runs prep stages (chunk ci, pass) in order.  A chunk's state
+    // chain ends with the N = 192 MMA; the next chunk's first prep pass runs
+    // while that MMA executes, and only then is the previous chunk finished
+    // (state update, outputs) -- its tail -- before the next MMAs are issued.
+    int64_t t0 = 0, t0p = 0;                 // first token of the prepped / finishing chunk
+    int L = 0, Lp = 0;                       // their lengths
+    bool loads_ok = true;
+    float2 khv[2][2] = {};                   // this thread's K^ values of the current prep pass
+    auto store_khat = [&](int pass_, int bb, int hr) {
+        const int b = 2 * mp + bb;
+        const uint32_t i = (uint32_t)(16 * b + 8 * hr + gq);
+        const uint32_t cg = (uint32_t)(pass_ * 64 + cA);
+        const uint32_t kho = OFF_KHT + (i >> 5) * AK_KBLK;
+        *reinterpret_cast<float *>(sm + kho + sw128(cg, (i & 31u) * 4u)) = khv[bb][hr].x;
+        *reinterpret_cast<float *>(sm + kho + sw128(cg + 1u, (i & 31u) * 4u)) = khv[bb][hr].y;
+    };
+#pragma unroll 1
+    for (int st = 0; st <= 2 * nchunks && !failed; ++st) {
+        const int pass = st & 1;
+        const int ci = st >> 1;              // chunk of this prep pass (nchunks: none, tail only)
+        const int tci = ci - 1;              // chunk finished by this stage's tail (pass 0)
+        if (pass == 0) {
+            t0p = t0; Lp = L;
+            loads_ok = true;
+            if (ci < nchunks) {
+                t0 = t_begin + (int64_t)ci * C;
+                L = (int)min((int64_t)C, t_end - t0);
+            }
+        }
         const uint32_t ld_par = (uint32_t)(ci & 1);
+        const bool ragged = L < C;
 
         // ================================================= prep + A MMAs, 2 passes of 64 key channels
         // Warp (nt, mp) of a pass owns channels 8 nt .. 8 nt + 7 of the pass and the
         // 16-token blocks 2 mp, 2 mp + 1; lane (gq, tq) holds channels cA = 8 nt + 2 tq,
         // cA + 1 of tokens 16 b + gq and 16 b + gq + 8 (mma fragment layout).
-        bool loads_ok = true;
-        const bool ragged = L < C;
-#pragma unroll 1
-        for (int pass = 0; pass < 2; ++pass) {
-            loads_ok = mbar_wait(&bar_qkg[pass], ld_par) && loads_ok;
-            ++qkg_done[pass];
-            const uint32_t raw = smb + (pass ? OFF_QKG1 : OFF_QKG0);
-            if (pass == 0) {
-                if (tid < C) s_beta[tid] = beta_next;
-                beta_next = load_beta(ci + 1);
-            }
-            // (1) decay prefix sums on the warp-level tensor cores: with
-            //     gc = max(g, floor) (zero past the chunk's end),
-            //       x_i   = sum of gc over block b(i) up to i      = G_i - r_b(i)
-            //       r_b+1 = sum of gc over blocks 0..b
-            //     as products of 0/1 matrices with gc (bf16 operands, fp32 sums:
-            //     exact up to the fp32 rounding of the sums)
-            uint32_t gf[2][4];                     // [tokens 32h..][block 2h + (j>>1), half j&1]
-            ldsm_x4_trans(gf[0], raw + QKG_G + sw128((uint32_t)lane, (uint32_t)nt * 16u));
-            ldsm_x4_trans(gf[1], raw + QKG_G + sw128((uint32_t)(32 + lane), (uint32_t)nt * 16u));
-            if (pass == 1 && warp == 0) {          // the rest of the pass-0 A MMAs
-                __syncwarp();
-                issue_a(0, 2, NB);
-                __syncwarp();
-            }
-            uint32_t gi[2][4];                     // indicator g <= fb (floor not a bf16 value)
+        if (ci < nchunks) {
+                loads_ok = mbar_wait(&bar_qkg[pass], ld_par) && loads_ok;
+                ++qkg_done[pass];
+                const uint32_t raw = smb + (pass ? OFF_QKG1 : OFF_QKG0);
+                if (pass == 0) {
+                    if (tid < C) s_beta[tid] = beta_next;
+                    beta_next = load_beta(ci + 1);
+                }
+                // (1) decay prefix sums on the warp-level tensor cores: with
+                //     gc = max(g, floor) (zero past the chunk's end),
+                //       x_i   = sum of gc over block b(i) up to i      = G_i - r_b(i)
+                //       r_b+1 = sum of gc over blocks 0..b
+                //     as products of 0/1 matrices with gc (bf16 operands, fp32 sums:
+                //     exact up to the fp32 rounding of the sums)
+                uint32_t gf[2][4];                     // [tokens 32h..][block 2h + (j>>1), half j&1]
+                ldsm_x4_trans(gf[0], raw + QKG_G + sw128((uint32_t)lane, (uint32_t)nt * 16u));
+                ldsm_x4_trans(gf[1], raw + QKG_G + sw128((uint32_t)(32 + lane), (uint32_t)nt * 16u));
+                if (pass == 1 && warp == 0) {          // the rest of the pass-0 A MMAs
+                    __syncwarp();
+                    issue_a(0, 2, NB);
+                    __syncwarp();
+                }
+                uint32_t gi[2][4];                     // indicator g <= fb (floor not a bf16 value)
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < 2; ++h) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const __nv_bfloat162 gv = *reinterpret_cast<const __nv_bfloat162 *>(&gf[h][j]);
-                    __nv_bfloat162 gc = __hmax2(gv, floor_b2);
-                    __nv_bfloat162 ind = __hle2(gv, floor_b2);
-                    if (ragged) {                  // tokens past the chunk's end contribute nothing
-                        const int tok = 32 * h + 8 * j + 2 * tq;
-                        const uint32_t keep = (tok < L ? 0x0000FFFFu : 0u) | (tok + 1 < L ? 0xFFFF0000u : 0u);
-                        gf[h][j] = *reinterpret_cast<uint32_t *>(&gc) & keep;
-                        gi[h][j] = *reinterpret_cast<uint32_t *>(&ind) & keep;
-                    } else {
-                        gf[h][j] = *reinterpret_cast<uint32_t *>(&gc);
-                        gi[h][j] = *reinterpret_cast<uint32_t *>(&ind);
+                    for (int j = 0; j < 4; ++j) {
+                        const __nv_bfloat162 gv = *reinterpret_cast<const __nv_bfloat162 *>(&gf[h][j]);
+                        __nv_bfloat162 gc = __hmax2(gv, floor_b2);
+                        __nv_bfloat162 ind = __hle2(gv, floor_b2);
+                        if (ragged) {                  // tokens past the chunk's end contribute nothing
+                            const int tok = 32 * h + 8 * j + 2 * tq;
+                            const uint32_t keep = (tok < L ? 0x0000FFFFu : 0u) | (tok + 1 < L ? 0xFFFF0000u : 0u);
+                            gf[h][j] = *reinterpret_cast<uint32_t *>(&gc) & keep;
+                            gi[h][j] = *reinterpret_cast<uint32_t *>(&ind) & keep;
+                        } else {
+                            gf[h][j] = *reinterpret_cast<uint32_t *>(&gc);
+                            gi[h][j] = *reinterpret_cast<uint32_t *>(&ind);
+                        }
                     }
                 }
-            }
-            float xs[2][4], rr[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-            for (int bb = 0; bb < 2; ++bb) {
-                const uint32_t b0 = mp ? gf[1][2 * bb] : gf[0][2 * bb];
-                const uint32_t b1 = mp ? gf[1][2 * bb + 1] : gf[0][2 * bb + 1];
-                xs[bb][0] = xs[bb][1] = xs[bb][2] = xs[bb][3] = 0.0f;
-                mma_16x8x16_bf16(xs[bb], a_blk, b0, b1);
-            }
-#pragma unroll
-            for (int kb = 0; kb < NB; ++kb) mma_16x8x16_bf16(rr, a_ref[kb], gf[kb >> 1][2 * (kb & 1)], gf[kb >> 1][2 * (kb & 1) + 1]);
-            if (floor_inexact) {                   // + (floor - fb) x (the same sums of the indicator)
-                float xi[2][4], ri[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                float xs[2][4], rr[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
                 for (int bb = 0; bb < 2; ++bb) {
-                    const uint32_t b0 = mp ? gi[1][2 * bb] : gi[0][2 * bb];
-                    const uint32_t b1 = mp ? gi[1][2 * bb + 1] : gi[0][2 * bb + 1];
-                    xi[bb][0] = xi[bb][1] = xi[bb][2] = xi[bb][3] = 0.0f;
-                    mma_16x8x16_bf16(xi[bb], a_blk, b0, b1);
+                    const uint32_t b0 = mp ? gf[1][2 * bb] : gf[0][2 * bb];
+                    const uint32_t b1 = mp ? gf[1][2 * bb + 1] : gf[0][2 * bb + 1];
+                    xs[bb][0] = xs[bb][1] = xs[bb][2] = xs[bb][3] = 0.0f;
+                    mma_16x8x16_bf16(xs[bb], a_blk, b0, b1);
                 }
 #pragma unroll
-                for (int kb = 0; kb < NB; ++kb) mma_16x8x16_bf16(ri, a_ref[kb], gi[kb >> 1][2 * (kb & 1)], gi[kb >> 1][2 * (kb & 1) + 1]);
+                for (int kb = 0; kb < NB; ++kb) mma_16x8x16_bf16(rr, a_ref[kb], gf[kb >> 1][2 * (kb & 1)], gf[kb >> 1][2 * (kb & 1) + 1]);
+                if (floor_inexact) {                   // + (floor - fb) x (the same sums of the indicator)
+                    float xi[2][4], ri[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    xs[0][e] = fmaf(floor_gap, xi[0][e], xs[0][e]);
-                    xs[1][e] = fmaf(floor_gap, xi[1][e], xs[1][e]);
-                    rr[e] = fmaf(floor_gap, ri[e], rr[e]);
-                }
-            }
-            // (2) block decay factors eT_b = e^{r_b+1 - r_b} for this lane's two channels
-            //     (rows 0..3 of the r tile sit in lanes 4 m + tq)
-            float2 eT[NB];
-            {
-                float pa = 0.0f, pb = 0.0f;
+                    for (int bb = 0; bb < 2; ++bb) {
+                        const uint32_t b0 = mp ? gi[1][2 * bb] : gi[0][2 * bb];
+                        const uint32_t b1 = mp ? gi[1][2 * bb + 1] : gi[0][2 * bb + 1];
+                        xi[bb][0] = xi[bb][1] = xi[bb][2] = xi[bb][3] = 0.0f;
+                        mma_16x8x16_bf16(xi[bb], a_blk, b0, b1);
+                    }
 #pragma unroll
-                for (int m = 0; m < NB; ++m) {
-                    const float ra = __shfl_sync(0xffffffffu, rr[0], 4 * m + tq);
-                    const float rb2 = __shfl_sync(0xffffffffu, rr[1], 4 * m + tq);
-                    eT[m] = make_float2(fexp(ra - pa), fexp(rb2 - pb));
-                    pa = ra; pb = rb2;
-                }
-            }
-            if (mp == 0 && gq == 0) {              // gamma = e^{r_4} for the state update
-                const float2 g4 = __fmul2_rn(__fmul2_rn(eT[0], eT[1]), __fmul2_rn(eT[2], eT[3]));
-                *reinterpret_cast<float2 *>(s_gam + (ci & 1) * D + pass * 64 + cA) = g4;
-            }
-            // (3) per-element factors; the stores that no MMA in flight reads go first
-            float2 qt[2][2], kt[2][2], kbar[2][2];
-            const float2 l2e = make_float2(L2E, L2E), nl2e = make_float2(-L2E, -L2E);
-            const uint32_t kh_col = OFF_KHT;       // + (i >> 5) * AK_KBLK + sw128(c, (i & 31) * 4)
+                    for (int kb = 0; kb < NB; ++kb) mma_16x8x16_bf16(ri, a_ref[kb], gi[kb >> 1][2 * (kb & 1)], gi[kb >> 1][2 * (kb & 1) + 1]);
 #pragma unroll
-            for (int bb = 0; bb < 2; ++bb) {
-                const int b = 2 * mp + bb;
-                float2 Eb = make_float2(1.0f, 1.0f), eK = make_float2(1.0f, 1.0f);
-#pragma unroll
-                for (int m = 0; m < NB; ++m) {
-                    if (m < b) Eb = __fmul2_rn(Eb, eT[m]);
-                    else eK = __fmul2_rn(eK, eT[m]);
-                }
-                uint32_t pq[2], pk[2];
-#pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {
-                    const int i = 16 * b + gq + 8 * hr;
-                    const float2 x2 = make_float2(xs[bb][2 * hr], xs[bb][2 * hr + 1]);
-                    const float2 t2 = __fmul2_rn(x2, l2e), u2 = __fmul2_rn(x2, nl2e);
-                    const float2 gt = make_float2(ex2_approx(t2.x), ex2_approx(t2.y));       // Gt_i
-                    const float2 ig = make_float2(ex2_approx(u2.x), ex2_approx(u2.y));       // 1 / Gt_i
-                    const uint32_t qoff = raw + QKG_Q + sw128((uint32_t)i, (uint32_t)cA * 2u);
-                    const float2 q2 = unpack_bf16x2(ld_shared_u32(qoff));
-                    const float2 k2 = unpack_bf16x2(ld_shared_u32(qoff + (QKG_K - QKG_Q)));
-                    qt[bb][hr] = __fmul2_rn(q2, gt);
-                    kt[bb][hr] = __fmul2_rn(k2, gt);
-                    kbar[bb][hr] = __fmul2_rn(k2, ig);                                        // Kbar_i
-                    const float2 qg = __fmul2_rn(qt[bb][hr], Eb), kg = __fmul2_rn(kt[bb][hr], Eb);
-                    pq[hr] = pack_bf16(qg.x, qg.y);
-                    pk[hr] = pack_bf16(kg.x, kg.y);
-                    // K^(4)^T [c x j] tf32: two channels of token i
-                    const float2 kh = __fmul2_rn(kbar[bb][hr], eK);
-                    const uint32_t cg = (uint32_t)(pass * 64 + cA);
-                    const uint32_t kho = kh_col + (uint32_t)(i >> 5) * AK_KBLK;
-                    *reinterpret_cast<float *>(sm + kho + sw128(cg, (uint32_t)(i & 31) * 4u)) = to_tf32(kh.x);
-                    *reinterpret_cast<float *>(sm + kho + sw128(cg + 1u, (uint32_t)(i & 31) * 4u)) = to_tf32(kh.y);
-                }
-                // Q e^G and K e^G (bf16 [c x i], tokens contiguous): transposing matrix stores
-                {
-                    const uint32_t row = (uint32_t)(pass * 64 + nt * 8 + (lane & 7));
-                    const uint32_t tb2 = (uint32_t)(16 * b + 8 * ((lane >> 3) & 1)) * 2u;
-                    stsm_x2_trans(smb + OFF_QG + sw128(row, tb2), pq[0], pq[1]);
-                    stsm_x2_trans(smb + OFF_KG + sw128(row, tb2), pk[0], pk[1]);
-                }
-            }
-            if (pass == 1) {                       // pass-0 A MMAs must be done with X~ and K^(b)
-                loads_ok = mbar_wait(bar_mma, mma_phase & 1) && loads_ok;
-                ++mma_phase;
-                tc_fence_after();
-            }
-            // (4) the A-MMA operands: X~ rows (q~ at 32 b + r, k~ at 32 b + 16 + r) and the
-            //     K^(b') copies, b' >= b (tf32 operands: the MMA reads the leading 19 bits)
-#pragma unroll
-            for (int bb = 0; bb < 2; ++bb) {
-                const int b = 2 * mp + bb;
-                float2 dfac[NB];                   // e^{r_b' - r_b} for b' > b
-                {
-                    float2 run = make_float2(1.0f, 1.0f);
-#pragma unroll
-                    for (int m = 0; m < NB; ++m) {
-                        if (m > b) run = __fmul2_rn(run, eT[m - 1]);
-                        dfac[m] = run;
+                    for (int e = 0; e < 4; ++e) {
+                        xs[0][e] = fmaf(floor_gap, xi[0][e], xs[0][e]);
+                        xs[1][e] = fmaf(floor_gap, xi[1][e], xs[1][e]);
+                        rr[e] = fmaf(floor_gap, ri[e], rr[e]);
                     }
                 }
-#pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {
-                    const uint32_t i = (uint32_t)(16 * b + 8 * hr) + (uint32_t)gq;
-                    const uint32_t xrow = (uint32_t)(32 * b + 8 * hr) + (uint32_t)gq;
-                    *reinterpret_cast<float2 *>(sm + xt_lane + xrow * 128u) = qt[bb][hr];
-                    *reinterpret_cast<float2 *>(sm + xt_lane + (xrow + 16u) * 128u) = kt[bb][hr];
+                // (2) block decay factors eT_b = e^{r_b+1 - r_b} for this lane's two channels
+                //     (rows 0..3 of the r tile sit in lanes 4 m + tq)
+                float2 eT[NB];
+                {
+                    float pa = 0.0f, pb = 0.0f;
 #pragma unroll
                     for (int m = 0; m < NB; ++m) {
-                        if (m < b) continue;
-                        const float2 v = m == b ? kbar[bb][hr] : __fmul2_rn(kbar[bb][hr], dfac[m]);
-                        *reinterpret_cast<float2 *>(sm + kb_lane + kb_base(m) + kblk * kb_rows(m) * 128u + i * 128u) = v;
+                        const float ra = __shfl_sync(0xffffffffu, rr[0], 4 * m + tq);
+                        const float rb2 = __shfl_sync(0xffffffffu, rr[1], 4 * m + tq);
+                        eT[m] = make_float2(fexp(ra - pa), fexp(rb2 - pb));
+                        pa = ra; pb = rb2;
                     }
                 }
-            }
-            // block barrier: the MMA issue needs every thread's operands (and the waits' outcome)
-            fence_async_smem();
-            tc_fence_before();
-            if (!__syncthreads_and(loads_ok)) { failed = true; break; }
-            tc_fence_after();
-            if (ci + 1 < nchunks) note_loads(1 << pass);
-            ++mma_issued;
-            if (warp == 0) {
-                // q, k, g of this pass are consumed: prefetch the next chunk's; the
-                // previous chunk's output tile is complete: store it
-                if (lane == 0) {
-                    if (ci + 1 < nchunks) issue_loads(ci + 1, 1 << pass);
-                    if (pass == 0 && o_row >= 0) store_o_tile();
+                if (mp == 0 && gq == 0) {              // gamma = e^{r_4} for the state update
+                    const float2 g4 = __fmul2_rn(__fmul2_rn(eT[0], eT[1]), __fmul2_rn(eT[2], eT[3]));
+                    *reinterpret_cast<float2 *>(s_gam + (ci & 1) * D + pass * 64 + cA) = g4;
                 }
-                __syncwarp();
-                // pass 0: blocks 0-1 now, blocks 2-3 early in warp 0's pass-1 prep (a long
-                // run of issues stalls the issuing warp); pass 1: everything now
-                issue_a(pass, 0, pass == 0 ? 2 : NB);
-            }
-            if (pass == 0) o_row = -1;
+                // (3) per-element factors; the stores that no MMA in flight reads go first
+                float2 qt[2][2], kt[2][2], kbar[2][2];
+                const float2 l2e = make_float2(L2E, L2E), nl2e = make_float2(-L2E, -L2E);
+#pragma unroll
+                for (int bb = 0; bb < 2; ++bb) {
+                    const int b = 2 * mp + bb;
+                    float2 Eb = make_float2(1.0f, 1.0f), eK = make_float2(1.0f, 1.0f);
+#pragma unroll
+                    for (int m = 0; m < NB; ++m) {
+                        if (m < b) Eb = __fmul2_rn(Eb, eT[m]);
+                        else eK = __fmul2_rn(eK, eT[m]);
+                    }
+                    uint32_t pq[2], pk[2];
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int i = 16 * b + gq + 8 * hr;
+                        const float2 x2 = make_float2(xs[bb][2 * hr], xs[bb][2 * hr + 1]);
+                        const float2 t2 = __fmul2_rn(x2, l2e), u2 = __fmul2_rn(x2, nl2e);
+                        const float2 gt = make_float2(ex2_approx(t2.x), ex2_approx(t2.y));       // Gt_i
+                        const float2 ig = make_float2(ex2_approx(u2.x), ex2_approx(u2.y));       // 1 / Gt_i
+                        const uint32_t qoff = raw + QKG_Q + sw128((uint32_t)i, (uint32_t)cA * 2u);
+                        const float2 q2 = unpack_bf16x2(ld_shared_u32(qoff));
+                        const float2 k2 = unpack_bf16x2(ld_shared_u32(qoff + (QKG_K - QKG_Q)));
+                        qt[bb][hr] = __fmul2_rn(q2, gt);
+                        kt[bb][hr] = __fmul2_rn(k2, gt);
+                        kbar[bb][hr] = __fmul2_rn(k2, ig);                                        // Kbar_i
+                        const float2 qg = __fmul2_rn(qt[bb][hr], Eb), kg = __fmul2_rn(kt[bb][hr], Eb);
+                        pq[hr] = pack_bf16(qg.x, qg.y);
+                        pk[hr] = pack_bf16(kg.x, kg.y);
+                        // K^(4)^T [c x j] tf32: two channels of token i; on the first pass the
+                        // previous chunk's last MMA may still read these rows: stored later
+                        const float2 kh = __fmul2_rn(kbar[bb][hr], eK);
+                        khv[bb][hr] = make_float2(to_tf32(kh.x), to_tf32(kh.y));
+                        if (pass == 1) store_khat(1, bb, hr);
+                    }
+                    // Q e^G and K e^G (bf16 [c x i], tokens contiguous): transposing matrix stores
+                    {
+                        const uint32_t row = (uint32_t)(pass * 64 + nt * 8 + (lane & 7));
+                        const uint32_t tb2 = (uint32_t)(16 * b + 8 * ((lane >> 3) & 1)) * 2u;
+                        stsm_x2_trans(smb + OFF_QG + sw128(row, tb2), pq[0], pq[1]);
+                        stsm_x2_trans(smb + OFF_KG + sw128(row, tb2), pk[0], pk[1]);
+                    }
+                }
+                if (pass == 1) {                       // pass-0 A MMAs must be done with X~ and K^(b)
+                    loads_ok = mbar_wait(bar_mma, mma_phase & 1) && loads_ok;
+                    ++mma_phase;
+                    tc_fence_after();
+                }
+                // (4) the A-MMA operands: X~ rows (q~ at 32 b + r, k~ at 32 b + 16 + r) and the
+                //     K^(b') copies, b' >= b (tf32 operands: the MMA reads the leading 19 bits)
+#pragma unroll
+                for (int bb = 0; bb < 2; ++bb) {
+                    const int b = 2 * mp + bb;
+                    float2 dfac[NB];                   // e^{r_b' - r_b} for b' > b
+                    {
+                        float2 run = make_float2(1.0f, 1.0f);
+#pragma unroll
+                        for (int m = 0; m < NB; ++m) {
+                            if (m > b) run = __fmul2_rn(run, eT[m - 1]);
+                            dfac[m] = run;
+                        }
+                    }
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const uint32_t i = (uint32_t)(16 * b + 8 * hr) + (uint32_t)gq;
+                        const uint32_t xrow = (uint32_t)(32 * b + 8 * hr) + (uint32_t)gq;
+                        *reinterpret_cast<float2 *>(sm + xt_lane + xrow * 128u) = qt[bb][hr];
+                        *reinterpret_cast<float2 *>(sm + xt_lane + (xrow + 16u) * 128u) = kt[bb][hr];
+#pragma unroll
+                        for (int m = 0; m < NB; ++m) {
+                            if (m < b) continue;
+                            const float2 v = m == b ? kbar[bb][hr] : __fmul2_rn(kbar[bb][hr], dfac[m]);
+                            *reinterpret_cast<float2 *>(sm + kb_lane + kb_base(m) + kblk * kb_rows(m) * 128u + i * 128u) = v;
+                        }
+                    }
+                }
         }
-        if (failed) break;
+        if (pass == 0) {
+            if (ci > 0) {
+                if (!wait_mma()) { failed = true; break; }
+
+                // ================================================= state update and outputs
+                // (no block barrier after this phase: the next chunk's prep touches none
+                // of what it reads -- gamma is double-buffered -- and the next MMA that
+                // overwrites these TMEM columns is issued after a block barrier)
+                {
+                    const float *gam = s_gam + (tci & 1) * D;
+#pragma unroll
+                    for (int hq = 0; hq < 2; ++hq) {       // dS^T rows c in [32 cq + 16 hq, +16)
+                        uint32_t rd[16];
+                        tmem_ld16(tbase + lane_base + T_DS + cq * 32 + hq * 16, rd);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            S[hq * 16 + e] = fmaf(gam[cq * 32 + hq * 16 + e], S[hq * 16 + e], __uint_as_float(rd[e]));
+                    }
+                    store_state_bf16();
+                    uint32_t r1[16], r2[16];
+                    tmem_ld16(tbase + lane_base + T_O1 + cq * 16, r1);
+                    tmem_ld16(tbase + lane_base + T_O2 + cq * 16, r2);
+                    tmem_wait_ld();
+                    if (store_o) {
+                        float x[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) x[e] = p.scale * (__uint_as_float(r1[e]) + __uint_as_float(r2[e]));
+                        const int nv = min(16, Lp - cq * 16);   // tokens of this thread inside the chunk
+                        const int64_t off0 = ((t0p + cq * 16) * H + hh) * D + vlane;
+                        if (gate) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                if (e < nv) x[e] *= sigmoid_fast(__bfloat162float(gate[off0 + (int64_t)e * H * D]));
+                        }
+                        if (Lp == C) {
+                            // full chunk: into the staging tile, stored by TMA after the next block barrier
+                            unsigned char *ost = sm + OFF_OST + (uint32_t)(vlane >> 6) * AK_KBLK;
+                            const uint32_t vb = (uint32_t)(vlane & 63) * 2u;
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                *reinterpret_cast<__nv_bfloat16 *>(ost + sw128((uint32_t)(cq * 16 + e), vb)) = __float2bfloat16_rn(x[e]);
+                            o_row = t0p;
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                if (e < nv) o[off0 + (int64_t)e * H * D] = __float2bfloat16_rn(x[e]);
+                        }
+                    }
+                }
+            }
+            if (ci == nchunks) break;
+#pragma unroll
+            for (int bb = 0; bb < 2; ++bb)
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) store_khat(0, bb, hr);
+        }
+        // block barrier: the MMA issue needs every thread's operands (and the waits' outcome)
+        fence_async_smem();
+        tc_fence_before();
+        if (!__syncthreads_and(loads_ok)) { failed = true; break; }
+        tc_fence_after();
+        if (ci + 1 < nchunks) note_loads(1 << pass);
+        ++mma_issued;
+        if (warp == 0) {
+            // q, k, g of this pass are consumed: prefetch the next chunk's; the
+            // previous chunk's output tile is complete: store it
+            if (lane == 0) {
+                if (ci + 1 < nchunks) issue_loads(ci + 1, 1 << pass);
+                if (pass == 0 && o_row >= 0) store_o_tile();
+            }
+            __syncwarp();
+            // pass 0: blocks 0-1 now, blocks 2-3 early in warp 0's pass-1 prep (a long
+            // run of issues stalls the issuing warp); pass 1: everything now
+            issue_a(pass, 0, pass == 0 ? 2 : NB);
+        }
+        if (pass == 0) o_row = -1;
+        if (pass == 0) continue;
+
         if (tid == 0) bulk_wait_read();        // the staged output tile has been read
         if (!wait_mma()) { failed = true; break; }
 
@@ -884,54 +964,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (leader) mma_tf32_ts(tbase + T_O2, tbase + T_VN + 8u * s, at(d_k16, OFF_AK + kb * AK_KBLK + koff), id_2, s > 0);
             }
             if (leader) mma_commit(bar_mma);
-        }
-        if (!wait_mma()) { failed = true; break; }
-
-        // ================================================= state update and outputs
-        // (no block barrier after this phase: the next chunk's prep touches none
-        // of what it reads -- gamma is double-buffered -- and the next MMA that
-        // overwrites these TMEM columns is issued after a block barrier)
-        {
-            const float *gam = s_gam + (ci & 1) * D;
-#pragma unroll
-            for (int hq = 0; hq < 2; ++hq) {       // dS^T rows c in [32 cq + 16 hq, +16)
-                uint32_t rd[16];
-                tmem_ld16(tbase + lane_base + T_DS + cq * 32 + hq * 16, rd);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    S[hq * 16 + e] = fmaf(gam[cq * 32 + hq * 16 + e], S[hq * 16 + e], __uint_as_float(rd[e]));
-            }
-            store_state_bf16();
-            uint32_t r1[16], r2[16];
-            tmem_ld16(tbase + lane_base + T_O1 + cq * 16, r1);
-            tmem_ld16(tbase + lane_base + T_O2 + cq * 16, r2);
-            tmem_wait_ld();
-            if (store_o) {
-                float x[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) x[e] = p.scale * (__uint_as_float(r1[e]) + __uint_as_float(r2[e]));
-                const int nv = min(16, L - cq * 16);   // tokens of this thread inside the chunk
-                const int64_t off0 = ((t0 + cq * 16) * H + hh) * D + vlane;
-                if (gate) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (e < nv) x[e] *= sigmoid_fast(__bfloat162float(gate[off0 + (int64_t)e * H * D]));
-                }
-                if (L == C) {
-                    // full chunk: into the staging tile, stored by TMA after the next block barrier
-                    unsigned char *ost = sm + OFF_OST + (uint32_t)(vlane >> 6) * AK_KBLK;
-                    const uint32_t vb = (uint32_t)(vlane & 63) * 2u;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        *reinterpret_cast<__nv_bfloat16 *>(ost + sw128((uint32_t)(cq * 16 + e), vb)) = __float2bfloat16_rn(x[e]);
-                    o_row = t0;
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (e < nv) o[off0 + (int64_t)e * H * D] = __float2bfloat16_rn(x[e]);
-                }
-            }
         }
     }
 
