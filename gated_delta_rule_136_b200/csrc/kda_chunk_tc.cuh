@@ -579,16 +579,23 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 // (2) block decay factors eT_b = e^{r_b+1 - r_b} for this lane's two channels
                 //     (rows 0..3 of the r tile sit in lanes 4 m + tq)
+                //     lane (gq, tq) evaluates one factor -- block gq % 4 of channel
+                //     cA + gq / 4 -- and gathers the other seven with shuffles
                 float2 eT[NB];
                 {
-                    float pa = 0.0f, pb = 0.0f;
+                    const int m = gq & 3;
+                    // r_{m+1} and r_m of channels cA (rr[0]) and cA + 1 (rr[1])
+                    const float hiA = __shfl_sync(0xffffffffu, rr[0], 4 * m + tq);
+                    const float hiB = __shfl_sync(0xffffffffu, rr[1], 4 * m + tq);
+                    const float loA = __shfl_sync(0xffffffffu, rr[0], (4 * m + 28 + tq) & 31);
+                    const float loB = __shfl_sync(0xffffffffu, rr[1], (4 * m + 28 + tq) & 31);
+                    const float hi = (gq >> 2) ? hiB : hiA;
+                    const float lo = m == 0 ? 0.0f : ((gq >> 2) ? loB : loA);
+                    const float e = fexp(hi - lo);
 #pragma unroll
-                    for (int m = 0; m < NB; ++m) {
-                        const float ra = __shfl_sync(0xffffffffu, rr[0], 4 * m + tq);
-                        const float rb2 = __shfl_sync(0xffffffffu, rr[1], 4 * m + tq);
-                        eT[m] = make_float2(fexp(ra - pa), fexp(rb2 - pb));
-                        pa = ra; pb = rb2;
-                    }
+                    for (int mm = 0; mm < NB; ++mm)
+                        eT[mm] = make_float2(__shfl_sync(0xffffffffu, e, 4 * mm + tq),
+                                             __shfl_sync(0xffffffffu, e, 4 * (mm + 4) + tq));
                 }
                 if (mp == 0 && gq == 0) {              // gamma = e^{r_4} for the state update
                     const float2 g4 = __fmul2_rn(__fmul2_rn(eT[0], eT[1]), __fmul2_rn(eT[2], eT[3]));
