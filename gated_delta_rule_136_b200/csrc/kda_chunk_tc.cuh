@@ -12,7 +12,7 @@
 //   K^(b)_j = Kbar_j e^{r_b - r_{b(j)}}  for b(j) <= b   ( = k_j e^{r_b - G_j} )
 //   A_qk[i,j] = (q_i Gt_i) . K^(b(i))_j   (j <= i),   A_kk[i,j] = beta_i (k_i Gt_i) . K^(b(i))_j  (j < i)
 //   T' = (I + A_kk)^-1 Diag(beta)
-//   Vn = T' (V - (k Gt e^{r_b}) S)   (= U - W S of the WY form, U = T' V, W = T' K e^G)
+//   Vn = T' V - T' ((k Gt e^{r_b}) S)   (= U - W S of the WY form, U = T' V, W = T' K e^G)
 //   O  = scale ((q Gt e^{r_b}) S + A_qk Vn) [* sigmoid(z)]
 //   S  = Diag(e^{r_4}) S + K^(4)^T Vn
 // which equals the token recurrence in real arithmetic (the intra-chunk part
@@ -20,7 +20,7 @@
 // section 基础设施, FlashKDA).
 //
 // Precision: the products the outputs are sensitive to run in tf32 (A_qk /
-// A_kk operands, T' Z, A_qk Vn, K^(4)^T Vn); (K e^G) S and (Q e^G) S run in bf16.
+// A_kk operands, T' (K e^G) S, A_qk Vn, K^(4)^T Vn); T' V, (K e^G) S and (Q e^G) S run in bf16.
 //
 // Orientation: the state products are computed transposed so that the value
 // channel v is the TMEM lane (M = 128): S^T and Vn^T live in TMEM as the A
@@ -29,9 +29,9 @@
 // One CTA (512 threads) carries one (sequence, head) unit; its phases per
 // chunk run in order:
 //   prep (2 passes of 64 key channels; TMA tiles of q, k, g)  ->  A MMAs (tf32)
-//   -> A readout -> block-triangular inverse (warps 0-3), while warps 4-15 form
-//      Z = V - (K e^G) S from a (Q e^G | K e^G) S MMA issued after the readout
-//   -> Vn = T' Z MMA (tf32)  ->  A_qk Vn, K^T Vn MMAs (tf32)
+//   -> A readout -> block-triangular inverse (warps 0-3)
+//   -> Vn = T' V - T' Y MMAs (Y = (K e^G) S from an MMA issued behind the A MMAs)
+//   -> A_qk Vn, K^T Vn MMAs (tf32)
 //   -> state update + output epilogue.
 // The next chunk's q, k, g, v tiles are loaded by TMA while the current
 // chunk's later phases run.
@@ -67,6 +67,7 @@ constexpr uint32_t SCR_LD = 68;                    // 16-byte aligned rows
 constexpr uint32_t OFF_TP = OFF_INTRA + 17408;     // T' tf32 K-major [64 i x 64 j]: 2 x 8 KB
 constexpr uint32_t OFF_XS = OFF_INTRA + 33792;     // inverse scratch: 4 warps x [32 x 8] fp32: 4 KB
 constexpr uint32_t XS_LD = 8;
+constexpr uint32_t OFF_TPB = OFF_INTRA + 37888;    // T' bf16 K-major [64 i x 64 j]: 8 KB
 constexpr uint32_t OFF_QG = OFF_INTRA + 73728;     // Q e^G bf16 MN-major [128 c x 64 i]: 16 KB
 constexpr uint32_t OFF_KG = OFF_QG + 16384;        // K e^G bf16 K-major [128 c x 64 j]: 16 KB
 // B operand of the second state MMA: rows 0-63 = A_qk [i x j], rows 64-191 =
@@ -82,8 +83,8 @@ constexpr uint32_t OFF_KHT = OFF_AK + 64u * 128u;  // + kb * AK_KBLK + row * 128
 constexpr uint32_t OFF_SMALL = OFF_AK + 2u * AK_KBLK;  // beta[64], gamma[2][128], barriers, tmem base
 constexpr uint32_t SMEM_BYTES = OFF_SMALL + 2048;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024; // slack for aligning the base
-static_assert(OFF_TP % 1024 == 0 && OFF_TP + 16384 <= OFF_XS && OFF_XS + 4096 <= OFF_INTRA + 73728,
-              "post-MMA tiles fit the intra region");
+static_assert(OFF_TP % 1024 == 0 && OFF_TP + 16384 <= OFF_XS && OFF_XS + 4096 <= OFF_TPB &&
+              OFF_TPB % 1024 == 0 && OFF_TPB + 8192 <= OFF_INTRA + 73728, "post-MMA tiles fit the intra region");
 static_assert((OFF_KG - OFF_QG) % 16 == 0, "Q e^G | K e^G as one MN-major operand");
 static_assert(OFF_KB + 40960 <= OFF_INTRA + 73728, "intra tiles fit");
 static_assert(SMEM_ALLOC <= 232448, "fits in 227 KB");
@@ -102,9 +103,9 @@ static_assert(kb_base(3) + 128u * 64u + 64u * 128u <= 40960u, "K^(b) reads stay 
 constexpr uint32_t T_DB = 0;      // A MMAs: 4 x 32 columns (M = 64 layout)
 constexpr uint32_t T_O2 = 0;      // (A_qk Vn)^T   [v x i]   } one MMA (N = 192), after the
 constexpr uint32_t T_DS = 64;     // dS^T          [v x c]   } A readout and Vn
-constexpr uint32_t T_VN = 192;    // Vn^T = Z^T T'^T, then its tf32 copy (A operand)
+constexpr uint32_t T_VN = 192;    // Vn^T = V^T T'^T - Y^T T'^T, then its tf32 copy (A operand)
 constexpr uint32_t T_O1 = 256;    // ((Q e^G) S)^T  [v x i]  } one MMA (N = 128)
-constexpr uint32_t T_Z = 320;     // ((K e^G) S)^T  [v x j], then Z^T (tf32 A operand)
+constexpr uint32_t T_Z = 320;     // -((K e^G) S)^T  [v x j] (read as a tf32 A operand)
 constexpr uint32_t T_S = 384;     // S^T bf16 A operand (2 per column)
 constexpr uint32_t TMEM_COLS = 512;
 
@@ -437,9 +438,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t id_a = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 64, 32);
     const uint32_t id_1 = instr_desc(FMT_BF16, K_MAJOR, MN_MAJOR, 128, 128);
     const uint32_t id_vn = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 128, 64);
+    const uint32_t id_u = instr_desc(FMT_BF16, MN_MAJOR, K_MAJOR, 128, 64);
     const uint32_t id_2 = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 128, 192);
     const uint64_t d_k16 = smem_desc_sw128(smb, 16, 1024);          // K-major template
-    const uint64_t d_qk = smem_desc_sw128(smb, OFF_KG - OFF_QG, 1024);  // [Q e^G | K e^G] MN-major
+    const uint64_t d_qk = smem_desc_sw128(smb, OFF_KG - OFF_QG, 1024);  // [Q e^G | -K e^G] MN-major
+    const uint64_t d_mnv = smem_desc_sw128(smb, 8192, 1024);             // v: MN blocks 8 KB apart
     auto at = [](uint64_t tmpl, uint32_t byte_off) -> uint64_t {     // same descriptor, moved start
         return tmpl + (uint64_t)(byte_off >> 4);
     };
@@ -629,14 +632,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         kbar[bb][hr] = __fmul2_rn(k2, ig);                                        // Kbar_i
                         const float2 qg = __fmul2_rn(qt[bb][hr], Eb), kg = __fmul2_rn(kt[bb][hr], Eb);
                         pq[hr] = pack_bf16(qg.x, qg.y);
-                        pk[hr] = pack_bf16(kg.x, kg.y);
+                        pk[hr] = pack_bf16(-kg.x, -kg.y);   // -K e^G: the MMA then yields -Y
                         // K^(4)^T [c x j] tf32: two channels of token i; on the first pass the
                         // previous chunk's last MMA may still read these rows: stored later
                         const float2 kh = __fmul2_rn(kbar[bb][hr], eK);
                         khv[bb][hr] = make_float2(to_tf32(kh.x), to_tf32(kh.y));
                         if (pass == 1) store_khat(1, bb, hr);
                     }
-                    // Q e^G and K e^G (bf16 [c x i], tokens contiguous): transposing matrix stores
+                    // Q e^G and -K e^G (bf16 [c x i], tokens contiguous): transposing matrix stores
                     {
                         const uint32_t row = (uint32_t)(pass * 64 + nt * 8 + (lane & 7));
                         const uint32_t tb2 = (uint32_t)(16 * b + 8 * ((lane >> 3) & 1)) * 2u;
@@ -787,7 +790,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bool z_ok = true;
         ++y_issued;
         // ================================================= T = (I + A_kk)^-1, then T' = T Diag(beta) (warps 0-3)
-        // and, concurrently, Z = V - (K e^G) S (warps 4-15)
         // Blocked inverse of the unit lower-triangular 64x64 matrix: 16x16
         // diagonal blocks by forward substitution, then the block merges
         //   [[T11, 0], [T21, T22]]:  T21 = -T22 (A21 T11)
@@ -861,20 +863,30 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // K-blocks: columns o..o+31 from T, the other 32 zero for rows 0-31;
                 // rows 32-63, columns 0-31 are written by the 32 -> 64 step
                 const int i = o + lane;
+                // also as bf16 (K-major [i x j], one 128-byte row) for the T' V product
                 unsigned char *tpr = sm + OFF_TP + (uint32_t)warp * 8192u;   // K-block of columns o..o+31
 #pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4) {
-                    const int j0 = o + 4 * c4;
-                    const float4 t4 = *reinterpret_cast<const float4 *>(scr + i * SCR_LD + j0);
-                    const float4 b4 = *reinterpret_cast<const float4 *>(s_beta + j0);
-                    *reinterpret_cast<float4 *>(tpr + sw128((uint32_t)i, (uint32_t)c4 * 16u)) =
-                        make_float4(t4.x * b4.x, t4.y * b4.y, t4.z * b4.z, t4.w * b4.w);
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    const int j0 = o + 8 * c8;
+                    const float4 ta = *reinterpret_cast<const float4 *>(scr + i * SCR_LD + j0);
+                    const float4 tb = *reinterpret_cast<const float4 *>(scr + i * SCR_LD + j0 + 4);
+                    const float4 ba = *reinterpret_cast<const float4 *>(s_beta + j0);
+                    const float4 bb4 = *reinterpret_cast<const float4 *>(s_beta + j0 + 4);
+                    const float4 va = make_float4(ta.x * ba.x, ta.y * ba.y, ta.z * ba.z, ta.w * ba.w);
+                    const float4 vb = make_float4(tb.x * bb4.x, tb.y * bb4.y, tb.z * bb4.z, tb.w * bb4.w);
+                    *reinterpret_cast<float4 *>(tpr + sw128((uint32_t)i, (uint32_t)c8 * 32u)) = va;
+                    *reinterpret_cast<float4 *>(tpr + sw128((uint32_t)i, (uint32_t)c8 * 32u + 16u)) = vb;
+                    *reinterpret_cast<uint4 *>(sm + OFF_TPB + sw128((uint32_t)i, (uint32_t)j0 * 2u)) =
+                        make_uint4(pack_bf16(va.x, va.y), pack_bf16(va.z, va.w), pack_bf16(vb.x, vb.y), pack_bf16(vb.z, vb.w));
                 }
                 if (warp == 0) {
 #pragma unroll
                     for (int c4 = 0; c4 < 8; ++c4)
                         *reinterpret_cast<float4 *>(sm + OFF_TP + 8192u + sw128((uint32_t)i, (uint32_t)c4 * 16u)) =
                             make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+                    for (int c8 = 4; c8 < 8; ++c8)
+                        *reinterpret_cast<uint4 *>(sm + OFF_TPB + sw128((uint32_t)i, (uint32_t)c8 * 16u)) = make_uint4(0u, 0u, 0u, 0u);
                 }
             }
             if (warp < 4) {
@@ -902,53 +914,44 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         make_float2(x[rt][0] * b0, x[rt][1] * b1);
                     *reinterpret_cast<float2 *>(sm + OFF_TP + sw128((uint32_t)i0 + 8u, (uint32_t)j * 4u)) =
                         make_float2(x[rt][2] * b0, x[rt][3] * b1);
+                    *reinterpret_cast<uint32_t *>(sm + OFF_TPB + sw128((uint32_t)i0, (uint32_t)j * 2u)) =
+                        pack_bf16(x[rt][0] * b0, x[rt][1] * b1);
+                    *reinterpret_cast<uint32_t *>(sm + OFF_TPB + sw128((uint32_t)i0 + 8u, (uint32_t)j * 2u)) =
+                        pack_bf16(x[rt][2] * b0, x[rt][3] * b1);
                 }
-            }
-            if (warp >= 4) {
-                // Z^T[v, j] = V[j, v] - Y^T[v, j], tf32, in place of Y^T: lane quarter
-                // w % 4; the three warps of a quarter share its four 16-token groups
-                z_ok = mbar_wait(bar_v, ld_par) && mbar_wait(bar_y, y_phase & 1);
-                tc_fence_after();
-                const unsigned char *vt = sm + OFF_V + (uint32_t)(vlane >> 6) * 8192u;
-                const uint32_t vb = (uint32_t)(vlane & 63) * 2u;
-                for (int grp = (warp >> 2) - 1; grp < 4; grp += 3) {
-                    uint32_t ry[16];
-                    tmem_ld16(tbase + lane_base + T_Z + 16u * grp, ry);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float vv = zero_v ? 0.0f
-                                                : __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
-                                                      vt + sw128((uint32_t)(16 * grp + e), vb)));
-                        ry[e] = __float_as_uint(to_tf32(vv - __uint_as_float(ry[e])));
-                    }
-                    tmem_st16(tbase + lane_base + T_Z + 16u * grp, ry);
-                }
-                tmem_wait_st();
             }
         }
+        if (tid == 0) z_ok = mbar_wait(bar_v, ld_par) && mbar_wait(bar_y, y_phase & 1);
         ++v_done;
         ++y_phase;
         fence_async_smem();
         tc_fence_before();
         if (!__syncthreads_and(z_ok)) { failed = true; break; }
         tc_fence_after();
-        if (ci + 1 < nchunks) {                      // v consumed: prefetch the next chunk's
-            if (tid == 0) issue_loads(ci + 1, 4);
-            note_loads(4);
-        }
 
-        // ================================================= Vn^T = Z^T T'^T (tf32, A from TMEM), then rounded to tf32
+        // ================================================= Vn^T = V^T T'^T + (-Y)^T T'^T, then rounded to tf32
+        // (bf16 with v as the MN-major A operand from its TMA tile, then tf32 with
+        // -Y^T from TMEM, into one accumulator)
         ++mma_issued;
         if (warp == 0) {
+            if (!zero_v) {                         // (a unit that treats v as zero skips T' V)
+#pragma unroll
+                for (int s = 0; s < 4; ++s)        // K = 64 tokens in steps of 16
+                    if (leader) mma_bf16_ss(tbase + T_VN, at(d_mnv, OFF_V + 2048u * s), at(d_k16, OFF_TPB + 32u * s), id_u, s > 0);
+            }
 #pragma unroll
             for (int s = 0; s < 8; ++s) {          // K = 64 tokens in steps of 8
                 const uint32_t kb = (uint32_t)(s >> 2), koff = (uint32_t)(s & 3) * 32u;
-                if (leader) mma_tf32_ts(tbase + T_VN, tbase + T_Z + 8u * s, at(d_k16, OFF_TP + kb * 8192u + koff), id_vn, s > 0);
+                if (leader) mma_tf32_ts(tbase + T_VN, tbase + T_Z + 8u * s, at(d_k16, OFF_TP + kb * 8192u + koff), id_vn,
+                                        (!zero_v || s > 0) ? 1u : 0u);
             }
             if (leader) mma_commit(bar_mma);
         }
         if (!wait_mma()) { failed = true; break; }
+        if (ci + 1 < nchunks) {                      // v consumed: prefetch the next chunk's
+            if (tid == 0) issue_loads(ci + 1, 4);
+            note_loads(4);
+        }
         {
             uint32_t rv[16];
             tmem_ld16(tbase + lane_base + T_VN + cq * 16, rv);

@@ -18,9 +18,11 @@ which is exact: g = 0, beta = 0, k = 0 make a padded token the identity):
   T = (I + A_kk)^-1   (16x16 diagonal blocks by substitution, then block merges)
   W = T (beta * k * Gt * D[b(i),0]),   U = T (beta * v)
   per chunk, with the carried state S:
-     Vn = U - W S                       (form "wy")
-        = T' (V - (k Gt D[b(i),0]) S)   (form "z", T' = T Diag(beta): what the
-                                         tensor-core kernel computes)
+     Vn = U - W S                        (form "wy")
+        = T' (V - (k Gt D[b(i),0]) S)    (form "z", T' = T Diag(beta))
+        = T' V - T' ((k Gt D[b(i),0]) S) (form "split": the two products with their
+                                          own operand precisions, as the
+                                          tensor-core kernel accumulates them)
      O  = scale ((q * Gt * D[b(i),0]) S + A_qk Vn)
      S  = Diag(D[nb,0]) S + K^(nb)^T Vn        (K^(nb) = k_j exp(G_{C-1} - G_j))
 
@@ -73,10 +75,10 @@ _ROUND = {"bf16": _bf16, "tf32": _tf32, "tf32t": _tf32_trunc,
 # operand -> storage precision in the tcgen05 kernel, and the form of its V_new
 KERNEL_PREC = {
     "Arow": "tf32t", "Acol": "tf32t",     # q~, k~ and K^(b) for A_qk / A_kk
-    "Aqk": "tf32", "T": "tf32t", "Z": "tf32", "Vn": "tf32", "Khat": "tf32",
+    "Aqk": "tf32", "T": "tf32t", "TV": "bf16", "Y": "tf32t", "Vn": "tf32", "Khat": "tf32",
     "KG": "bf16", "S": "bf16", "QG": "bf16",
 }
-KERNEL_FORM = "z"
+KERNEL_FORM = "split"
 
 
 def _block_inverse(A, sub=16):
@@ -157,6 +159,10 @@ def chunked_kda(q, k, v, g, beta, S0=None, scale=None, gate=None, g_floor=-5.0,
             if form == "z":
                 Z = rb("Z", vc - rb("KG", kc * Gt * Dq) @ Sb)
                 Vn = rb("Vn", Tb @ Z)
+            elif form == "split":
+                T_raw = _block_inverse(A_kk, sub) * bc[None, :]
+                Y = rb("Y", rb("KG", kc * Gt * Dq) @ Sb)
+                Vn = rb("Vn", rb("TV", T_raw) @ vc - Tb @ Y)
             else:
                 W = rb("W", Tb @ rb("KG", kc * Gt * Dq))
                 U = Tb @ vc

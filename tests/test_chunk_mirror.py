@@ -22,7 +22,7 @@ def _inputs(rng, T, H, d, g_mode="softplus"):
     return q, k, v, g, beta
 
 
-@pytest.mark.parametrize("form", ["wy", "z"])
+@pytest.mark.parametrize("form", ["wy", "z", "split"])
 @pytest.mark.parametrize("C", [16, 32, 64])
 @pytest.mark.parametrize("g_mode", ["softplus", "floor"])
 def test_mirror_matches_oracle_fp64(C, g_mode, form):
