@@ -58,9 +58,11 @@ constexpr uint32_t OFF_QKG1 = 24576;      // pass 1: channels 64-127
 constexpr uint32_t QKG_Q = 0, QKG_K = 8192, QKG_G = 16384;
 constexpr uint32_t OFF_V = 49152;         // v: MN-major A operand, 2 MN blocks x 8 KB
 constexpr uint32_t OFF_INTRA = 65536;     // 72 KB, reused after the A MMAs
-//   during prep / A MMAs (per pass of 64 channels = 2 tf32 K-blocks):
+//   during prep / A MMAs (per pass of 64 channels):
 constexpr uint32_t OFF_XT = OFF_INTRA;             // X~ [128 rows x 64 ch] tf32 K-major: 2 x 16 KB
-constexpr uint32_t OFF_KB = OFF_INTRA + 32768;     // K^(b), b = 0..3, packed rows 16(b+1): 40 KB
+constexpr uint32_t OFF_KD = OFF_INTRA + 32768;     // Kbar [64 rows j x 64 ch] tf32 K-major: 2 x 8 KB
+constexpr uint32_t OFF_XB = OFF_INTRA + 49152;     // X~ rows 32-127 (blocks 1-3) bf16 K-major: 12 KB
+constexpr uint32_t OFF_KO = OFF_INTRA + 61440;     // K^(b) rows j < 16 b, b = 1..3, bf16 K-major: 12 KB
 //   after the A MMAs:
 constexpr uint32_t OFF_SCR = OFF_INTRA;            // A_kk -> T, fp32 [64][68]
 constexpr uint32_t SCR_LD = 68;                    // 16-byte aligned rows
@@ -86,21 +88,22 @@ constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024; // slack for aligning the bas
 static_assert(OFF_TP % 1024 == 0 && OFF_TP + 16384 <= OFF_XS && OFF_XS + 4096 <= OFF_TPB &&
               OFF_TPB % 1024 == 0 && OFF_TPB + 8192 <= OFF_INTRA + 73728, "post-MMA tiles fit the intra region");
 static_assert((OFF_KG - OFF_QG) % 16 == 0, "Q e^G | K e^G as one MN-major operand");
-static_assert(OFF_KB + 40960 <= OFF_INTRA + 73728, "intra tiles fit");
+static_assert(OFF_KO + 12288 == OFF_INTRA + 73728, "intra tiles fit");
 static_assert(SMEM_ALLOC <= 232448, "fits in 227 KB");
 
-// K^(b) packed layout: tile b has 16(b+1) valid rows; its two 128-byte
-// K-blocks are stored back to back.  The MMA (M = 64) reads 64 rows from each
-// K-block start; rows past the valid ones read neighbouring bytes of this
-// area, which only feed accumulator rows that are never used.
-__host__ __device__ constexpr uint32_t kb_rows(int b) { return 16u * (b + 1); }
-// start of tile b: sum over b' < b of 2 K-blocks x 16(b'+1) rows x 128 B
-__host__ __device__ constexpr uint32_t kb_base(int b) { return 2048u * (uint32_t)b * (uint32_t)(b + 1); }
-static_assert(kb_base(1) == 4096u && kb_base(2) == 12288u && kb_base(3) == 24576u, "packing");
-static_assert(kb_base(3) + 128u * 64u + 64u * 128u <= 40960u, "K^(b) reads stay in the area");
+// Off-diagonal column operands: tile b (b = 1..3) holds K^(b) rows j < 16 b
+// (tokens of the blocks before b) in bf16, one 128-byte K-block of 64 channels;
+// tiles are packed back to back.  The MMA (M = 64) reads 64 rows from a tile's
+// start; rows past the valid ones read neighbouring bytes (the next tile, or
+// for b = 3 the first 2 KB after the intra region), which only feed
+// accumulator rows that are never used.
+__host__ __device__ constexpr uint32_t ko_base(int b) { return 1024u * (uint32_t)b * (uint32_t)(b - 1); }
+static_assert(ko_base(1) == 0u && ko_base(2) == 2048u && ko_base(3) == 6144u, "packing");
+static_assert(OFF_KO + ko_base(3) + 64u * 128u <= OFF_QG + 16384u, "K^(b) reads stay in shared memory");
 
 // ---- TMEM columns
-constexpr uint32_t T_DB = 0;      // A MMAs: 4 x 32 columns (M = 64 layout)
+constexpr uint32_t T_DD = 0;      // diagonal A MMA [64 j x 128 X~ rows] (M = 64 layout)
+constexpr uint32_t T_DO = 128;    // off-diagonal A MMAs: 3 x 32 columns (blocks 1-3)
 constexpr uint32_t T_O2 = 0;      // (A_qk Vn)^T   [v x i]   } one MMA (N = 192), after the
 constexpr uint32_t T_DS = 64;     // dS^T          [v x c]   } A readout and Vn
 constexpr uint32_t T_VN = 192;    // Vn^T = V^T T'^T - Y^T T'^T, then its tf32 copy (A operand)
@@ -314,7 +317,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t kbyte = (uint32_t)(cA & 31) * 4u;
     const uint32_t sw_lane = ((((kbyte >> 4) & 7u) ^ (uint32_t)gq) << 4) + (kbyte & 15u);
     const uint32_t xt_lane = OFF_XT + kblk * 16384u + sw_lane;
-    const uint32_t kb_lane = OFF_KB + sw_lane;
+    const uint32_t kd_lane = OFF_KD + kblk * 8192u + sw_lane;
+    // the same for the bf16 tiles (one 128-byte K-block of 64 channels)
+    const uint32_t xb_lane = OFF_XB + (((((uint32_t)cA * 2u) >> 4) ^ (uint32_t)gq) << 4) + (((uint32_t)cA * 2u) & 15u);
     // constant A fragments of the prefix-sum products (bf16 1.0 = 0x3F80):
     //   a_blk: 16x16 lower triangle with diagonal;  a_ref[kb]: rows m < 4 select block kb <= m
     uint32_t a_blk[4];
@@ -435,7 +440,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     };
 
     // MMA descriptors that do not depend on the chunk (start addresses advance per K-step)
-    const uint32_t id_a = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 64, 32);
+    const uint32_t id_d = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 64, 128);
+    const uint32_t id_o = instr_desc(FMT_BF16, K_MAJOR, K_MAJOR, 64, 32);
     const uint32_t id_1 = instr_desc(FMT_BF16, K_MAJOR, MN_MAJOR, 128, 128);
     const uint32_t id_vn = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 128, 64);
     const uint32_t id_u = instr_desc(FMT_BF16, MN_MAJOR, K_MAJOR, 128, 64);
@@ -446,23 +452,34 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     auto at = [](uint64_t tmpl, uint32_t byte_off) -> uint64_t {     // same descriptor, moved start
         return tmpl + (uint64_t)(byte_off >> 4);
     };
-    // Warp 0: the A MMAs of blocks [b0, b1) of a prep pass (tf32, 8 K-steps of 8
-    // channels each); when the pass's last block is issued: commit, then this
-    // pass's half of [O1 | Y]^T = S^T [Q e^G | K e^G]^T (bf16, A = S^T from TMEM),
-    // which runs behind the A MMAs, off the critical path.
-    auto issue_a = [&](int pass_, int b0, int b1) {
+    // Warp 0: the A MMAs of a prep pass, in two parts.
+    //   part 0: the diagonal product D[j, n] = Kbar_j . X~_n over the pass's 64
+    //           channels (tf32, M = 64, N = 128: every block against every
+    //           block, of which the diagonal 16 x 32 tiles are used), and the
+    //           off-diagonal product of block 1;
+    //   part 1: the off-diagonal products of blocks 2 and 3 (bf16, M = 64, N = 32:
+    //           K^(b) rows j < 16 b against X~ rows of block b); then commit, and
+    //           this pass's half of [O1 | -Y]^T = S^T [Q e^G | -K e^G]^T (bf16, A =
+    //           S^T from TMEM), which runs behind the A MMAs, off the critical path.
+    auto issue_a = [&](int pass_, int part) {
+        if (part == 0) {
 #pragma unroll
-        for (int bb = 0; bb < NB; ++bb) {
-            if (bb < b0 || bb >= b1) continue;
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
+            for (int s = 0; s < 8; ++s) {          // tf32 K-steps of 8 channels
                 const uint32_t kb = (uint32_t)(s >> 2), koff = (uint32_t)(s & 3) * 32u;
-                const uint64_t ad = at(d_k16, OFF_KB + kb_base(bb) + kb * kb_rows(bb) * 128u + koff);
-                const uint64_t bd = at(d_k16, OFF_XT + kb * 16384u + 32u * bb * 128u + koff);
-                if (leader) mma_tf32_ss(tbase + T_DB + 32 * bb, ad, bd, id_a, (pass_ > 0 || s > 0) ? 1u : 0u);
+                if (leader) mma_tf32_ss(tbase + T_DD, at(d_k16, OFF_KD + kb * 8192u + koff),
+                                        at(d_k16, OFF_XT + kb * 16384u + koff), id_d, (pass_ > 0 || s > 0) ? 1u : 0u);
             }
         }
-        if (b1 == NB) {
+#pragma unroll
+        for (int bo = 1; bo < NB; ++bo) {
+            if ((bo == 1) != (part == 0)) continue;
+#pragma unroll
+            for (int s = 0; s < 4; ++s)            // bf16 K-steps of 16 channels
+                if (leader) mma_bf16_ss(tbase + T_DO + 32u * (bo - 1), at(d_k16, OFF_KO + ko_base(bo) + 32u * s),
+                                        at(d_k16, OFF_XB + 32u * (bo - 1) * 128u + 32u * s), id_o,
+                                        (pass_ > 0 || s > 0) ? 1u : 0u);
+        }
+        if (part == 1) {
             if (leader) mma_commit(bar_mma);
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
@@ -530,7 +547,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ldsm_x4_trans(gf[1], raw + QKG_G + sw128((uint32_t)(32 + lane), (uint32_t)nt * 16u));
                 if (pass == 1 && warp == 0) {          // the rest of the pass-0 A MMAs
                     __syncwarp();
-                    issue_a(0, 2, NB);
+                    issue_a(0, 1);
                     __syncwarp();
                 }
                 uint32_t gi[2][4];                     // indicator g <= fb (floor not a bf16 value)
@@ -652,8 +669,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     ++mma_phase;
                     tc_fence_after();
                 }
-                // (4) the A-MMA operands: X~ rows (q~ at 32 b + r, k~ at 32 b + 16 + r) and the
-                //     K^(b') copies, b' >= b (tf32 operands: the MMA reads the leading 19 bits)
+                // (4) the A-MMA operands: X~ rows (q~ at 32 b + r, k~ at 32 b + 16 + r) and Kbar
+                //     (tf32 operands of the diagonal product: the MMA reads the leading 19
+                //     bits), X~ rows of blocks 1-3 again in bf16, and the K^(b') copies,
+                //     b' > b, in bf16 for the off-diagonal products
 #pragma unroll
                 for (int bb = 0; bb < 2; ++bb) {
                     const int b = 2 * mp + bb;
@@ -672,11 +691,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         const uint32_t xrow = (uint32_t)(32 * b + 8 * hr) + (uint32_t)gq;
                         *reinterpret_cast<float2 *>(sm + xt_lane + xrow * 128u) = qt[bb][hr];
                         *reinterpret_cast<float2 *>(sm + xt_lane + (xrow + 16u) * 128u) = kt[bb][hr];
+                        *reinterpret_cast<float2 *>(sm + kd_lane + i * 128u) = kbar[bb][hr];
+                        if (b > 0) {
+                            *reinterpret_cast<uint32_t *>(sm + xb_lane + (xrow - 32u) * 128u) = pack_bf16(qt[bb][hr].x, qt[bb][hr].y);
+                            *reinterpret_cast<uint32_t *>(sm + xb_lane + (xrow - 16u) * 128u) = pack_bf16(kt[bb][hr].x, kt[bb][hr].y);
+                        }
 #pragma unroll
-                        for (int m = 0; m < NB; ++m) {
-                            if (m < b) continue;
-                            const float2 v = m == b ? kbar[bb][hr] : __fmul2_rn(kbar[bb][hr], dfac[m]);
-                            *reinterpret_cast<float2 *>(sm + kb_lane + kb_base(m) + kblk * kb_rows(m) * 128u + i * 128u) = v;
+                        for (int m = 1; m < NB; ++m) {
+                            if (m <= b) continue;
+                            const float2 v = __fmul2_rn(kbar[bb][hr], dfac[m]);
+                            *reinterpret_cast<uint32_t *>(sm + xb_lane - OFF_XB + OFF_KO + ko_base(m) + i * 128u) = pack_bf16(v.x, v.y);
                         }
                     }
                 }
@@ -753,9 +777,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (pass == 0 && o_row >= 0) store_o_tile();
             }
             __syncwarp();
-            // pass 0: blocks 0-1 now, blocks 2-3 early in warp 0's pass-1 prep (a long
-            // run of issues stalls the issuing warp); pass 1: everything now
-            issue_a(pass, 0, pass == 0 ? 2 : NB);
+            // pass 0: part 0 now, part 1 early in warp 0's pass-1 prep (a long run of
+            // issues stalls the issuing warp); pass 1: everything now
+            issue_a(pass, 0);
+            if (pass == 1) issue_a(1, 1);
         }
         if (pass == 0) o_row = -1;
         if (pass == 0) continue;
@@ -763,11 +788,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (tid == 0) bulk_wait_read();        // the staged output tile has been read
         if (!wait_mma()) { failed = true; break; }
 
-        // ================================================= A readout: warp (lq, cq): rows j, row block b = cq
+        // ================================================= A readout: warp (lq, cq): rows j of block lq, rows i of block cq
         {
+            // rows j of block lq against X~ rows of block cq: the diagonal product for
+            // lq == cq, block cq's off-diagonal product for lq < cq (lq > cq: j > i, masked)
+            const uint32_t acol = lq < cq ? T_DO + 32u * (uint32_t)(cq - 1) : T_DD + 32u * (uint32_t)cq;
             uint32_t ra[16], rk[16];
-            tmem_ld16(tbase + lane_base + T_DB + 32 * cq, ra);
-            tmem_ld16(tbase + lane_base + T_DB + 32 * cq + 16, rk);
+            tmem_ld16(tbase + lane_base + acol, ra);
+            tmem_ld16(tbase + lane_base + acol + 16, rk);
             tmem_wait_ld();
             if (lane < 16) {
                 const int j = lq * 16 + lane;

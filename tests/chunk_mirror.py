@@ -74,7 +74,8 @@ _ROUND = {"bf16": _bf16, "tf32": _tf32, "tf32t": _tf32_trunc,
 
 # operand -> storage precision in the tcgen05 kernel, and the form of its V_new
 KERNEL_PREC = {
-    "Arow": "tf32t", "Acol": "tf32t",     # q~, k~ and K^(b) for A_qk / A_kk
+    "Arow": "tf32t", "Acol": "tf32t",     # q~, k~ and Kbar of the diagonal A blocks
+    "Aoff": "bf16",                       # q~, k~ and K^(b) of the off-diagonal A blocks
     "Aqk": "tf32", "T": "tf32t", "TV": "bf16", "Y": "tf32t", "Vn": "tf32", "Khat": "tf32",
     "KG": "bf16", "S": "bf16", "QG": "bf16",
 }
@@ -147,9 +148,16 @@ def chunked_kda(q, k, v, g, beta, S0=None, scale=None, gate=None, g_floor=-5.0,
                 rows = slice(b * sub, (b + 1) * sub)
                 # rows j of K^(b) past block b overflow; they only meet masked (j > i) entries
                 with np.errstate(over="ignore", invalid="ignore"):
-                    colop = rb("Acol", np.where(blk <= b, 1.0, 0.0)[:, None] * np.nan_to_num(Kb[b], posinf=0.0))
+                    colraw = np.where(blk <= b, 1.0, 0.0)[:, None] * np.nan_to_num(Kb[b], posinf=0.0)
+                colop = rb("Acol", colraw)
                 A_qk[rows] = Qt[rows] @ colop.T
                 A_kk[rows] = Kt[rows] @ colop.T
+                if "Aoff" in prec:
+                    # off-diagonal blocks (j in blocks < b) from their own operand precision
+                    off = slice(0, b * sub)
+                    qo, ko, co = (_ROUND[prec["Aoff"]](x) for x in (qc[rows] * Gt[rows], kc[rows] * Gt[rows], colraw[off]))
+                    A_qk[rows, off] = qo @ co.T
+                    A_kk[rows, off] = ko @ co.T
             ii, jj = np.meshgrid(np.arange(C), np.arange(C), indexing="ij")
             A_qk = np.where(jj <= ii, A_qk, 0.0)
             A_kk = np.where(jj < ii, A_kk, 0.0) * bc[:, None]
