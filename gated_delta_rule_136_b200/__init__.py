@@ -2,7 +2,7 @@
 in-place decode behind a C ABI (``include/kda.h``), with a thin PyTorch
 binding.  See ``kda.chunk_fwd`` and ``kda.decode_step``."""
 from .kda import (KDAError, chunk_fwd, decode_step, device_status, load_library,  # noqa: F401
-                  workspace_size)
+                  selftest_bounded_wait, workspace_size)
 
 __all__ = ["chunk_fwd", "decode_step", "device_status", "load_library", "workspace_size",
-           "KDAError"]
+           "selftest_bounded_wait", "KDAError"]

@@ -481,6 +481,26 @@ kda_status kda_decode_step(const kda_decode_desc *desc, const void *q, const voi
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+namespace {
+// One warp waits, bounded, on an mbarrier whose phase nothing completes.
+__global__ void selftest_wait_kernel(uint32_t max_polls) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        kda::tc::mbar_init(&bar, 1);
+        kda::tc::mbar_fence_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)kda::tc::mbar_wait(&bar, 0, max_polls);
+    __syncthreads();
+}
+}  // namespace
+
+kda_status kda_selftest_bounded_wait(int32_t max_polls, cudaStream_t stream) {
+    if (max_polls < 1 || max_polls > 65536) return KDA_ERR_INVALID_ARG;
+    selftest_wait_kernel<<<1, 32, 0, stream>>>((uint32_t)max_polls);
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 kda_status kda_get_device_status(cudaStream_t stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
     unsigned int word = 0, zero = 0;

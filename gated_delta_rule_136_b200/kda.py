@@ -25,7 +25,7 @@ KDA_BF16, KDA_FP32 = 0, 1
 # Every function include/kda.h declares.
 EXPORTED_SYMBOLS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
                     "kda_get_device_status", "kda_status_string", "kda_version",
-                    "kda_chunk_fwd_noalloc")
+                    "kda_chunk_fwd_noalloc", "kda_selftest_bounded_wait")
 NOALLOC_MAX_SEQS = 65536   # KDA_NOALLOC_MAX_SEQS in include/kda.h
 
 
@@ -79,6 +79,8 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_status_string.restype = ctypes.c_char_p
         lib.kda_version.restype = ctypes.c_int32
+        lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_int32, vp]
+        lib.kda_selftest_bounded_wait.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -252,6 +254,17 @@ def device_status(device=None) -> int:
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     with torch.cuda.device(dev):
         return int(lib.kda_get_device_status(_stream_handle(dev)))
+
+
+def selftest_bounded_wait(max_polls: int = 1024, device=None) -> int:
+    """``kda_selftest_bounded_wait``: one bounded device-side wait that runs out
+    (nothing completes its barrier); returns the launch status.  The timeout it
+    records is read, and cleared, by :func:`device_status`."""
+    _require_cuda()
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return int(lib.kda_selftest_bounded_wait(int(max_polls), _stream_handle(dev)))
 
 
 def _noalloc_fn(lib):

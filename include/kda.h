@@ -191,6 +191,18 @@ kda_status kda_chunk_fwd_noalloc(const kda_fwd_desc *desc,
  */
 kda_status kda_get_device_status(cudaStream_t stream);
 
+/*
+ * Diagnostic (the pages have no counterpart): runs one bounded device-side
+ * wait on a barrier that nothing completes, with the same wait primitive the
+ * prefill kernels use, so that the timeout path can be exercised without a
+ * hang or a fault.  The wait gives up after `max_polls` polls (1 .. 65536),
+ * sets the timeout bit of the device error word and the kernel returns; read
+ * it with kda_get_device_status (which reports KDA_ERR_TIMEOUT and clears
+ * it).  Returns KDA_ERR_INVALID_ARG for a poll count outside that range,
+ * KDA_ERR_CUDA if the launch fails, else KDA_OK.
+ */
+kda_status kda_selftest_bounded_wait(int32_t max_polls, cudaStream_t stream);
+
 /* Static, human-readable name of a status code. */
 const char *kda_status_string(kda_status status);
 

@@ -137,3 +137,9 @@ def test_decode_validation(lib):
     assert _dec(lib, d, o=A + 8 * MB + 256) == 1      # o inside S
     assert _dec(lib, d, S=A + 8 * MB + 4) == 1        # S not 16-byte aligned
     assert _dec(lib, d, gate=A + 8 * MB) == 1         # gate inside S
+
+
+@pytest.mark.parametrize("polls", [0, -1, 65537])
+def test_selftest_rejects_bad_poll_counts(lib, polls):
+    """Checked on the host before any launch, so this runs without a GPU."""
+    assert lib.kda_selftest_bounded_wait(polls, None) == 1   # KDA_ERR_INVALID_ARG
