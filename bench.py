@@ -244,7 +244,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=DEC_STEPS)
     ap.add_argument("--all-workloads", action="store_true",
                     help="also time the varlen (64 x [512, 32768] x 64 heads) and the "
-                         "1M-token x 32-head floor-stress prefill")
+                         "1M-token x 32-head floor-stress prefill, and the headline prefill "
+                         "with state snapshots every 512 tokens")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     B, T, H = args.batch, args.seqlen, args.heads
@@ -452,6 +453,40 @@ def main():
                             "roofline_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
             del w, ow, Sw, wsw
             torch.cuda.empty_cache()
+
+        # the headline prefill with state snapshots every 512 tokens (prefix-cache hook)
+        from gated_delta_rule_136_b200 import chunk_fwd_snapshots
+        w = inputs.prefill_inputs([T] * B, H=H, dk=DK, dv=DV, device=dev, seed=rank)
+        interval = 512
+        run = lambda: chunk_fwd_snapshots(w["q"], w["k"], w["v"], w["g"], w["beta"], interval,
+                                          cu_seqlens=w["cu_seqlens"],
+                                          cu_seqlens_host=w["cu_seqlens_host"])
+        for _ in range(2):
+            run()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        tw0 = time.time()
+        a.record(stream)
+        for _ in range(reps):
+            run()
+        b.record(stream)
+        barrier()
+        if sampler:
+            sampler.mark(tw0, time.time())
+        if device_status(dev) != 0:
+            raise RuntimeError("device error word after the snapshot prefill")
+        ms = max_over_ranks(a.elapsed_time(b)) / reps
+        nsnap = B * (T // interval)
+        byts = B * T * H * bytes_per_token_head() + B * H * DK * DV * 4 + nsnap * H * DK * DV * 4
+        others[f"prefill B={B} T={T} H={H} with state snapshots every {interval} tokens"] = {
+            "tokens": B * T, "ms": ms, "tokens_per_s": world * B * T / (ms / 1e3),
+            "snapshot_bytes": nsnap * H * DK * DV * 4, "alg_gbs": byts / (ms / 1e3) / 1e9,
+            "roofline_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "note": "timed through the Python binding, which allocates the snapshot buffer and "
+                    "uploads the slot table on every call"}
+        del w
+        torch.cuda.empty_cache()
 
     if sampler:
         sampler.stop()

@@ -62,6 +62,7 @@ struct SimtParams {
     float *S_T;
     int32_t num_heads;
     float scale, g_floor;
+    SnapOut snap;
 };
 
 template <int DK, int DV, typename TIO>
@@ -270,6 +271,12 @@ __global__ void __launch_bounds__(2 * DV, 1) chunk_simt_kernel(SimtParams p)
                 acc = fmaf(kh.w, vn[4 * b + 3], acc);
             }
             S[r] = acc;
+        }
+        const int64_t slot = snap_slot(p.snap, n, c0 + L - t_begin);
+        if (slot >= 0) {
+#pragma unroll
+            for (int r = 0; r < RH; ++r)
+                p.snap.states[((slot * H + h) * DK + half * RH + r) * DV + vcol] = S[r];
         }
         __syncthreads();
     }

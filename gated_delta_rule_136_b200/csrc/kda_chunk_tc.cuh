@@ -124,6 +124,8 @@ struct TcUnit {
     const float *S0;       // [dk x dv] start state or nullptr (zeros / identity)
     float *S_out;          // [dk x dv] final state or nullptr
     int32_t head, flags;
+    int32_t seq;           // sequence index (snapshot slots)
+    int64_t seq_start;     // the sequence's first token (snapshot positions)
 };
 
 struct TcParams {
@@ -136,6 +138,7 @@ struct TcParams {
     int32_t num_heads;
     float scale, g_floor;
     const TcUnit *units;   // when set, block b runs units[b] instead of a (sequence, head)
+    SnapOut snap;          // state snapshots (units with UNIT_STORE_O only)
 };
 
 // byte offset of (row, byte kb within a 128-byte K-block row) in a swizzled block
@@ -255,6 +258,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 
+// SNAP: the variant that stores state snapshots (TcParams::snap); the other
+// compiles without that code.
+template <bool SNAP>
 __global__ void __launch_bounds__(NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
@@ -278,10 +284,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const float *S0p;
     float *S_outp;
     int32_t flags;
+    int snap_n;                          // sequence index and first token, for snapshots
+    int64_t seq_start;
     if (p.units) {
         const TcUnit u = p.units[blockIdx.x];
         hh = u.head; t_begin = u.t_begin; t_end = u.t_end;
         S0p = u.S0; S_outp = u.S_out; flags = u.flags;
+        snap_n = u.seq; seq_start = u.seq_start;
     } else {
         const int n_slot = blockIdx.x / H;
         hh = blockIdx.x % H;
@@ -291,6 +300,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         S0p = p.S0 ? p.S0 + unit * D * D : nullptr;
         S_outp = p.S_T ? p.S_T + unit * D * D : nullptr;
         flags = UNIT_STORE_O;
+        snap_n = n; seq_start = t_begin;
     }
     const bool store_o = (flags & UNIT_STORE_O) != 0;
     const bool zero_v = (flags & UNIT_ZERO_V) != 0;
@@ -725,6 +735,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             S[hq * 16 + e] = fmaf(gam[cq * 32 + hq * 16 + e], S[hq * 16 + e], __uint_as_float(rd[e]));
                     }
                     store_state_bf16();
+                    if (SNAP && store_o) {       // snapshot of the state after this chunk, if due
+                        const int64_t slot = snap_slot(p.snap, snap_n, t0p + Lp - seq_start);
+                        if (slot >= 0) {
+                            float *dst = p.snap.states + ((slot * H + hh) * D + cq * 32) * D + vlane;
+#pragma unroll
+                            for (int r = 0; r < 32; ++r) dst[r * D] = S[r];
+                        }
+                    }
                     uint32_t r1[16], r2[16];
                     tmem_ld16(tbase + lane_base + T_O1 + cq * 16, r1);
                     tmem_ld16(tbase + lane_base + T_O2 + cq * 16, r2);

@@ -23,4 +23,26 @@ __device__ __forceinline__ void st(__nv_bfloat16 *p, int64_t i, float x) { p[i] 
 
 __device__ __forceinline__ float sigmoidf(float z) { return 1.0f / (1.0f + expf(-z)); }
 
+// Snapshots of the state at token offsets that are multiples of `interval`
+// (the prefix-cache hook): slot base[n] + m - 1 of `states` ([total][H][dk][dv]
+// fp32) receives sequence n's state after its first m * interval tokens.
+struct SnapOut {
+    float *states;          // nullptr: no snapshots
+    const int64_t *base;    // [num_seqs + 1], caller-provided first slot per sequence
+    int64_t total;          // slots in `states`
+    int32_t interval;       // a positive multiple of the chunk
+};
+
+// Slot for the state after `rel` tokens of sequence n, or -1 if none is due.
+// A slot outside [0, total) records a bounds error and is skipped.
+__device__ __forceinline__ int64_t snap_slot(const SnapOut &sn, int n, int64_t rel) {
+    if (!sn.states || rel <= 0 || rel % sn.interval != 0) return -1;
+    const int64_t slot = sn.base[n] + rel / sn.interval - 1;
+    if (slot < 0 || slot >= sn.total) {
+        if (threadIdx.x == 0) raise_error(ERR_BOUNDS);
+        return -1;
+    }
+    return slot;
+}
+
 }  // namespace kda

@@ -271,14 +271,13 @@ cudaError_t launch_tc_units(const kda_fwd_desc &d, const void *q, const void *k,
         !encode_bf16_2d(&tg, g, rows, cols) || !encode_bf16_2d(&tv, v, rows, cols) ||
         !encode_bf16_2d(&to, p.o, rows, cols))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(kda::tck::chunk_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto kern = p.snap.states ? kda::tck::chunk_tc_kernel<true> : kda::tck::chunk_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kda::tck::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
     if (blocks == 0) return cudaSuccess;
-    kda::tck::chunk_tc_kernel<<<(unsigned)blocks, kda::tck::NT, kda::tck::SMEM_ALLOC, stream>>>(
-        tq, tk, tg, tv, to, p);
+    kern<<<(unsigned)blocks, kda::tck::NT, kda::tck::SMEM_ALLOC, stream>>>(tq, tk, tg, tv, to, p);
     return cudaGetLastError();
 }
 
@@ -287,14 +286,14 @@ cudaError_t launch_tc_units(const kda_fwd_desc &d, const void *q, const void *k,
 cudaError_t launch_prefill(const kda_fwd_desc &d, const void *q, const void *k, const void *v,
                            const void *g, const void *beta, const float *S0,
                            const int32_t *cu_seqlens, const int32_t *seq_order, const void *gate,
-                           void *o, float *S_T, cudaStream_t stream) {
+                           void *o, float *S_T, const kda::SnapOut &sn, cudaStream_t stream) {
     if (tc_path_applies(d, q, k, v, g, o)) {
         kda::tck::TcParams tp{beta, gate, S0, cu_seqlens, seq_order, o, S_T, d.num_heads, d.scale,
-                              d.g_floor, nullptr};
+                              d.g_floor, nullptr, sn};
         return launch_tc(d, q, k, v, g, tp, stream);
     }
     SimtParams p{q, k, v, g, beta, gate, S0, cu_seqlens, seq_order, o, S_T,
-                 d.num_heads, d.scale, d.g_floor};
+                 d.num_heads, d.scale, d.g_floor, sn};
     return d.io_dtype == KDA_BF16 ? dispatch_simt<__nv_bfloat16>(d.dk, d.dv, p, d.num_seqs, stream)
                                   : dispatch_simt<float>(d.dk, d.dv, p, d.num_seqs, stream);
 }
@@ -303,7 +302,7 @@ cudaError_t launch_prefill(const kda_fwd_desc &d, const void *q, const void *k, 
 cudaError_t launch_split(const kda_fwd_desc &d, const SegPlan &pl, const int32_t *cu,
                          const void *q, const void *k, const void *v, const void *g,
                          const void *beta, const float *S0, const void *gate, void *o, float *S_T,
-                         unsigned char *ws, cudaStream_t stream) {
+                         const kda::SnapOut &sn, unsigned char *ws, cudaStream_t stream) {
     using kda::tck::TcUnit;
     const WsLayout w = ws_layout(&d, pl);
     const int32_t N = d.num_seqs, H = d.num_heads;
@@ -322,7 +321,7 @@ cudaError_t launch_split(const kda_fwd_desc &d, const SegPlan &pl, const int32_t
             const float *s0 = S0 ? S0 + unit * DD : nullptr;
             float *st = S_T ? S_T + unit * DD : nullptr;
             if (P == 1) {
-                p2.push_back(TcUnit{t0, t1, s0, st, h, kda::tck::UNIT_STORE_O});
+                p2.push_back(TcUnit{t0, t1, s0, st, h, kda::tck::UNIT_STORE_O, n, t0});
                 continue;
             }
             float *base = mats + blk * (size_t)P * 3u * DD;
@@ -333,12 +332,12 @@ cudaError_t launch_split(const kda_fwd_desc &d, const SegPlan &pl, const int32_t
             for (int32_t sp = 0; sp < P; ++sp) {
                 const int64_t a = t0 + (int64_t)sp * pl.seglen[n];
                 const int64_t b = std::min<int64_t>(t1, a + pl.seglen[n]);
-                if (sp + 1 < P) p1.push_back(TcUnit{a, b, sp == 0 ? s0 : nullptr, Sloc(sp), h, 0});
+                if (sp + 1 < P) p1.push_back(TcUnit{a, b, sp == 0 ? s0 : nullptr, Sloc(sp), h, 0, n, t0});
                 if (sp >= 1 && sp + 1 < P)
                     p1.push_back(TcUnit{a, b, nullptr, Mp(sp), h,
-                                        kda::tck::UNIT_ZERO_V | kda::tck::UNIT_S0_IDENTITY});
+                                        kda::tck::UNIT_ZERO_V | kda::tck::UNIT_S0_IDENTITY, n, t0});
                 p2.push_back(TcUnit{a, b, sp == 0 ? s0 : Sin(sp), sp + 1 == P ? st : nullptr, h,
-                                    kda::tck::UNIT_STORE_O});
+                                    kda::tck::UNIT_STORE_O, n, t0});
             }
             jobs.push_back(kda::ScanJob{Sloc(0), Mp(0), Sin(0), (int64_t)(3u * DD), P});
         }
@@ -360,7 +359,7 @@ cudaError_t launch_split(const kda_fwd_desc &d, const SegPlan &pl, const int32_t
     if ((e = cudaMemcpyAsync(dj, jobs.data(), jobs.size() * sizeof(kda::ScanJob), cudaMemcpyHostToDevice,
                              stream)) != cudaSuccess)
         return e;
-    kda::tck::TcParams tp{beta, gate, nullptr, nullptr, nullptr, o, nullptr, H, d.scale, d.g_floor, d1};
+    kda::tck::TcParams tp{beta, gate, nullptr, nullptr, nullptr, o, nullptr, H, d.scale, d.g_floor, d1, sn};
     if (!p1.empty()) {
         tp.units = d1;
         if ((e = launch_tc_units(d, q, k, v, g, tp, (int64_t)p1.size(), stream)) != cudaSuccess) return e;
@@ -400,11 +399,12 @@ size_t kda_chunk_fwd_workspace_size(const kda_fwd_desc *desc, const int32_t *cu_
     return fwd_workspace_bytes(desc, cu_seqlens_host);
 }
 
-kda_status kda_chunk_fwd(const kda_fwd_desc *desc, const void *q, const void *k, const void *v,
-                         const void *g, const void *beta, const float *S0,
-                         const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
-                         const void *gate, void *o, float *S_T, void *workspace,
-                         size_t workspace_bytes, cudaStream_t stream) {
+namespace {
+kda_status chunk_fwd_impl(const kda_fwd_desc *desc, const kda_snapshots *snap, const void *q,
+                          const void *k, const void *v, const void *g, const void *beta,
+                          const float *S0, const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                          const void *gate, void *o, float *S_T, void *workspace,
+                          size_t workspace_bytes, cudaStream_t stream) {
     kda_status st = validate_fwd_desc(desc);
     if (st != KDA_OK) return st;
     st = validate_host_seqlens(desc, cu_seqlens_host);
@@ -427,6 +427,29 @@ kda_status kda_chunk_fwd(const kda_fwd_desc *desc, const void *q, const void *k,
     }
     if (overlaps(ro, rs)) return KDA_ERR_INVALID_ARG;
 
+    kda::SnapOut sn{nullptr, nullptr, 0, 64};
+    Range rsn{}, rsb{};
+    if (snap) {
+        if (snap->interval <= 0 || snap->interval % 64 != 0 || snap->total < 0) return KDA_ERR_INVALID_ARG;
+        if (snap->total > 0) {
+            if (!snap->states || !snap->base) return KDA_ERR_INVALID_ARG;
+            if (cu_seqlens_host) {               // the slots the sequences need must exist
+                int64_t need_slots = 0;
+                for (int32_t n = 0; n < d.num_seqs; ++n)
+                    need_slots += ((int64_t)cu_seqlens_host[n + 1] - cu_seqlens_host[n]) / snap->interval;
+                if (need_slots > snap->total) return KDA_ERR_INVALID_ARG;
+            }
+            rsn = range_of(snap->states, snap->total * H * d.dk * d.dv * 4);
+            rsb = range_of(snap->base, 8 * (int64_t)(d.num_seqs + 1));
+            for (const Range &r : ins)
+                if (overlaps(rsn, r)) return KDA_ERR_INVALID_ARG;
+            if (overlaps(rsn, ro) || overlaps(rsn, rs) || overlaps(rsb, ro) || overlaps(rsb, rs) ||
+                overlaps(rsb, rsn))
+                return KDA_ERR_INVALID_ARG;
+            sn = kda::SnapOut{snap->states, snap->base, snap->total, snap->interval};
+        }
+    }
+
     const size_t need = fwd_workspace_bytes(desc, cu_seqlens_host);
     if (need > 0) {
         if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
@@ -434,13 +457,14 @@ kda_status kda_chunk_fwd(const kda_fwd_desc *desc, const void *q, const void *k,
         const Range rw = range_of(workspace, (int64_t)need);
         for (const Range &r : ins)
             if (overlaps(rw, r)) return KDA_ERR_INVALID_ARG;
-        if (overlaps(rw, ro) || overlaps(rw, rs)) return KDA_ERR_INVALID_ARG;
+        if (overlaps(rw, ro) || overlaps(rw, rs) || overlaps(rw, rsn) || overlaps(rw, rsb))
+            return KDA_ERR_INVALID_ARG;
     }
 
     const SegPlan pl = plan_segments(d, cu_seqlens_host);
     if (pl.active && tc_path_applies(d, q, k, v, g, o)) {
         const cudaError_t e = launch_split(d, pl, cu_seqlens_host, q, k, v, g, beta, S0, gate, o, S_T,
-                                           static_cast<unsigned char *>(workspace), stream);
+                                           sn, static_cast<unsigned char *>(workspace), stream);
         return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     }
 
@@ -448,8 +472,29 @@ kda_status kda_chunk_fwd(const kda_fwd_desc *desc, const void *q, const void *k,
     cudaError_t e = kda::launch_plan_longest_first(cu_seqlens, d.num_seqs, seq_order, stream);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
 
-    e = launch_prefill(d, q, k, v, g, beta, S0, cu_seqlens, seq_order, gate, o, S_T, stream);
+    e = launch_prefill(d, q, k, v, g, beta, S0, cu_seqlens, seq_order, gate, o, S_T, sn, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+}  // namespace
+
+kda_status kda_chunk_fwd(const kda_fwd_desc *desc, const void *q, const void *k, const void *v,
+                         const void *g, const void *beta, const float *S0,
+                         const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                         const void *gate, void *o, float *S_T, void *workspace,
+                         size_t workspace_bytes, cudaStream_t stream) {
+    return chunk_fwd_impl(desc, nullptr, q, k, v, g, beta, S0, cu_seqlens, cu_seqlens_host, gate, o,
+                          S_T, workspace, workspace_bytes, stream);
+}
+
+kda_status kda_chunk_fwd_snapshots(const kda_fwd_desc *desc, const kda_snapshots *snap,
+                                   const void *q, const void *k, const void *v, const void *g,
+                                   const void *beta, const float *S0, const int32_t *cu_seqlens,
+                                   const int32_t *cu_seqlens_host, const void *gate, void *o,
+                                   float *S_T, void *workspace, size_t workspace_bytes,
+                                   cudaStream_t stream) {
+    if (!snap) return KDA_ERR_INVALID_ARG;
+    return chunk_fwd_impl(desc, snap, q, k, v, g, beta, S0, cu_seqlens, cu_seqlens_host, gate, o,
+                          S_T, workspace, workspace_bytes, stream);
 }
 
 kda_status kda_decode_step(const kda_decode_desc *desc, const void *q, const void *k,
@@ -601,6 +646,6 @@ extern "C" kda_status kda_chunk_fwd_noalloc(const kda_fwd_desc *desc, const void
     // so the previous call's contents never need clearing
     cudaError_t e = kda::launch_plan_longest_first(cu_seqlens, d.num_seqs, seq_order, stream);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
-    e = launch_prefill(d, q, k, v, g, beta, S0, cu_seqlens, seq_order, gate, o, S_T, stream);
+    e = launch_prefill(d, q, k, v, g, beta, S0, cu_seqlens, seq_order, gate, o, S_T, kda::SnapOut{nullptr, nullptr, 0, 64}, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

@@ -9,6 +9,7 @@ fallback, and a missing library or GPU raises.
 from __future__ import annotations
 
 import ctypes
+import itertools
 import math
 import threading
 
@@ -25,8 +26,15 @@ KDA_BF16, KDA_FP32 = 0, 1
 # Every function include/kda.h declares.
 EXPORTED_SYMBOLS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
                     "kda_get_device_status", "kda_status_string", "kda_version",
-                    "kda_chunk_fwd_noalloc", "kda_selftest_bounded_wait")
+                    "kda_chunk_fwd_noalloc", "kda_selftest_bounded_wait",
+                    "kda_chunk_fwd_snapshots")
 NOALLOC_MAX_SEQS = 65536   # KDA_NOALLOC_MAX_SEQS in include/kda.h
+
+
+class Snapshots(ctypes.Structure):
+    """``kda_snapshots``."""
+    _fields_ = [("interval", ctypes.c_int32), ("total", ctypes.c_int64),
+                ("base", ctypes.c_void_p), ("states", ctypes.c_void_p)]
 
 
 class KDAError(RuntimeError):
@@ -79,6 +87,10 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_status_string.restype = ctypes.c_char_p
         lib.kda_version.restype = ctypes.c_int32
+        lib.kda_chunk_fwd_snapshots.argtypes = [ctypes.POINTER(FwdDesc), ctypes.POINTER(Snapshots),
+                                                vp, vp, vp, vp, vp, vp, i32p, i32p, vp, vp, vp, vp,
+                                                sz, vp]
+        lib.kda_chunk_fwd_snapshots.restype = ctypes.c_int
         lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_int32, vp]
         lib.kda_selftest_bounded_wait.restype = ctypes.c_int
         _lib = lib
@@ -131,6 +143,27 @@ def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, scale=None, gate=None,
     single sequence or a fixed-length batch); ``cu_seqlens_host`` an optional
     host copy (list or CPU tensor) used to validate and plan.
     """
+    o, S_T, _, _ = _chunk_fwd(q, k, v, g, beta, S0, cu_seqlens, scale, gate, g_floor, chunk,
+                              cu_seqlens_host, output_final_state, out, final_state_out, workspace, 0)
+    return o, S_T
+
+
+def chunk_fwd_snapshots(q, k, v, g, beta, interval: int, S0=None, cu_seqlens=None, scale=None,
+                        gate=None, g_floor: float = -5.0, chunk: int = 0, cu_seqlens_host=None,
+                        output_final_state: bool = True):
+    """``kda_chunk_fwd_snapshots``: the prefill of :func:`chunk_fwd` plus the
+    state after every ``interval`` tokens of each sequence (a multiple of 64).
+    Returns ``(o, S_T, snaps, base)``: ``snaps`` fp32 [total, H, dk, dv] and
+    ``base`` int64 [N+1] (CPU) with sequence n's snapshots at rows
+    ``base[n] .. base[n+1]-1`` (after ``interval``, ``2 interval``, ... tokens).
+    ``cu_seqlens_host`` is required (a single sequence or a fixed-length
+    batch supplies its own)."""
+    return _chunk_fwd(q, k, v, g, beta, S0, cu_seqlens, scale, gate, g_floor, chunk,
+                      cu_seqlens_host, output_final_state, None, None, None, int(interval))
+
+
+def _chunk_fwd(q, k, v, g, beta, S0, cu_seqlens, scale, gate, g_floor, chunk, cu_seqlens_host,
+               output_final_state, out, final_state_out, workspace, snapshot_interval):
     _require_cuda()
     lib = load_library()
     batched = q.dim() == 4
@@ -173,6 +206,7 @@ def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, scale=None, gate=None,
     if scale is None:
         scale = 1.0 / math.sqrt(dk)
     host_arr = None
+    vals = None
     if cu_seqlens_host is not None:
         vals = [int(x) for x in (cu_seqlens_host.tolist() if hasattr(cu_seqlens_host, "tolist")
                                  else cu_seqlens_host)]
@@ -192,16 +226,33 @@ def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, scale=None, gate=None,
         _check(S_T, "final_state_out", (N, H, dk, dv), torch.float32, device)
     if ws_bytes > 0 and (workspace is None or workspace.numel() < ws_bytes):
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+    cu_ptr = ctypes.cast(ctypes.c_void_p(cu_seqlens.data_ptr()), ctypes.POINTER(ctypes.c_int32))
+    wsp = _ptr(workspace) if ws_bytes > 0 else None
+    snaps = base_host = None
     with torch.cuda.device(device):
-        st = lib.kda_chunk_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                               _ptr(S0), ctypes.cast(ctypes.c_void_p(cu_seqlens.data_ptr()),
-                                                     ctypes.POINTER(ctypes.c_int32)),
-                               host_arr, _ptr(gate), _ptr(o), _ptr(S_T),
-                               _ptr(workspace) if ws_bytes > 0 else None, ws_bytes,
-                               _stream_handle(device))
+        if snapshot_interval:
+            if cu_seqlens_host is None:
+                raise ValueError("snapshots need cu_seqlens_host")
+            counts = [(vals[n + 1] - vals[n]) // int(snapshot_interval) for n in range(N)]
+            base_host = torch.tensor([0] + list(itertools.accumulate(counts)), dtype=torch.int64)
+            total = int(base_host[-1])
+            snaps = torch.empty((total, H, dk, dv), dtype=torch.float32, device=device)
+            base_dev = base_host.to(device)
+            sd = Snapshots(int(snapshot_interval), total, base_dev.data_ptr() if total else None,
+                           snaps.data_ptr() if total else None)
+            st = lib.kda_chunk_fwd_snapshots(ctypes.byref(desc), ctypes.byref(sd), _ptr(q), _ptr(k),
+                                             _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), cu_ptr, host_arr,
+                                             _ptr(gate), _ptr(o), _ptr(S_T), wsp, ws_bytes,
+                                             _stream_handle(device))
+            where = "kda_chunk_fwd_snapshots"
+        else:
+            st = lib.kda_chunk_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                   _ptr(S0), cu_ptr, host_arr, _ptr(gate), _ptr(o), _ptr(S_T), wsp,
+                                   ws_bytes, _stream_handle(device))
+            where = "kda_chunk_fwd"
     if st != KDA_OK:
-        raise KDAError(st, "kda_chunk_fwd")
-    return o.view(out_shape), S_T
+        raise KDAError(st, where)
+    return o.view(out_shape), S_T, snaps, base_host
 
 
 def workspace_size(T, N, H, dk, dv, dtype=torch.bfloat16, chunk=0, g_floor=-5.0,

@@ -192,6 +192,42 @@ kda_status kda_chunk_fwd_noalloc(const kda_fwd_desc *desc,
 kda_status kda_get_device_status(cudaStream_t stream);
 
 /*
+ * State snapshots at token offsets (the prefix-cache hook: a cache of states
+ * at positions that are multiples of a hash granularity, Kimi K3 report
+ * digest, section 基础设施).  For sequence n and m = 1 .. floor(L_n /
+ * interval), slot base[n] + m - 1 of `states` receives the state after the
+ * sequence's first m * interval tokens (S0 included): fp32 [dk x dv] per
+ * head, laid out [total][num_heads][dk][dv].
+ *   interval: tokens between snapshots, a positive multiple of 64.
+ *   total:    slots in `states` (0: no snapshots are written).
+ *   base:     device array of num_seqs + 1 int64, normally the exclusive
+ *             prefix sum of floor(L_n / interval).  The kernels check every
+ *             slot against [0, total) and record KDA_ERR_DEVICE_BOUNDS
+ *             (kda_get_device_status) instead of writing outside it.
+ *   states:   device, caller-owned; must not overlap any other buffer.
+ */
+typedef struct {
+    int32_t interval;
+    int64_t total;
+    const int64_t *base;
+    float *states;
+} kda_snapshots;
+
+/*
+ * kda_chunk_fwd plus state snapshots (see kda_snapshots): the same
+ * arguments, checks and results, and in addition the snapshot states.  With
+ * cu_seqlens_host given, the slots the sequences need are also checked
+ * against snap->total on the host.  Returns KDA_ERR_INVALID_ARG for a null
+ * `snap`, a bad interval or overlapping snapshot buffers.
+ */
+kda_status kda_chunk_fwd_snapshots(const kda_fwd_desc *desc, const kda_snapshots *snap,
+                                   const void *q, const void *k, const void *v, const void *g,
+                                   const void *beta, const float *S0, const int32_t *cu_seqlens,
+                                   const int32_t *cu_seqlens_host, const void *gate, void *o,
+                                   float *S_T, void *workspace, size_t workspace_bytes,
+                                   cudaStream_t stream);
+
+/*
  * Diagnostic (the pages have no counterpart): runs one bounded device-side
  * wait on a barrier that nothing completes, with the same wait primitive the
  * prefill kernels use, so that the timeout path can be exercised without a

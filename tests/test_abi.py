@@ -143,3 +143,26 @@ def test_decode_validation(lib):
 def test_selftest_rejects_bad_poll_counts(lib, polls):
     """Checked on the host before any launch, so this runs without a GPU."""
     assert lib.kda_selftest_bounded_wait(polls, None) == 1   # KDA_ERR_INVALID_ARG
+
+
+def _snapfwd(lib, desc, snap, cu_host=None, o=A + 24 * MB):
+    cu_p = ctypes.cast(ctypes.c_void_p(A + 20 * MB), ctypes.POINTER(ctypes.c_int32))
+    return lib.kda_chunk_fwd_snapshots(ctypes.byref(desc), ctypes.byref(snap) if snap else None,
+                                       A, A + 4 * MB, A + 8 * MB, A + 12 * MB, A + 16 * MB, None,
+                                       cu_p, cu_host, None, o, None, A + 64 * MB, 1 << 20, None)
+
+
+def test_snapshots_validation(lib):
+    """Rejected on the host before any launch (fake pointers never touched)."""
+    d = _desc(num_seqs=2, total_tokens=300)
+    cu_host = (ctypes.c_int32 * 3)(0, 200, 300)           # 200 // 64 + 100 // 64 = 4 slots needed
+    ok = dict(interval=64, total=4, base=A + 80 * MB, states=A + 96 * MB)
+    assert _snapfwd(lib, d, None) == 1                                      # no descriptor
+    for bad in (dict(interval=0), dict(interval=32), dict(interval=-64), dict(total=-1),
+                dict(states=None), dict(base=None),
+                dict(total=3),                                              # fewer slots than needed
+                dict(states=A + 8 * MB),                                    # states inside v
+                dict(base=A + 24 * MB),                                     # base inside o
+                dict(states=A + 64 * MB)):                                  # states inside workspace
+        snap = kda.Snapshots(**{**ok, **bad})
+        assert _snapfwd(lib, d, snap, cu_host) == 1, bad
