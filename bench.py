@@ -244,8 +244,9 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=DEC_STEPS)
     ap.add_argument("--all-workloads", action="store_true",
                     help="also time the varlen (64 x [512, 32768] x 64 heads) and the "
-                         "1M-token x 32-head floor-stress prefill, and the headline prefill "
-                         "with state snapshots every 512 tokens")
+                         "1M-token x 32-head floor-stress prefill, the headline prefill "
+                         "with state snapshots every 512 tokens, and speculative-decode "
+                         "verify/commit rounds")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     B, T, H = args.batch, args.seqlen, args.heads
@@ -486,6 +487,48 @@ def main():
             "note": "timed through the Python binding, which allocates the snapshot buffer and "
                     "uploads the slot table on every call"}
         del w
+        torch.cuda.empty_cache()
+
+        # speculative decode: verify D = 4 draft tokens, commit 3, per round (decode batch)
+        from gated_delta_rule_136_b200 import spec_commit, spec_verify
+        Dd = 4
+        sd = inputs.prefill_inputs([Dd] * DEC_B, H=DEC_H, dk=DK, dv=DV, device=dev, seed=rank,
+                                   s0_std=0.02, gate=True)
+        xs = {n: sd[n].view(DEC_B, Dd, *sd[n].shape[1:]) for n in ("q", "k", "v", "g", "beta", "gate")}
+        Ssp = sd["S0"]
+        osp = torch.empty_like(xs["v"])
+        accd = torch.full((DEC_B,), 3, dtype=torch.int32, device=dev)
+
+        def spec_round():
+            spec_verify(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], Ssp, gate=xs["gate"], out=osp)
+            spec_commit(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], Ssp, accd)
+
+        for _ in range(args.warmup):
+            spec_round()
+        barrier()
+        rounds = 50
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tw0 = time.time()
+        a.record(stream)
+        for _ in range(rounds):
+            spec_round()
+        b.record(stream)
+        barrier()
+        if sampler:
+            sampler.mark(tw0, time.time())
+        if device_status(dev) != 0:
+            raise RuntimeError("device error word after speculative decode")
+        ms = max_over_ranks(a.elapsed_time(b)) / rounds
+        heads = DEC_B * DEC_H
+        byts = heads * (3 * DK * DV * 4 + Dd * (2 * (3 * DK + DV + 1) + 2 * DV + 2 * DV)
+                        + 3 * 2 * (3 * DK + DV + 1))
+        others[f"speculative decode batch={DEC_B} H={DEC_H}: verify {Dd} draft tokens, commit 3"] = {
+            "rounds_per_s": world * 1e3 / ms, "ms_per_round": ms,
+            "verified_tokens_per_s": world * DEC_B * Dd / (ms / 1e3),
+            "alg_gbs": byts / (ms / 1e3) / 1e9, "roofline_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "note": "the state crosses HBM three times per round (verify read, commit read and "
+                    "write) instead of twice per token"}
+        del sd, xs, Ssp, osp, accd
         torch.cuda.empty_cache()
 
     if sampler:

@@ -2,7 +2,7 @@
 in-place decode behind a C ABI (``include/kda.h``), with a thin PyTorch
 binding.  See ``kda.chunk_fwd`` and ``kda.decode_step``."""
 from .kda import (KDAError, chunk_fwd, chunk_fwd_snapshots, decode_step, device_status,  # noqa: F401
-                  load_library, selftest_bounded_wait, workspace_size)
+                  load_library, selftest_bounded_wait, spec_commit, spec_verify, workspace_size)
 
 __all__ = ["chunk_fwd", "chunk_fwd_snapshots", "decode_step", "device_status", "load_library", "workspace_size",
-           "selftest_bounded_wait", "KDAError"]
+           "selftest_bounded_wait", "spec_verify", "spec_commit", "KDAError"]

@@ -18,6 +18,7 @@
 #include "kda_chunk_simt.cuh"
 #include "kda_chunk_tc.cuh"
 #include "kda_decode.cuh"
+#include "kda_spec.cuh"
 #include "kda_plan.cuh"
 #include "kda_segment.cuh"
 
@@ -389,6 +390,49 @@ cudaError_t dispatch_decode(int dk, int dv, const DecodeParams &p, int64_t u, cu
     return launch_decode<64, 64, TIO>(p, u, s);
 }
 
+template <int DK, int DV, typename TIO, bool COMMIT>
+cudaError_t launch_spec(const kda::SpecParams &p, int64_t units, cudaStream_t stream) {
+    if (units > INT32_MAX) return cudaErrorInvalidConfiguration;
+    kda::spec_kernel<DK, DV, TIO, COMMIT><<<(unsigned)units, 256, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename TIO, bool COMMIT>
+cudaError_t dispatch_spec(int dk, int dv, const kda::SpecParams &p, int64_t u, cudaStream_t s) {
+    if (dk == 128 && dv == 128) return launch_spec<128, 128, TIO, COMMIT>(p, u, s);
+    if (dk == 128 && dv == 64) return launch_spec<128, 64, TIO, COMMIT>(p, u, s);
+    if (dk == 64 && dv == 128) return launch_spec<64, 128, TIO, COMMIT>(p, u, s);
+    return launch_spec<64, 64, TIO, COMMIT>(p, u, s);
+}
+
+// Checks shared by verify and commit: the descriptor, required pointers, and
+// that the state (and, for verify, the outputs) overlap no input.
+kda_status validate_spec(const kda_spec_desc *desc, const void *q, const void *k, const void *v,
+                         const void *g, const void *beta, const float *S, const void *gate,
+                         const void *o, const int32_t *accepted) {
+    if (!desc) return KDA_ERR_INVALID_ARG;
+    const kda_spec_desc &d = *desc;
+    if (d.batch < 1 || d.num_heads < 1 || d.dk <= 0 || d.dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (d.draft < 1 || d.draft > KDA_SPEC_MAX_DRAFT) return KDA_ERR_INVALID_ARG;
+    if (!supported_dim(d.dk) || !supported_dim(d.dv)) return KDA_ERR_UNSUPPORTED;
+    if (d.io_dtype != KDA_BF16 && d.io_dtype != KDA_FP32) return KDA_ERR_INVALID_ARG;
+    if (!std::isfinite(d.scale)) return KDA_ERR_INVALID_ARG;
+    if (!(d.g_floor >= kMinFloor && d.g_floor <= 0.0f)) return KDA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !g || !beta || !S) return KDA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(S) % 16 != 0) return KDA_ERR_INVALID_ARG;
+    const int64_t units = (int64_t)d.batch * d.num_heads, rows = units * d.draft;
+    const size_t esz = d.io_dtype == KDA_BF16 ? 2 : 4;
+    const int64_t nk = rows * d.dk * (int64_t)esz, nv = rows * d.dv * (int64_t)esz;
+    const Range rS = range_of(S, units * d.dk * d.dv * 4), ro = range_of(o, o ? nv : 0);
+    const Range ins[] = {range_of(q, nk), range_of(k, nk), range_of(g, nk), range_of(v, nv),
+                         range_of(beta, rows * (int64_t)esz), range_of(gate, gate ? nv : 0),
+                         range_of(accepted, accepted ? 4 * (int64_t)d.batch : 0)};
+    for (const Range &r : ins)
+        if (overlaps(rS, r) || overlaps(ro, r)) return KDA_ERR_INVALID_ARG;
+    if (overlaps(rS, ro)) return KDA_ERR_INVALID_ARG;
+    return KDA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -523,6 +567,36 @@ kda_status kda_decode_step(const kda_decode_desc *desc, const void *q, const voi
     DecodeParams p{q, k, v, g, beta, gate, S, o, d.scale, d.g_floor};
     cudaError_t e = d.io_dtype == KDA_BF16 ? dispatch_decode<__nv_bfloat16>(d.dk, d.dv, p, units, stream)
                                            : dispatch_decode<float>(d.dk, d.dv, p, units, stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_spec_verify(const kda_spec_desc *desc, const void *q, const void *k, const void *v,
+                           const void *g, const void *beta, const float *S, const void *gate,
+                           void *o, cudaStream_t stream) {
+    if (!o) return KDA_ERR_INVALID_ARG;
+    const kda_status st = validate_spec(desc, q, k, v, g, beta, S, gate, o, nullptr);
+    if (st != KDA_OK) return st;
+    const kda_spec_desc &d = *desc;
+    kda::SpecParams p{q, k, v, g, beta, gate, const_cast<float *>(S), o, nullptr, d.num_heads,
+                      d.draft, d.scale, d.g_floor};
+    const int64_t units = (int64_t)d.batch * d.num_heads;
+    cudaError_t e = d.io_dtype == KDA_BF16 ? dispatch_spec<__nv_bfloat16, false>(d.dk, d.dv, p, units, stream)
+                                           : dispatch_spec<float, false>(d.dk, d.dv, p, units, stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_spec_commit(const kda_spec_desc *desc, const void *q, const void *k, const void *v,
+                           const void *g, const void *beta, float *S, const int32_t *accepted,
+                           cudaStream_t stream) {
+    if (!accepted) return KDA_ERR_INVALID_ARG;
+    const kda_status st = validate_spec(desc, q, k, v, g, beta, S, nullptr, nullptr, accepted);
+    if (st != KDA_OK) return st;
+    const kda_spec_desc &d = *desc;
+    kda::SpecParams p{q, k, v, g, beta, nullptr, S, nullptr, accepted, d.num_heads, d.draft,
+                      d.scale, d.g_floor};
+    const int64_t units = (int64_t)d.batch * d.num_heads;
+    cudaError_t e = d.io_dtype == KDA_BF16 ? dispatch_spec<__nv_bfloat16, true>(d.dk, d.dv, p, units, stream)
+                                           : dispatch_spec<float, true>(d.dk, d.dv, p, units, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -27,7 +27,7 @@ KDA_BF16, KDA_FP32 = 0, 1
 EXPORTED_SYMBOLS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
                     "kda_get_device_status", "kda_status_string", "kda_version",
                     "kda_chunk_fwd_noalloc", "kda_selftest_bounded_wait",
-                    "kda_chunk_fwd_snapshots")
+                    "kda_chunk_fwd_snapshots", "kda_spec_verify", "kda_spec_commit")
 NOALLOC_MAX_SEQS = 65536   # KDA_NOALLOC_MAX_SEQS in include/kda.h
 
 
@@ -56,6 +56,15 @@ class DecodeDesc(ctypes.Structure):
                 ("dk", ctypes.c_int32), ("dv", ctypes.c_int32), ("io_dtype", ctypes.c_int),
                 ("scale", ctypes.c_float), ("g_floor", ctypes.c_float)]
 
+
+class SpecDesc(ctypes.Structure):
+    """``kda_spec_desc``."""
+    _fields_ = [("batch", ctypes.c_int32), ("num_heads", ctypes.c_int32),
+                ("dk", ctypes.c_int32), ("dv", ctypes.c_int32), ("draft", ctypes.c_int32),
+                ("io_dtype", ctypes.c_int), ("scale", ctypes.c_float), ("g_floor", ctypes.c_float)]
+
+
+SPEC_MAX_DRAFT = 64   # KDA_SPEC_MAX_DRAFT in include/kda.h
 
 _lib = None
 _lock = threading.Lock()
@@ -91,6 +100,10 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
                                                 vp, vp, vp, vp, vp, vp, i32p, i32p, vp, vp, vp, vp,
                                                 sz, vp]
         lib.kda_chunk_fwd_snapshots.restype = ctypes.c_int
+        lib.kda_spec_verify.argtypes = [ctypes.POINTER(SpecDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.kda_spec_verify.restype = ctypes.c_int
+        lib.kda_spec_commit.argtypes = [ctypes.POINTER(SpecDesc), vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.kda_spec_commit.restype = ctypes.c_int
         lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_int32, vp]
         lib.kda_selftest_bounded_wait.restype = ctypes.c_int
         _lib = lib
@@ -296,6 +309,55 @@ def decode_step(q, k, v, g, beta, S, gate=None, scale=None, g_floor: float = -5.
     if st != KDA_OK:
         raise KDAError(st, "kda_decode_step")
     return o
+
+
+def _spec_desc(q, k, v, g, beta, S, gate, scale, g_floor):
+    B, D, H, dk = q.shape
+    dv = v.shape[-1]
+    device, dtype = q.device, q.dtype
+    _check(q, "q", (B, D, H, dk), dtype, device)
+    _check(k, "k", (B, D, H, dk), dtype, device)
+    _check(g, "g", (B, D, H, dk), dtype, device)
+    _check(v, "v", (B, D, H, dv), dtype, device)
+    _check(beta, "beta", (B, D, H), dtype, device)
+    _check(S, "S", (B, H, dk, dv), torch.float32, device)
+    if gate is not None:
+        _check(gate, "gate", (B, D, H, dv), dtype, device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(dk)
+    return SpecDesc(B, H, dk, dv, D, _io_dtype(q), float(scale), float(g_floor))
+
+
+def spec_verify(q, k, v, g, beta, S, gate=None, scale=None, g_floor: float = -5.0, out=None):
+    """``kda_spec_verify``: outputs of D draft tokens per sequence, replayed from
+    ``S`` without changing it.  q, k, g [B,D,H,dk]; v, gate [B,D,H,dv]; beta
+    [B,D,H]; S fp32 [B,H,dk,dv].  Returns o [B,D,H,dv]."""
+    _require_cuda()
+    lib = load_library()
+    desc = _spec_desc(q, k, v, g, beta, S, gate, scale, g_floor)
+    o = out if out is not None else torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    _check(o, "out", tuple(v.shape), q.dtype, q.device)
+    with torch.cuda.device(q.device):
+        st = lib.kda_spec_verify(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                 _ptr(S), _ptr(gate), _ptr(o), _stream_handle(q.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_spec_verify")
+    return o
+
+
+def spec_commit(q, k, v, g, beta, S, accepted, scale=None, g_floor: float = -5.0):
+    """``kda_spec_commit``: applies the first ``accepted[b]`` of the D draft tokens
+    of sequence b to ``S`` in place (``accepted`` int32 [B] on the GPU)."""
+    _require_cuda()
+    lib = load_library()
+    desc = _spec_desc(q, k, v, g, beta, S, None, scale, g_floor)
+    _check(accepted, "accepted", (q.shape[0],), torch.int32, q.device)
+    with torch.cuda.device(q.device):
+        st = lib.kda_spec_commit(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                 _ptr(S), _ptr(accepted), _stream_handle(q.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_spec_commit")
+    return S
 
 
 def device_status(device=None) -> int:

@@ -153,6 +153,46 @@ kda_status kda_decode_step(const kda_decode_desc *desc,
                            const void *gate, void *o, cudaStream_t stream);
 
 /*
+ * Speculative-decode verify and commit (the replay of the Kimi K3 report
+ * digest, section 基础设施: the target model checks D draft tokens at once,
+ * then only the accepted prefix is committed to the state, in place).
+ * Acceptance is decided outside attention, from the outputs, so these are
+ * two calls over the same D tokens per sequence:
+ *   kda_spec_verify: outputs of all D tokens, as D consecutive decode steps
+ *                    from S would give them; S is only read.
+ *   kda_spec_commit: applies the first accepted[b] tokens of sequence b
+ *                    (clamped to [0, D]) to S in place; 0 leaves S untouched.
+ * Each call streams every head's state once, whatever D is (D decode steps
+ * would stream it D times in each direction).
+ *
+ *   q, k, g  device io_dtype [B, D, H, dk] (token-major per sequence)
+ *   v        device io_dtype [B, D, H, dv];  beta  device io_dtype [B, D, H]
+ *   S        device fp32 [B, H, dk, dv], 16-byte aligned
+ *   gate     device io_dtype [B, D, H, dv] gate logits or NULL (verify only)
+ *   o        device io_dtype [B, D, H, dv] (verify) -- must not overlap S or inputs
+ *   accepted device int32 [B] (commit)
+ * Returns KDA_ERR_INVALID_ARG for a bad descriptor (draft outside
+ * 1..KDA_SPEC_MAX_DRAFT), null pointers or overlaps, KDA_ERR_UNSUPPORTED for
+ * head sizes other than 64 or 128, KDA_ERR_CUDA if the launch fails.
+ */
+#define KDA_SPEC_MAX_DRAFT 64
+
+typedef struct {
+    int32_t batch, num_heads, dk, dv;
+    int32_t draft;              /* D, tokens per sequence */
+    kda_dtype io_dtype;
+    float scale, g_floor;
+} kda_spec_desc;
+
+kda_status kda_spec_verify(const kda_spec_desc *desc, const void *q, const void *k, const void *v,
+                           const void *g, const void *beta, const float *S, const void *gate,
+                           void *o, cudaStream_t stream);
+
+kda_status kda_spec_commit(const kda_spec_desc *desc, const void *q, const void *k, const void *v,
+                           const void *g, const void *beta, float *S, const int32_t *accepted,
+                           cudaStream_t stream);
+
+/*
  * kda_chunk_fwd without any caller-provided device memory.  The pages have
  * no counterpart to this entry point: it exists for callers that cannot hand
  * the library a workspace, such as a plugin interface that passes only the

@@ -166,3 +166,35 @@ def test_snapshots_validation(lib):
                 dict(states=A + 64 * MB)):                                  # states inside workspace
         snap = kda.Snapshots(**{**ok, **bad})
         assert _snapfwd(lib, d, snap, cu_host) == 1, bad
+
+
+def _spec(**kw):
+    base = dict(batch=2, num_heads=2, dk=128, dv=128, draft=4, io_dtype=kda.KDA_BF16, scale=0.09,
+                g_floor=-5.0)
+    base.update(kw)
+    return kda.SpecDesc(**base)
+
+
+def _verify(lib, desc, S=A + 40 * MB, o=A + 48 * MB, gate=None):
+    return lib.kda_spec_verify(ctypes.byref(desc), A, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB,
+                               S, gate, o, None)
+
+
+def _commit(lib, desc, S=A + 40 * MB, acc=A + 56 * MB):
+    return lib.kda_spec_commit(ctypes.byref(desc), A, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB,
+                               S, acc, None)
+
+
+def test_spec_validation(lib):
+    """Rejected on the host before any launch (fake pointers never touched)."""
+    for bad in (dict(draft=0), dict(draft=kda.SPEC_MAX_DRAFT + 1), dict(batch=0),
+                dict(io_dtype=5), dict(g_floor=-7.0), dict(scale=float("inf"))):
+        assert _verify(lib, _spec(**bad)) == 1, bad
+        assert _commit(lib, _spec(**bad)) == 1, bad
+    assert _verify(lib, _spec(dk=96)) == 2
+    assert _verify(lib, _spec(), o=None) == 1                  # verify needs outputs
+    assert _commit(lib, _spec(), acc=None) == 1                # commit needs the counts
+    assert _verify(lib, _spec(), S=A + 2 * MB) == 1            # S inside v
+    assert _verify(lib, _spec(), o=A + 40 * MB + 64) == 1      # o inside S
+    assert _commit(lib, _spec(), S=A + 40 * MB + 8) == 1       # S not 16-byte aligned
+    assert _commit(lib, _spec(), acc=A + 40 * MB + 4096) == 1  # counts inside S
