@@ -12,6 +12,13 @@
 // Inputs are token-major per sequence: q, k, g [B, D, H, dk]; v, gate, o
 // [B, D, H, dv]; beta [B, D, H].  Each pass streams the 64 KiB state once
 // (verify: read; commit: read + write), whatever D is.
+//
+// One CTA of 256 threads per (sequence, head).  Tokens are staged 8 at a time
+// in shared memory as {alpha, alpha k, alpha q, beta k} per state row; each
+// thread keeps F rows x 4 columns of the state in registers and updates them
+// with packed f32x2 arithmetic; u and w are summed over the row groups through
+// shared memory, double-buffered by token parity, so each token costs one
+// barrier.  The output of token j is written by row group j mod RG.
 #pragma once
 
 #include "kda_common.cuh"
@@ -33,12 +40,14 @@ __global__ void __launch_bounds__(256) spec_kernel(SpecParams p)
     constexpr int NT = 256;
     constexpr int C4 = DV / 4;        // float4 per state row
     constexpr int RG = NT / C4;       // row groups
-    constexpr int F = DK / RG;        // state rows per thread
+    constexpr int F = DK / RG;        // state rows per thread: rows rg * F .. rg * F + F - 1
+    constexpr int G = 8;              // tokens staged in shared memory at a time
     static_assert(DK % RG == 0, "row split");
 
-    __shared__ float sq[DK], sk[DK], sa[DK], sv[DV];
-    __shared__ float4 red_u[RG][C4], red_w[RG][C4];
-    __shared__ float s_kq;
+    // per staged token and state row: {alpha, alpha k, alpha q, beta k}
+    __shared__ float4 srow[G][DK];
+    __shared__ float sv[G][DV], sz[COMMIT ? 1 : G][DV], skq[G];
+    __shared__ float4 red_u[2][RG][C4], red_w[2][RG][C4];   // by token parity
 
     const TIO *q = static_cast<const TIO *>(p.q);
     const TIO *k = static_cast<const TIO *>(p.k);
@@ -48,7 +57,7 @@ __global__ void __launch_bounds__(256) spec_kernel(SpecParams p)
     const TIO *gate = static_cast<const TIO *>(p.gate);
     TIO *o = static_cast<TIO *>(p.o);
 
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int col4 = tid % C4;
     const int rg = tid / C4;
     const int H = p.num_heads, D = p.draft;
@@ -63,81 +72,148 @@ __global__ void __launch_bounds__(256) spec_kernel(SpecParams p)
         if (ntok == 0) return;                   // nothing accepted: S stays as it is
     }
 
-    float4 s[F];
+    // the state slice as column pairs: s[f][0] = columns 4 col4 + {0,1}, s[f][1] = + {2,3}
+    float2 s[F][2];
 #pragma unroll
-    for (int f = 0; f < F; ++f) s[f] = __ldcs(&Sp[(rg + f * RG) * C4 + col4]);
+    for (int f = 0; f < F; ++f) {
+        const float4 x = __ldcs(&Sp[(rg * F + f) * C4 + col4]);
+        s[f][0] = make_float2(x.x, x.y);
+        s[f][1] = make_float2(x.z, x.w);
+    }
 
-    for (int t = 0; t < ntok; ++t) {
-        const int64_t row = (b * D + t) * H + h;  // (token, head) row of the packed inputs
-        for (int i = tid; i < DK; i += NT) {
-            sq[i] = ld(q, row * DK + i);
-            sk[i] = ld(k, row * DK + i);
-            sa[i] = expf(fmaxf(ld(g, row * DK + i), p.g_floor));
+    for (int t0 = 0; t0 < ntok; t0 += G) {
+        const int nt = ntok - t0 < G ? ntok - t0 : G;
+        __syncthreads();                         // the previous group's values are consumed
+        // stage the group's tokens, row (b, t, h) of the packed inputs
+        if (COMMIT) {
+            // one element after another (measured faster for the commit than
+            // issuing every load first); q is not needed
+            for (int i = tid; i < nt * DK; i += NT) {
+                const int j = i / DK, c = i % DK;
+                const int64_t row = (b * D + t0 + j) * H + h;
+                const float kk = ld(k, row * DK + c);
+                const float a = expf(fmaxf(ld(g, row * DK + c), p.g_floor));
+                srow[j][c] = make_float4(a, a * kk, 0.0f, ld(beta, row) * kk);
+            }
+            for (int i = tid; i < nt * DV; i += NT) {
+                const int j = i / DV, c = i % DV;
+                sv[j][c] = ld(v, ((b * D + t0 + j) * H + h) * DV + c);
+            }
+        } else {
+            // every load issued before the first shared-memory store
+            constexpr int EK = G * DK / NT, EV = G * DV / NT;
+            float kk[EK], qq[EK], gg[EK], bb[EK], vv[EV], zz[EV];
+#pragma unroll
+            for (int e = 0; e < EK; ++e) {
+                const int i = tid + e * NT, j = i / DK, c = i % DK;
+                if (j < nt) {
+                    const int64_t row = (b * D + t0 + j) * H + h;
+                    kk[e] = ld(k, row * DK + c);
+                    qq[e] = ld(q, row * DK + c);
+                    gg[e] = ld(g, row * DK + c);
+                    bb[e] = ld(beta, row);
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < EV; ++e) {
+                const int i = tid + e * NT, j = i / DV, c = i % DV;
+                if (j < nt) {
+                    const int64_t off = ((b * D + t0 + j) * H + h) * DV + c;
+                    vv[e] = ld(v, off);
+                    zz[e] = gate ? ld(gate, off) : 0.0f;
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < EK; ++e) {
+                const int i = tid + e * NT, j = i / DK, c = i % DK;
+                if (j < nt) {
+                    const float a = expf(fmaxf(gg[e], p.g_floor));
+                    srow[j][c] = make_float4(a, a * kk[e], a * qq[e], bb[e] * kk[e]);
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < EV; ++e) {
+                const int i = tid + e * NT, j = i / DV, c = i % DV;
+                if (j < nt) {
+                    sv[j][c] = vv[e];
+                    sz[COMMIT ? 0 : j][c] = gate ? sigmoidf(zz[e]) : 1.0f;
+                }
+            }
         }
-        for (int i = tid; i < DV; i += NT) sv[i] = ld(v, row * DV + i);
         __syncthreads();
-
-        if (!COMMIT && tid < 32) {
+        if (!COMMIT && warp < nt) {              // beta (k.q) of token `warp`
             float acc = 0.0f;
-            for (int i = tid; i < DK; i += 32) acc = fmaf(sk[i], sq[i], acc);
+            for (int i = lane; i < DK; i += 32) {
+                const float4 r = srow[warp][i];
+                acc = fmaf(r.w, r.z / r.x, acc);   // (beta k)(alpha q) / alpha
+            }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-            if (tid == 0) s_kq = acc;
+            if (lane == 0) skq[warp] = acc;
         }
 
-        float4 u = make_float4(0.f, 0.f, 0.f, 0.f), w = u;
+        for (int j = 0; j < nt; ++j) {
+            const int par = j & 1;
+            float2 u0 = make_float2(0.f, 0.f), u1 = u0, w0 = u0, w1 = u0;
 #pragma unroll
-        for (int f = 0; f < F; ++f) {
-            const int c = rg + f * RG;
-            const float a = sa[c], kc = sk[c], qc = sq[c];
-            s[f].x *= a; s[f].y *= a; s[f].z *= a; s[f].w *= a;
-            u.x = fmaf(s[f].x, kc, u.x); u.y = fmaf(s[f].y, kc, u.y);
-            u.z = fmaf(s[f].z, kc, u.z); u.w = fmaf(s[f].w, kc, u.w);
-            if (!COMMIT) {
-                w.x = fmaf(s[f].x, qc, w.x); w.y = fmaf(s[f].y, qc, w.y);
-                w.z = fmaf(s[f].z, qc, w.z); w.w = fmaf(s[f].w, qc, w.w);
+            for (int f = 0; f < F; ++f) {
+                const float4 r = srow[j][rg * F + f];
+                const float2 ak = make_float2(r.y, r.y);
+                u0 = __ffma2_rn(s[f][0], ak, u0);
+                u1 = __ffma2_rn(s[f][1], ak, u1);
+                if (!COMMIT) {
+                    const float2 aq = make_float2(r.z, r.z);
+                    w0 = __ffma2_rn(s[f][0], aq, w0);
+                    w1 = __ffma2_rn(s[f][1], aq, w1);
+                }
             }
-        }
-        red_u[rg][col4] = u;
-        if (!COMMIT) red_w[rg][col4] = w;
-        __syncthreads();
+            red_u[par][rg][col4] = make_float4(u0.x, u0.y, u1.x, u1.y);
+            if (!COMMIT) red_w[par][rg][col4] = make_float4(w0.x, w0.y, w1.x, w1.y);
+            // one barrier per token: the other parity's buffers were read before it
+            __syncthreads();
 
-        float4 U = make_float4(0.f, 0.f, 0.f, 0.f), W = U;
+            float2 U0 = make_float2(0.f, 0.f), U1 = U0;
 #pragma unroll
-        for (int r = 0; r < RG; ++r) {
-            const float4 a = red_u[r][col4];
-            U.x += a.x; U.y += a.y; U.z += a.z; U.w += a.w;
-            if (!COMMIT) {
-                const float4 c = red_w[r][col4];
-                W.x += c.x; W.y += c.y; W.z += c.z; W.w += c.w;
+            for (int r = 0; r < RG; ++r) {
+                const float4 x = red_u[par][r][col4];
+                U0 = __fadd2_rn(U0, make_float2(x.x, x.y));
+                U1 = __fadd2_rn(U1, make_float2(x.z, x.w));
+            }
+            const float4 vj = *reinterpret_cast<const float4 *>(&sv[j][4 * col4]);
+            const float2 d0 = make_float2(vj.x - U0.x, vj.y - U0.y);
+            const float2 d1 = make_float2(vj.z - U1.x, vj.w - U1.y);
+            // S = alpha S + (beta k) d^T
+#pragma unroll
+            for (int f = 0; f < F; ++f) {
+                const float4 r = srow[j][rg * F + f];
+                const float2 al = make_float2(r.x, r.x), bk = make_float2(r.w, r.w);
+                s[f][0] = __ffma2_rn(s[f][0], al, __fmul2_rn(bk, d0));
+                s[f][1] = __ffma2_rn(s[f][1], al, __fmul2_rn(bk, d1));
+            }
+            if (!COMMIT && rg == j % RG) {         // the output of token j, one row group
+                float2 W0 = make_float2(0.f, 0.f), W1 = W0;
+#pragma unroll
+                for (int r = 0; r < RG; ++r) {
+                    const float4 y = red_w[par][r][col4];
+                    W0 = __fadd2_rn(W0, make_float2(y.x, y.y));
+                    W1 = __fadd2_rn(W1, make_float2(y.z, y.w));
+                }
+                const int64_t off = ((b * D + t0 + j) * H + h) * DV + 4 * col4;
+                const float bkq = skq[j];
+                const float4 zg = *reinterpret_cast<const float4 *>(&sz[COMMIT ? 0 : j][4 * col4]);
+                st(o, off + 0, p.scale * fmaf(bkq, d0.x, W0.x) * zg.x);
+                st(o, off + 1, p.scale * fmaf(bkq, d0.y, W0.y) * zg.y);
+                st(o, off + 2, p.scale * fmaf(bkq, d1.x, W1.x) * zg.z);
+                st(o, off + 3, p.scale * fmaf(bkq, d1.y, W1.y) * zg.w);
             }
         }
-        const float bt = ld(beta, row);
-        const float4 d = make_float4(sv[4 * col4 + 0] - U.x, sv[4 * col4 + 1] - U.y,
-                                     sv[4 * col4 + 2] - U.z, sv[4 * col4 + 3] - U.w);
-#pragma unroll
-        for (int f = 0; f < F; ++f) {
-            const float bk = bt * sk[rg + f * RG];
-            s[f].x = fmaf(bk, d.x, s[f].x); s[f].y = fmaf(bk, d.y, s[f].y);
-            s[f].z = fmaf(bk, d.z, s[f].z); s[f].w = fmaf(bk, d.w, s[f].w);
-        }
-        if (!COMMIT && rg == 0) {
-            const float bkq = bt * s_kq;
-            const float oo[4] = {W.x + bkq * d.x, W.y + bkq * d.y, W.z + bkq * d.z, W.w + bkq * d.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int64_t off = row * DV + 4 * col4 + e;
-                float x = p.scale * oo[e];
-                if (gate) x *= sigmoidf(ld(gate, off));
-                st(o, off, x);
-            }
-        }
-        __syncthreads();                         // the token's shared values are consumed
     }
 
     if (COMMIT) {
 #pragma unroll
-        for (int f = 0; f < F; ++f) __stcs(&Sp[(rg + f * RG) * C4 + col4], s[f]);
+        for (int f = 0; f < F; ++f)
+            __stcs(&Sp[(rg * F + f) * C4 + col4],
+                   make_float4(s[f][0].x, s[f][0].y, s[f][1].x, s[f][1].y));
     }
 }
 

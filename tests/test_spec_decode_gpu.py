@@ -77,3 +77,27 @@ def test_commit_all_equals_decode_steps():
                 torch.tensor([-3, 0, 0, 0], dtype=torch.int32, device="cuda"))
     assert torch.equal(S2, S)
     assert device_status() == 0
+
+
+@pytest.mark.parametrize("D,dk,dv,dtype", [(19, 128, 64, torch.float32), (64, 64, 128, torch.bfloat16)])
+def test_long_draft_without_gate(D, dk, dv, dtype):
+    """Drafts longer than one staged group of tokens (ragged last group), no
+    output gate, dk != dv; the full commit gives the oracle's final state."""
+    B, H = 2, 3
+    inp = inputs.prefill_inputs([D] * B, H=H, dk=dk, dv=dv, dtype=dtype, device="cuda", seed=53 + D,
+                                s0_std=0.05, gate=False)
+    x = {n: inp[n].view(B, D, *inp[n].shape[1:]) for n in ("q", "k", "v", "g", "beta")}
+    S = inp["S0"].clone()
+    o = spec_verify(x["q"], x["k"], x["v"], x["g"], x["beta"], S)
+    cu = np.array(inp["cu_seqlens_host"], dtype=np.int64)
+    o_ref, S_ref = oracle.kda_fwd_ref(*(_cpu(inp[n]) for n in ("q", "k", "v", "g", "beta")),
+                                      cu_seqlens=cu, S0=_cpu(inp["S0"]))
+    spec_commit(x["q"], x["k"], x["v"], x["g"], x["beta"], S,
+                torch.full((B,), D, dtype=torch.int32, device="cuda"))
+    if dtype == torch.float32:
+        assert rel_max(o.view(B * D, H, dv), o_ref) <= TOL_FP32
+        assert rel_max(S, S_ref) <= TOL_FP32
+    else:
+        assert rel_max_beyond_bf16(o.view(B * D, H, dv), o_ref) <= TOL_BF16
+        assert rel_max(S, S_ref) <= TOL_BF16
+    assert device_status() == 0
