@@ -270,7 +270,9 @@ cudaError_t launch_tc_units(const kda_fwd_desc &d, const void *q, const void *k,
     const uint64_t rows = (uint64_t)d.total_tokens, cols = (uint64_t)d.num_heads * 128u;
     if (!encode_bf16_2d(&tq, q, rows, cols) || !encode_bf16_2d(&tk, k, rows, cols) ||
         !encode_bf16_2d(&tg, g, rows, cols) || !encode_bf16_2d(&tv, v, rows, cols) ||
-        !encode_bf16_2d(&to, p.o, rows, cols))
+        // no output buffer (summaries): the map is never stored through, since
+        // no unit carries UNIT_STORE_O; q stands in for a valid address
+        !encode_bf16_2d(&to, p.o ? p.o : q, rows, cols))
         return cudaErrorInvalidValue;
     auto kern = p.snap.states ? kda::tck::chunk_tc_kernel<true> : kda::tck::chunk_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -340,7 +342,7 @@ cudaError_t launch_split(const kda_fwd_desc &d, const SegPlan &pl, const int32_t
                 p2.push_back(TcUnit{a, b, sp == 0 ? s0 : Sin(sp), sp + 1 == P ? st : nullptr, h,
                                     kda::tck::UNIT_STORE_O, n, t0});
             }
-            jobs.push_back(kda::ScanJob{Sloc(0), Mp(0), Sin(0), (int64_t)(3u * DD), P});
+            jobs.push_back(kda::ScanJob{Sloc(0), Mp(0), Sin(0), (int64_t)(3u * DD), P, nullptr});
         }
     }
     auto longest_first = [](const TcUnit &x, const TcUnit &y) {
@@ -598,6 +600,99 @@ kda_status kda_spec_commit(const kda_spec_desc *desc, const void *q, const void 
     cudaError_t e = d.io_dtype == KDA_BF16 ? dispatch_spec<__nv_bfloat16, true>(d.dk, d.dv, p, units, stream)
                                            : dispatch_spec<float, true>(d.dk, d.dv, p, units, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- context parallel (KCP)
+size_t kda_segment_summary_workspace_size(const kda_fwd_desc *desc) {
+    if (validate_fwd_desc(desc) != KDA_OK) return SIZE_MAX;
+    return align256(2u * sizeof(kda::tck::TcUnit) * (size_t)desc->num_seqs * (size_t)desc->num_heads);
+}
+
+kda_status kda_segment_summary(const kda_fwd_desc *desc, const void *q, const void *k,
+                               const void *v, const void *g, const void *beta, const float *S0,
+                               const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                               float *S_loc, float *M, void *workspace, size_t workspace_bytes,
+                               cudaStream_t stream) {
+    using kda::tck::TcUnit;
+    kda_status st = validate_fwd_desc(desc);
+    if (st != KDA_OK) return st;
+    const kda_fwd_desc &d = *desc;
+    if (d.io_dtype != KDA_BF16 || d.dk != 128 || d.dv != 128 || d.chunk == 16) return KDA_ERR_UNSUPPORTED;
+    if (d.total_tokens < 1 || d.total_tokens > INT32_MAX - 64) return KDA_ERR_INVALID_ARG;
+    if (!cu_seqlens || !cu_seqlens_host || !S_loc || !q || !k || !v || !g || !beta) return KDA_ERR_INVALID_ARG;
+    if ((st = validate_host_seqlens(desc, cu_seqlens_host)) != KDA_OK) return st;
+    for (const void *ptr : {q, k, v, g})      // moved by TMA
+        if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return KDA_ERR_INVALID_ARG;
+
+    const int32_t N = d.num_seqs, H = d.num_heads;
+    const int64_t T = d.total_tokens, DD = 128 * 128;
+    const int64_t nk = T * H * 128 * 2, nb = T * H * 2, ns = (int64_t)N * H * DD * 4;
+    const Range ins[] = {range_of(q, nk), range_of(k, nk), range_of(g, nk), range_of(v, nk),
+                         range_of(beta, nb), range_of(S0, S0 ? ns : 0),
+                         range_of(cu_seqlens, 4 * (int64_t)(N + 1))};
+    const Range rl = range_of(S_loc, ns), rm = range_of(M, M ? ns : 0);
+    for (const Range &r : ins)
+        if (overlaps(rl, r) || overlaps(rm, r)) return KDA_ERR_INVALID_ARG;
+    if (overlaps(rl, rm)) return KDA_ERR_INVALID_ARG;
+    const size_t need = kda_segment_summary_workspace_size(desc);
+    if (!workspace || workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256 != 0)
+        return KDA_ERR_WORKSPACE;
+    const Range rw = range_of(workspace, (int64_t)need);
+    for (const Range &r : ins)
+        if (overlaps(rw, r)) return KDA_ERR_INVALID_ARG;
+    if (overlaps(rw, rl) || overlaps(rw, rm)) return KDA_ERR_INVALID_ARG;
+
+    // one chain per (sequence, head) for S_loc, one more for M: the M chain
+    // starts from the identity with v taken as zero
+    std::vector<TcUnit> units;
+    units.reserve((size_t)N * H * (M ? 2 : 1));
+    for (int32_t n = 0; n < N; ++n) {
+        for (int32_t h = 0; h < H; ++h) {
+            const int64_t u = (int64_t)n * H + h;
+            units.push_back(TcUnit{cu_seqlens_host[n], cu_seqlens_host[n + 1], S0 ? S0 + u * DD : nullptr,
+                                   S_loc + u * DD, h, 0, n, cu_seqlens_host[n]});
+            if (M)
+                units.push_back(TcUnit{cu_seqlens_host[n], cu_seqlens_host[n + 1], nullptr, M + u * DD, h,
+                                       kda::tck::UNIT_ZERO_V | kda::tck::UNIT_S0_IDENTITY, n,
+                                       cu_seqlens_host[n]});
+        }
+    }
+    std::stable_sort(units.begin(), units.end(), [](const TcUnit &x, const TcUnit &y) {
+        return (x.t_end - x.t_begin) > (y.t_end - y.t_begin);
+    });
+    TcUnit *du = static_cast<TcUnit *>(workspace);
+    if (cudaMemcpyAsync(du, units.data(), units.size() * sizeof(TcUnit), cudaMemcpyHostToDevice,
+                        stream) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    kda::tck::TcParams tp{beta, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, H, d.scale,
+                          d.g_floor, du, kda::SnapOut{nullptr, nullptr, 0, 64}};
+    return launch_tc_units(d, q, k, v, g, tp, (int64_t)units.size(), stream) == cudaSuccess ? KDA_OK
+                                                                                           : KDA_ERR_CUDA;
+}
+
+kda_status kda_state_combine(const kda_combine_desc *desc, const float *summaries, float *S_in,
+                             cudaStream_t stream) {
+    if (!desc || !summaries || !S_in) return KDA_ERR_INVALID_ARG;
+    const kda_combine_desc &c = *desc;
+    if (c.num_seqs < 1 || c.num_heads < 1 || c.num_summaries < 1 || c.dk <= 0 || c.dv <= 0)
+        return KDA_ERR_INVALID_ARG;
+    if (c.dk != 128 || c.dv != 128) return KDA_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(summaries) % 16 != 0 || reinterpret_cast<uintptr_t>(S_in) % 16 != 0)
+        return KDA_ERR_INVALID_ARG;
+    const int64_t DD = 128 * 128;
+    const int64_t units = mul3(c.num_seqs, c.num_heads, 1);
+    const int64_t per_piece = mul3(units, 2, DD);
+    if (units < 0 || per_piece < 0 || units > INT32_MAX) return KDA_ERR_INVALID_ARG;
+    const int64_t all = mul3(per_piece, c.num_summaries, 4);
+    if (all < 0) return KDA_ERR_INVALID_ARG;
+    if (overlaps(range_of(summaries, all), range_of(S_in, units * DD * 4))) return KDA_ERR_INVALID_ARG;
+    const size_t smem = 2u * (size_t)DD * sizeof(float);
+    if (cudaFuncSetAttribute(kda::state_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    kda::state_combine_kernel<<<(unsigned)units, 256, smem, stream>>>(summaries, S_in, units,
+                                                                      c.num_summaries);
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 namespace {

@@ -9,7 +9,9 @@
 // and a second pass reruns every segment from its S_in (the context-parallel
 // decomposition of the fupanwang.com Kimi K3 report digest, section 基础设施:
 // own state plus the incoming state times the transition product, joined by a
-// prefix scan).
+// prefix scan).  Across GPUs the same fold runs on the summaries that every
+// rank contributes to an all-gather (kda_state_combine): there only the last
+// start state, S_last, is written.
 #pragma once
 
 #include "kda_common.cuh"
@@ -19,26 +21,27 @@ namespace kda {
 struct ScanJob {
     const float *S_loc;   // [P][dk][dv] segment-local final states (stride job_stride)
     const float *M;       // [P][dk][dk] segment transition products
-    float *S_in;          // [P][dk][dv] start states (entries 1..P-1 written)
+    float *S_in;          // [P][dk][dv] start states (entries 1..P-1 written), or null
     int64_t stride;       // floats between consecutive segments' matrices
     int32_t num_segments;
+    float *S_last;        // if not null: S_in(P-1) is also written here
 };
 
 // One CTA (256 threads) per (sequence, head).  dk = dv = 128; thread (v, half)
 // computes rows c in [64 half, 64 half + 64) of column v.
-__global__ void __launch_bounds__(256) segment_scan_kernel(const ScanJob *jobs)
+__device__ __forceinline__ void scan_one(const ScanJob &job)
 {
     constexpr int D = 128;
     extern __shared__ float4 scan_smem[];
     float *Ms = reinterpret_cast<float *>(scan_smem);   // [D][D]
     float *Ss = Ms + D * D;                              // [D][D]
-    const ScanJob job = jobs[blockIdx.x];
     const int tid = threadIdx.x, v = tid & 127, half = tid >> 7;
 
     for (int idx = tid; idx < D * D; idx += 256) {
         const float x = job.S_loc[idx];
         Ss[idx] = x;
-        job.S_in[job.stride + idx] = x;     // S_in(1) = S_loc,0
+        if (job.S_in) job.S_in[job.stride + idx] = x;     // S_in(1) = S_loc,0
+        if (job.S_last && job.num_segments == 2) job.S_last[idx] = x;
     }
     __syncthreads();
     for (int seg = 1; seg + 1 < job.num_segments; ++seg) {
@@ -60,14 +63,33 @@ __global__ void __launch_bounds__(256) segment_scan_kernel(const ScanJob *jobs)
             }
         }
         __syncthreads();
-        float *out = job.S_in + (seg + 1) * job.stride;
+        float *out = job.S_in ? job.S_in + (seg + 1) * job.stride
+                              : (seg + 2 == job.num_segments ? job.S_last : nullptr);
+        float *out2 = job.S_in && seg + 2 == job.num_segments ? job.S_last : nullptr;
 #pragma unroll
         for (int r = 0; r < 64; ++r) {
             Ss[(half * 64 + r) * D + v] = acc[r];
-            out[(half * 64 + r) * D + v] = acc[r];
+            if (out) out[(half * 64 + r) * D + v] = acc[r];
+            if (out2) out2[(half * 64 + r) * D + v] = acc[r];
         }
         __syncthreads();
     }
+}
+
+__global__ void __launch_bounds__(256) segment_scan_kernel(const ScanJob *jobs)
+{
+    scan_one(jobs[blockIdx.x]);
+}
+
+// kda_state_combine: block u folds the summaries of (sequence, head) u, laid
+// out [P][2][units][D][D] (S_loc, then M), into S_last[u].
+__global__ void __launch_bounds__(256) state_combine_kernel(const float *summaries, float *S_in,
+                                                            int64_t units, int32_t num_summaries)
+{
+    constexpr int64_t DD = 128 * 128;
+    const int64_t u = blockIdx.x;
+    scan_one(ScanJob{summaries + u * DD, summaries + (units + u) * DD, nullptr, 2 * units * DD,
+                     num_summaries + 1, S_in + u * DD});
 }
 
 }  // namespace kda

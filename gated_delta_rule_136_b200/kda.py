@@ -27,7 +27,9 @@ KDA_BF16, KDA_FP32 = 0, 1
 EXPORTED_SYMBOLS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
                     "kda_get_device_status", "kda_status_string", "kda_version",
                     "kda_chunk_fwd_noalloc", "kda_selftest_bounded_wait",
-                    "kda_chunk_fwd_snapshots", "kda_spec_verify", "kda_spec_commit")
+                    "kda_chunk_fwd_snapshots", "kda_spec_verify", "kda_spec_commit",
+                    "kda_segment_summary_workspace_size", "kda_segment_summary",
+                    "kda_state_combine")
 NOALLOC_MAX_SEQS = 65536   # KDA_NOALLOC_MAX_SEQS in include/kda.h
 
 
@@ -62,6 +64,12 @@ class SpecDesc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("num_heads", ctypes.c_int32),
                 ("dk", ctypes.c_int32), ("dv", ctypes.c_int32), ("draft", ctypes.c_int32),
                 ("io_dtype", ctypes.c_int), ("scale", ctypes.c_float), ("g_floor", ctypes.c_float)]
+
+
+class CombineDesc(ctypes.Structure):
+    """``kda_combine_desc``."""
+    _fields_ = [("num_seqs", ctypes.c_int32), ("num_heads", ctypes.c_int32),
+                ("dk", ctypes.c_int32), ("dv", ctypes.c_int32), ("num_summaries", ctypes.c_int32)]
 
 
 SPEC_MAX_DRAFT = 64   # KDA_SPEC_MAX_DRAFT in include/kda.h
@@ -104,6 +112,13 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.kda_spec_verify.restype = ctypes.c_int
         lib.kda_spec_commit.argtypes = [ctypes.POINTER(SpecDesc), vp, vp, vp, vp, vp, vp, vp, vp]
         lib.kda_spec_commit.restype = ctypes.c_int
+        lib.kda_segment_summary_workspace_size.argtypes = [ctypes.POINTER(FwdDesc)]
+        lib.kda_segment_summary_workspace_size.restype = sz
+        lib.kda_segment_summary.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, vp, vp, vp, i32p,
+                                            i32p, vp, vp, vp, sz, vp]
+        lib.kda_segment_summary.restype = ctypes.c_int
+        lib.kda_state_combine.argtypes = [ctypes.POINTER(CombineDesc), vp, vp, vp]
+        lib.kda_state_combine.restype = ctypes.c_int
         lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_int32, vp]
         lib.kda_selftest_bounded_wait.restype = ctypes.c_int
         _lib = lib
@@ -358,6 +373,70 @@ def spec_commit(q, k, v, g, beta, S, accepted, scale=None, g_floor: float = -5.0
     if st != KDA_OK:
         raise KDAError(st, "kda_spec_commit")
     return S
+
+
+def segment_summary(q, k, v, g, beta, cu_seqlens, cu_seqlens_host, S0=None, with_M: bool = True,
+                    scale=None, g_floor: float = -5.0):
+    """``kda_segment_summary``: the affine summary of each sequence piece,
+    S_end = M S_start + S_loc.  q, k, g, v [T,H,128] bf16; beta [T,H];
+    ``cu_seqlens`` int32 [N+1] on the GPU and its host copy.  Returns one fp32
+    buffer [2,N,H,128,128]: [0] = S_loc (from S0 if given, else from zero),
+    [1] = M (zeros when ``with_M`` is False).  The layout is what an
+    all-gather of every rank's buffer hands to :func:`state_combine`."""
+    _require_cuda()
+    lib = load_library()
+    device = q.device
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    cu_host = [int(x) for x in cu_seqlens_host]
+    N = len(cu_host) - 1
+    for name, t, shape in (("q", q, (T, H, dk)), ("k", k, (T, H, dk)), ("g", g, (T, H, dk)),
+                           ("v", v, (T, H, dv)), ("beta", beta, (T, H))):
+        _check(t, name, shape, q.dtype, device)
+    _check(cu_seqlens, "cu_seqlens", (N + 1,), torch.int32, device)
+    if S0 is not None:
+        _check(S0, "S0", (N, H, dk, dv), torch.float32, device)
+    desc = FwdDesc(total_tokens=T, num_seqs=N, num_heads=H, dk=dk, dv=dv, io_dtype=_io_dtype(q),
+                   scale=float(dk ** -0.5 if scale is None else scale), g_floor=float(g_floor),
+                   chunk=0, max_seqlen=0)
+    ws_bytes = lib.kda_segment_summary_workspace_size(ctypes.byref(desc))
+    if ws_bytes == ctypes.c_size_t(-1).value:
+        raise KDAError(1, "kda_segment_summary_workspace_size")
+    ws = torch.empty(max(int(ws_bytes), 256), dtype=torch.uint8, device=device)
+    summ = torch.empty((2, N, H, dk, dv), dtype=torch.float32, device=device)
+    if not with_M:
+        summ[1].zero_()
+    cu_h = (ctypes.c_int32 * (N + 1))(*cu_host)
+    with torch.cuda.device(device):
+        st = lib.kda_segment_summary(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                     _ptr(S0), ctypes.cast(_ptr(cu_seqlens), ctypes.POINTER(ctypes.c_int32)),
+                                     cu_h, _ptr(summ[0]), _ptr(summ[1]) if with_M else None, _ptr(ws),
+                                     ws.numel(), _stream_handle(device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_segment_summary")
+    return summ
+
+
+def state_combine(summaries, out=None):
+    """``kda_state_combine``: folds P piece summaries [P,2,N,H,128,128] (fp32,
+    in piece order) into the start state of piece P: S = S_loc(0), then
+    S = M(p) S + S_loc(p).  Returns S_in fp32 [N,H,128,128]."""
+    _require_cuda()
+    lib = load_library()
+    P, two, N, H, dk, dv = summaries.shape
+    if two != 2:
+        raise ValueError("summaries must be [P, 2, N, H, dk, dv]")
+    _check(summaries, "summaries", tuple(summaries.shape), torch.float32, summaries.device)
+    S_in = out if out is not None else torch.empty((N, H, dk, dv), dtype=torch.float32,
+                                                   device=summaries.device)
+    _check(S_in, "out", (N, H, dk, dv), torch.float32, summaries.device)
+    desc = CombineDesc(num_seqs=N, num_heads=H, dk=dk, dv=dv, num_summaries=P)
+    with torch.cuda.device(summaries.device):
+        st = lib.kda_state_combine(ctypes.byref(desc), _ptr(summaries), _ptr(S_in),
+                                   _stream_handle(summaries.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_state_combine")
+    return S_in
 
 
 def device_status(device=None) -> int:

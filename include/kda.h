@@ -268,6 +268,64 @@ kda_status kda_chunk_fwd_snapshots(const kda_fwd_desc *desc, const kda_snapshots
                                    cudaStream_t stream);
 
 /*
+ * Context-parallel prefill across GPUs (KCP, Kimi K3 report digest, section
+ * 基础设施): a long sequence is cut into contiguous pieces, one per rank.
+ * Over a piece the state map is affine, S_end = M S_start + S_loc, with M the
+ * product of the piece's transitions (I - beta k k^T) Diag(alpha), latest on
+ * the left, and S_loc the state the piece grows from S_start = 0.  Every rank
+ * summarises its piece (kda_segment_summary), the summaries are all-gathered
+ * (the caller's collective; a fixed 2 x dk x dv fp32 per sequence and head),
+ * each rank folds those of the ranks before it into its start state
+ * (kda_state_combine) and reruns its piece from there with outputs
+ * (kda_chunk_fwd with S0 = that state).
+ *
+ * kda_segment_summary: for each sequence n of the batch (desc, q, k, v, g,
+ * beta and cu_seqlens as in kda_chunk_fwd; the piece of sequence n on this
+ * rank is tokens cu_seqlens[n] .. cu_seqlens[n+1]):
+ *   S_loc [num_seqs][num_heads][dk][dv] fp32, device: the state after the
+ *         piece starting from S0 (if given, fp32 [num_seqs][num_heads][dk][dv])
+ *         or from zero.  Required.
+ *   M     [num_seqs][num_heads][dk][dk] fp32, device: the transition product,
+ *         or NULL to skip it (the first piece of a sequence needs none).
+ * cu_seqlens_host (num_seqs + 1 int32, host) is required: the work list is
+ * built on the host.  The workspace (device, 256-byte aligned) must hold
+ * kda_segment_summary_workspace_size(desc) bytes.  Covers bf16 I/O with
+ * dk = dv = 128 (the tensor-core kernel), else KDA_ERR_UNSUPPORTED.
+ * KDA_ERR_INVALID_ARG for a bad descriptor, null or overlapping buffers or
+ * bad host seqlens; KDA_ERR_WORKSPACE for a short workspace.  Asynchronous on
+ * `stream`.
+ */
+size_t kda_segment_summary_workspace_size(const kda_fwd_desc *desc);
+kda_status kda_segment_summary(const kda_fwd_desc *desc, const void *q, const void *k,
+                               const void *v, const void *g, const void *beta, const float *S0,
+                               const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                               float *S_loc, float *M, void *workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
+
+/*
+ * Folds P = num_summaries piece summaries, in piece order, into the start
+ * state of piece P:  S = S_loc(0);  S = M(p) S + S_loc(p) for p = 1 .. P-1
+ * (M(0) is not read: the first piece's S_loc already starts from S0).
+ *   summaries: device fp32 [P][2][num_seqs][num_heads][dk][dv]: per piece,
+ *              S_loc then M (dk = dv), which is what an all-gather of each
+ *              rank's contiguous (S_loc, M) buffer produces.
+ *   S_in:      device fp32 [num_seqs][num_heads][dk][dv], written.
+ * Both 16-byte aligned and disjoint.  dk = dv = 128, else
+ * KDA_ERR_UNSUPPORTED; KDA_ERR_INVALID_ARG for P < 1 or bad sizes or
+ * pointers.  Asynchronous on `stream`.
+ */
+typedef struct {
+    int32_t num_seqs;
+    int32_t num_heads;
+    int32_t dk;
+    int32_t dv;
+    int32_t num_summaries;
+} kda_combine_desc;
+
+kda_status kda_state_combine(const kda_combine_desc *desc, const float *summaries, float *S_in,
+                             cudaStream_t stream);
+
+/*
  * Diagnostic (the pages have no counterpart): runs one bounded device-side
  * wait on a barrier that nothing completes, with the same wait primitive the
  * prefill kernels use, so that the timeout path can be exercised without a

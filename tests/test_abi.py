@@ -198,3 +198,53 @@ def test_spec_validation(lib):
     assert _verify(lib, _spec(), o=A + 40 * MB + 64) == 1      # o inside S
     assert _commit(lib, _spec(), S=A + 40 * MB + 8) == 1       # S not 16-byte aligned
     assert _commit(lib, _spec(), acc=A + 40 * MB + 4096) == 1  # counts inside S
+
+
+def _summary(lib, desc, S_loc=A + 40 * MB, M=A + 48 * MB, S0=None, cu_host=None, ws=A + 64 * MB,
+             ws_bytes=1 << 20, q=A):
+    cu_p = ctypes.cast(ctypes.c_void_p(A + 20 * MB), ctypes.POINTER(ctypes.c_int32))
+    if cu_host is None:
+        cu_host = (ctypes.c_int32 * 2)(0, desc.total_tokens)
+    return lib.kda_segment_summary(ctypes.byref(desc), q, A + 4 * MB, A + 8 * MB, A + 12 * MB,
+                                   A + 16 * MB, S0, cu_p, cu_host, S_loc, M, ws, ws_bytes, None)
+
+
+def test_segment_summary_validation(lib):
+    """Rejected on the host before any launch (fake pointers never touched)."""
+    d = _desc()
+    assert lib.kda_segment_summary_workspace_size(ctypes.byref(_desc(num_heads=0))) == SIZE_MAX
+    assert lib.kda_segment_summary_workspace_size(ctypes.byref(d)) % 256 == 0
+    assert _summary(lib, _desc(io_dtype=kda.KDA_FP32)) == 2          # tensor-core shape only
+    assert _summary(lib, _desc(dk=64)) == 2
+    assert _summary(lib, _desc(chunk=16)) == 2
+    assert _summary(lib, _desc(total_tokens=0)) == 1
+    assert _summary(lib, d, S_loc=None) == 1
+    assert lib.kda_segment_summary(ctypes.byref(d), A, A + 4 * MB, A + 8 * MB, A + 12 * MB,
+                                   A + 16 * MB, None, None, (ctypes.c_int32 * 2)(0, 64),
+                                   A + 40 * MB, None, A + 64 * MB, 1 << 20, None) == 1   # no cu_seqlens
+    assert lib.kda_segment_summary(ctypes.byref(d), A, A + 4 * MB, A + 8 * MB, A + 12 * MB,
+                                   A + 16 * MB, None,
+                                   ctypes.cast(ctypes.c_void_p(A + 20 * MB), ctypes.POINTER(ctypes.c_int32)),
+                                   None, A + 40 * MB, None, A + 64 * MB, 1 << 20, None) == 1  # no host copy
+    assert _summary(lib, d, cu_host=(ctypes.c_int32 * 2)(0, 63)) == 1    # host seqlens disagree
+    assert _summary(lib, d, q=A + 8) == 1                                 # q not 16-byte aligned
+    assert _summary(lib, d, S_loc=A + 4 * MB + 64) == 1                   # S_loc inside k
+    assert _summary(lib, d, M=A + 40 * MB + 4096) == 1                    # M overlaps S_loc
+    assert _summary(lib, d, ws=None) == 3
+    assert _summary(lib, d, ws_bytes=8) == 3
+    assert _summary(lib, d, ws=A + 64 * MB + 16) == 3                     # not 256-byte aligned
+    assert _summary(lib, d, ws=A + 40 * MB) == 1                          # workspace on S_loc
+
+
+def test_state_combine_validation(lib):
+    ok = dict(num_seqs=2, num_heads=2, dk=128, dv=128, num_summaries=3)
+    S_in = A + 200 * MB
+    for bad in (dict(num_seqs=0), dict(num_heads=0), dict(num_summaries=0), dict(dk=0)):
+        assert lib.kda_state_combine(ctypes.byref(kda.CombineDesc(**{**ok, **bad})), A, S_in, None) == 1
+    assert lib.kda_state_combine(ctypes.byref(kda.CombineDesc(**{**ok, "dk": 64, "dv": 64})), A, S_in,
+                                 None) == 2
+    d = kda.CombineDesc(**ok)
+    assert lib.kda_state_combine(ctypes.byref(d), None, S_in, None) == 1
+    assert lib.kda_state_combine(ctypes.byref(d), A, None, None) == 1
+    assert lib.kda_state_combine(ctypes.byref(d), A + 4, S_in, None) == 1     # misaligned
+    assert lib.kda_state_combine(ctypes.byref(d), A, A + MB, None) == 1        # S_in inside summaries
