@@ -531,6 +531,40 @@ def main():
         del sd, xs, Ssp, osp, accd
         torch.cuda.empty_cache()
 
+        if world > 1:
+            # context-parallel prefill (KCP): one 2^20-token sequence, H=32, cut into one
+            # piece per rank; the piece summaries cross ranks in one NCCL all-gather
+            from gated_delta_rule_136_b200 import kcp_chunk_fwd, split_pieces
+            Lk, Hk = 1 << 20, 32
+            a0, b0 = split_pieces([Lk], world)[rank][0]
+            wk = inputs.prefill_inputs([b0 - a0], H=Hk, dk=DK, dv=DV, device=dev, seed=100 + rank,
+                                       s0_std=None, g_mode="floor_stress")
+            runk = lambda: kcp_chunk_fwd(wk["q"], wk["k"], wk["v"], wk["g"], wk["beta"], wk["cu_seqlens"],
+                                         wk["cu_seqlens_host"])
+            for _ in range(2):
+                runk()
+            barrier()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 3
+            tw0 = time.time()
+            a.record(stream)
+            for _ in range(reps):
+                runk()
+            b.record(stream)
+            barrier()
+            if sampler:
+                sampler.mark(tw0, time.time())
+            if device_status(dev) != 0:
+                raise RuntimeError("device error word after context-parallel prefill")
+            ms = max_over_ranks(a.elapsed_time(b)) / reps
+            others[f"context-parallel prefill: 1 sequence x 2^20 tokens, H={Hk}, one piece per rank"] = {
+                "tokens": Lk, "ranks": world, "ms": ms, "tokens_per_s": Lk / (ms / 1e3),
+                "scaling": "strong",
+                "note": "summary (state from zero and transition product per piece), NCCL all-gather "
+                        "of the summaries, fold, rerun of each piece with outputs"}
+            del wk
+            torch.cuda.empty_cache()
+
     if sampler:
         sampler.stop()
         clocks = sampler.summary()
