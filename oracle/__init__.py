@@ -202,6 +202,60 @@ def transition_product_ref(q, k, v, g, beta, S0=None, scale=None, gate=None,
     return o, S_t
 
 
+def kda_bwd_ref(q, k, v, g, beta, do, cu_seqlens=None, S0=None, gate=None, dS_T=None,
+                scale=None, g_floor=-5.0):
+    """Gradients of the KDA forward, in fp64, by reverse-mode differentiation
+    (PyTorch autograd) of the token-by-token recurrence written out below.
+
+    The forward is the one :func:`kda_fwd_ref` computes, per head:
+        alpha_t = exp(max(g_t, g_floor)),  S' = Diag(alpha_t) S,
+        S = S' + beta_t k_t (v_t - S'^T k_t)^T,  o_t = scale S^T q_t [* sigmoid(gate_t)].
+    The gradient is that of L = sum(o * do) + sum(S_T * dS_T): the vector-
+    Jacobian product with the output gradient ``do`` [T,H,dv] and, optionally,
+    the final-state gradient ``dS_T`` [N,H,dk,dv].  Where g equals the floor the
+    derivative of max(g, floor) is taken as 1 (the clamp passes it through).
+    Returns a dict of float64 numpy arrays: dq, dk, dv, dg, dbeta, and dgate
+    and dS0 when ``gate`` / ``S0`` are given.  Meant for short sequences: the
+    recurrence is unrolled in the autograd graph.
+    """
+    import torch
+
+    def leaf(x):
+        return None if x is None else torch.from_numpy(_f64(x)).requires_grad_(True)
+
+    q, k, v, g, beta, gate, S0 = (leaf(x) for x in (q, k, v, g, beta, gate, S0))
+    do = torch.from_numpy(_f64(do))
+    dS_T = None if dS_T is None else torch.from_numpy(_f64(dS_T))
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    cu = ([0, T] if cu_seqlens is None else
+          [int(x) for x in np.asarray(cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens)])
+    if scale is None:
+        scale = 1.0 / np.sqrt(dk)
+    alpha = torch.exp(torch.clamp(g, min=g_floor))
+    loss = torch.zeros((), dtype=torch.float64)
+    for n in range(len(cu) - 1):
+        S = S0[n] if S0 is not None else torch.zeros(H, dk, dv, dtype=torch.float64)
+        for t in range(cu[n], cu[n + 1]):
+            S = alpha[t][:, :, None] * S
+            u = torch.einsum("hkv,hk->hv", S, k[t])
+            S = S + beta[t][:, None, None] * k[t][:, :, None] * (v[t] - u)[:, None, :]
+            o = scale * torch.einsum("hkv,hk->hv", S, q[t])
+            if gate is not None:
+                o = o * torch.sigmoid(gate[t])
+            loss = loss + (o * do[t]).sum()
+        if dS_T is not None:
+            loss = loss + (S * dS_T[n]).sum()
+    loss.backward()
+    out = {"dq": q.grad, "dk": k.grad, "dv": v.grad, "dg": g.grad, "dbeta": beta.grad}
+    if gate is not None:
+        out["dgate"] = gate.grad
+    if S0 is not None:
+        out["dS0"] = S0.grad
+    return {name: (np.zeros(x.shape) if x is None else x.numpy()) for name, x in
+            ((nm, out[nm]) for nm in out)}
+
+
 def rel_err(x, ref) -> float:
     """max|x - ref| / RMS(ref): the parity metric used throughout."""
     x = _f64(x)
