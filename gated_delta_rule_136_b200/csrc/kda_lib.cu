@@ -21,6 +21,7 @@
 #include "kda_spec.cuh"
 #include "kda_plan.cuh"
 #include "kda_segment.cuh"
+#include "kda_bwd.cuh"
 
 namespace {
 
@@ -600,6 +601,116 @@ kda_status kda_spec_commit(const kda_spec_desc *desc, const void *q, const void 
     cudaError_t e = d.io_dtype == KDA_BF16 ? dispatch_spec<__nv_bfloat16, true>(d.dk, d.dv, p, units, stream)
                                            : dispatch_spec<float, true>(d.dk, d.dv, p, units, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- backward
+namespace {
+struct BwdLayout {
+    size_t base = 0, states = 0, o = 0, fws = 0, scratch = 0, total = 0;
+    int64_t slots = 0;
+    size_t fws_bytes = 0;
+};
+
+BwdLayout bwd_layout(const kda_fwd_desc &d, const int32_t *cu) {
+    BwdLayout w;
+    for (int32_t n = 0; n < d.num_seqs; ++n) w.slots += ((int64_t)cu[n + 1] - cu[n]) / kda::bwd::CH;
+    const size_t esz = d.io_dtype == KDA_BF16 ? 2 : 4;
+    const size_t DD = (size_t)kda::bwd::D * kda::bwd::D;
+    size_t off = 0;
+    w.base = off;    off += align256(sizeof(int64_t) * (size_t)(d.num_seqs + 1));
+    w.states = off;  off += align256((size_t)w.slots * d.num_heads * DD * sizeof(float));
+    w.o = off;       off += align256((size_t)d.total_tokens * d.num_heads * kda::bwd::D * esz);
+    w.fws_bytes = fwd_workspace_bytes(&d, cu);
+    w.fws = off;     off += align256(w.fws_bytes);
+    w.scratch = off; off += align256((size_t)d.num_seqs * d.num_heads * kda::bwd::SCRATCH_FLOATS * sizeof(float));
+    w.total = off;
+    return w;
+}
+}  // namespace
+
+size_t kda_chunk_bwd_workspace_size(const kda_fwd_desc *desc, const int32_t *cu_seqlens_host) {
+    if (validate_fwd_desc(desc) != KDA_OK || !cu_seqlens_host) return SIZE_MAX;
+    if (validate_host_seqlens(desc, cu_seqlens_host) != KDA_OK) return SIZE_MAX;
+    return bwd_layout(*desc, cu_seqlens_host).total;
+}
+
+kda_status kda_chunk_bwd(const kda_fwd_desc *desc, const void *q, const void *k, const void *v,
+                         const void *g, const void *beta, const float *S0, const int32_t *cu_seqlens,
+                         const int32_t *cu_seqlens_host, const void *gate, const void *dout,
+                         const float *dS_T, void *dq, void *dk, void *dv, void *dg, void *dbeta,
+                         void *dgate, float *dS0, void *workspace, size_t workspace_bytes,
+                         cudaStream_t stream) {
+    kda_status st = validate_fwd_desc(desc);
+    if (st != KDA_OK) return st;
+    const kda_fwd_desc &d = *desc;
+    if (d.dk != kda::bwd::D || d.dv != kda::bwd::D) return KDA_ERR_UNSUPPORTED;
+    if (!cu_seqlens || !cu_seqlens_host) return KDA_ERR_INVALID_ARG;
+    if ((st = validate_host_seqlens(desc, cu_seqlens_host)) != KDA_OK) return st;
+    const bool any = d.total_tokens > 0;
+    if (any && (!q || !k || !v || !g || !beta || !dout || !dq || !dk || !dv || !dg || !dbeta))
+        return KDA_ERR_INVALID_ARG;
+    if (any && gate && !dgate) return KDA_ERR_INVALID_ARG;
+    const int32_t N = d.num_seqs, H = d.num_heads;
+    if ((int64_t)N * H > INT32_MAX) return KDA_ERR_INVALID_ARG;
+    for (const void *ptr : {static_cast<const void *>(S0), static_cast<const void *>(dS_T),
+                            static_cast<const void *>(dS0)})   // moved as float4
+        if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return KDA_ERR_INVALID_ARG;
+    const size_t esz = d.io_dtype == KDA_BF16 ? 2 : 4;
+    const int64_t T = d.total_tokens, DD = (int64_t)kda::bwd::D * kda::bwd::D;
+    const int64_t nk = T * H * 128 * (int64_t)esz, nb = T * H * (int64_t)esz, ns = (int64_t)N * H * DD * 4;
+    const Range ins[] = {range_of(q, nk), range_of(k, nk), range_of(g, nk), range_of(v, nk),
+                         range_of(beta, nb), range_of(gate, gate ? nk : 0), range_of(dout, nk),
+                         range_of(S0, S0 ? ns : 0), range_of(dS_T, dS_T ? ns : 0),
+                         range_of(cu_seqlens, 4 * (int64_t)(N + 1))};
+    const Range outs[] = {range_of(dq, nk), range_of(dk, nk), range_of(dv, nk), range_of(dg, nk),
+                          range_of(dbeta, nb), range_of(dgate, gate ? nk : 0), range_of(dS0, dS0 ? ns : 0)};
+    for (const Range &a : outs) {
+        for (const Range &b : ins)
+            if (overlaps(a, b)) return KDA_ERR_INVALID_ARG;
+    }
+    for (size_t i = 0; i < sizeof(outs) / sizeof(outs[0]); ++i)
+        for (size_t j = i + 1; j < sizeof(outs) / sizeof(outs[0]); ++j)
+            if (overlaps(outs[i], outs[j])) return KDA_ERR_INVALID_ARG;
+    const BwdLayout w = bwd_layout(d, cu_seqlens_host);
+    if (!workspace || workspace_bytes < w.total || reinterpret_cast<uintptr_t>(workspace) % 256 != 0)
+        return KDA_ERR_WORKSPACE;
+    const Range rw = range_of(workspace, (int64_t)w.total);
+    for (const Range &r : ins)
+        if (overlaps(rw, r)) return KDA_ERR_INVALID_ARG;
+    for (const Range &r : outs)
+        if (overlaps(rw, r)) return KDA_ERR_INVALID_ARG;
+    if (!any) {
+        // nothing to differentiate through: dS0 = dS_T (or zero)
+        if (!dS0) return KDA_OK;
+        const cudaError_t e = dS_T ? cudaMemcpyAsync(dS0, dS_T, (size_t)ns, cudaMemcpyDeviceToDevice, stream)
+                                   : cudaMemsetAsync(dS0, 0, (size_t)ns, stream);
+        return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
+
+    // the states at every 64-token chunk start: the forward with snapshots
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    std::vector<int64_t> base((size_t)N + 1, 0);
+    for (int32_t n = 0; n < N; ++n)
+        base[n + 1] = base[n] + ((int64_t)cu_seqlens_host[n + 1] - cu_seqlens_host[n]) / kda::bwd::CH;
+    int64_t *base_dev = reinterpret_cast<int64_t *>(ws + w.base);
+    if (cudaMemcpyAsync(base_dev, base.data(), base.size() * sizeof(int64_t), cudaMemcpyHostToDevice,
+                        stream) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    float *states = reinterpret_cast<float *>(ws + w.states);
+    const kda_snapshots sn{kda::bwd::CH, w.slots, base_dev, states};
+    st = chunk_fwd_impl(desc, &sn, q, k, v, g, beta, S0, cu_seqlens, cu_seqlens_host, nullptr,
+                        ws + w.o, nullptr, w.fws_bytes ? ws + w.fws : nullptr, w.fws_bytes, stream);
+    if (st != KDA_OK) return st;
+
+    kda::bwd::BwdParams bp{q, k, v, g, beta, gate, dout, S0, dS_T, cu_seqlens, states, base_dev,
+                           reinterpret_cast<float *>(ws + w.scratch), dq, dk, dv, dg, dbeta, dgate, dS0,
+                           H, d.scale, d.g_floor};
+    auto kern = d.io_dtype == KDA_BF16 ? kda::bwd::bwd_kernel<__nv_bfloat16> : kda::bwd::bwd_kernel<float>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kda::bwd::SMEM_BYTES) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    kern<<<(unsigned)((int64_t)N * H), kda::bwd::NT, kda::bwd::SMEM_BYTES, stream>>>(bp);
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------- context parallel (KCP)

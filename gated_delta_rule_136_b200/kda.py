@@ -29,7 +29,7 @@ EXPORTED_SYMBOLS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode
                     "kda_chunk_fwd_noalloc", "kda_selftest_bounded_wait",
                     "kda_chunk_fwd_snapshots", "kda_spec_verify", "kda_spec_commit",
                     "kda_segment_summary_workspace_size", "kda_segment_summary",
-                    "kda_state_combine")
+                    "kda_state_combine", "kda_chunk_bwd_workspace_size", "kda_chunk_bwd")
 NOALLOC_MAX_SEQS = 65536   # KDA_NOALLOC_MAX_SEQS in include/kda.h
 
 
@@ -119,6 +119,11 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.kda_segment_summary.restype = ctypes.c_int
         lib.kda_state_combine.argtypes = [ctypes.POINTER(CombineDesc), vp, vp, vp]
         lib.kda_state_combine.restype = ctypes.c_int
+        lib.kda_chunk_bwd_workspace_size.argtypes = [ctypes.POINTER(FwdDesc), i32p]
+        lib.kda_chunk_bwd_workspace_size.restype = sz
+        lib.kda_chunk_bwd.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, vp, vp, vp, i32p, i32p, vp,
+                                      vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.kda_chunk_bwd.restype = ctypes.c_int
         lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_int32, vp]
         lib.kda_selftest_bounded_wait.restype = ctypes.c_int
         _lib = lib
@@ -437,6 +442,59 @@ def state_combine(summaries, out=None):
     if st != KDA_OK:
         raise KDAError(st, "kda_state_combine")
     return S_in
+
+
+def chunk_bwd(q, k, v, g, beta, dout, cu_seqlens=None, cu_seqlens_host=None, S0=None, gate=None,
+              dS_T=None, scale=None, g_floor: float = -5.0, want_dS0: bool = True):
+    """``kda_chunk_bwd``: gradients of sum(o * dout) + sum(S_T * dS_T) through
+    the prefill of :func:`chunk_fwd` (same inputs and layouts; dk = dv = 128).
+    Returns a dict: dq, dk, dv, dg, dbeta (input dtype), dgate (if ``gate``)
+    and dS0 (fp32 [N,H,dk,dv], if ``want_dS0``)."""
+    _require_cuda()
+    lib = load_library()
+    device = q.device
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is None:
+        cu_seqlens_host = [0, T]
+        cu_seqlens = torch.tensor(cu_seqlens_host, dtype=torch.int32, device=device)
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.cpu().tolist()
+    cu_host = [int(x) for x in cu_seqlens_host]
+    N = len(cu_host) - 1
+    for name, t, shape in (("q", q, (T, H, dk)), ("k", k, (T, H, dk)), ("g", g, (T, H, dk)),
+                           ("v", v, (T, H, dv)), ("beta", beta, (T, H)), ("dout", dout, (T, H, dv))):
+        _check(t, name, shape, q.dtype, device)
+    if gate is not None:
+        _check(gate, "gate", (T, H, dv), q.dtype, device)
+    _check(cu_seqlens, "cu_seqlens", (N + 1,), torch.int32, device)
+    for name, t in (("S0", S0), ("dS_T", dS_T)):
+        if t is not None:
+            _check(t, name, (N, H, dk, dv), torch.float32, device)
+    desc = FwdDesc(total_tokens=T, num_seqs=N, num_heads=H, dk=dk, dv=dv, io_dtype=_io_dtype(q),
+                   scale=float(dk ** -0.5 if scale is None else scale), g_floor=float(g_floor),
+                   chunk=0, max_seqlen=0)
+    cu_h = (ctypes.c_int32 * (N + 1))(*cu_host)
+    ws_bytes = lib.kda_chunk_bwd_workspace_size(ctypes.byref(desc), cu_h)
+    if ws_bytes == ctypes.c_size_t(-1).value:
+        raise KDAError(1, "kda_chunk_bwd_workspace_size")
+    ws = torch.empty(max(int(ws_bytes), 256), dtype=torch.uint8, device=device)
+    out = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+           "dg": torch.empty_like(g), "dbeta": torch.empty_like(beta)}
+    if gate is not None:
+        out["dgate"] = torch.empty_like(gate)
+    if want_dS0:
+        out["dS0"] = torch.empty((N, H, dk, dv), dtype=torch.float32, device=device)
+    with torch.cuda.device(device):
+        st = lib.kda_chunk_bwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                               _ptr(S0), ctypes.cast(_ptr(cu_seqlens), ctypes.POINTER(ctypes.c_int32)),
+                               cu_h, _ptr(gate), _ptr(dout), _ptr(dS_T), _ptr(out["dq"]),
+                               _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
+                               _ptr(out.get("dgate")), _ptr(out.get("dS0")), _ptr(ws), ws.numel(),
+                               _stream_handle(device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_bwd")
+    return out
 
 
 def device_status(device=None) -> int:

@@ -268,6 +268,35 @@ kda_status kda_chunk_fwd_snapshots(const kda_fwd_desc *desc, const kda_snapshots
                                    cudaStream_t stream);
 
 /*
+ * Backward of the prefill (training; the report digest's FlashKDA serves
+ * training and prefill, section 基础设施): the gradients of
+ * L = sum(o * dout) + sum(S_T * dS_T) through the recurrence of
+ * kda_chunk_fwd, with the same descriptor, inputs and layouts.
+ *   dout   [T][H][dv], dtype of the inputs: gradient of o (required).
+ *   dS_T   fp32 [num_seqs][H][dk][dv]: gradient of the final state, or NULL (zero).
+ *   dq, dk, dg [T][H][dk]; dv [T][H][dv]; dbeta [T][H]: written, input dtype.
+ *   dgate  [T][H][dv]: written when gate is given (required then).
+ *   dS0    fp32 [num_seqs][H][dk][dv]: gradient of S0, written when not NULL.
+ * S0, dS_T and dS0 must be 16-byte aligned.
+ * The derivative of max(g, g_floor) is taken as 1 where g >= g_floor.
+ * cu_seqlens_host is required.  Internally the forward runs once with state
+ * snapshots every 64 tokens into the workspace, then one CTA per (sequence,
+ * head) recomputes each chunk's states from its snapshot and runs the
+ * recurrence backwards.  Workspace (device, 256-byte aligned):
+ * kda_chunk_bwd_workspace_size(desc, cu_seqlens_host) bytes (SIZE_MAX for a
+ * bad descriptor).  dk = dv = 128, else KDA_ERR_UNSUPPORTED;
+ * KDA_ERR_INVALID_ARG for null, overlapping or inconsistent arguments,
+ * KDA_ERR_WORKSPACE for a short or misaligned workspace.  Asynchronous.
+ */
+size_t kda_chunk_bwd_workspace_size(const kda_fwd_desc *desc, const int32_t *cu_seqlens_host);
+kda_status kda_chunk_bwd(const kda_fwd_desc *desc, const void *q, const void *k, const void *v,
+                         const void *g, const void *beta, const float *S0, const int32_t *cu_seqlens,
+                         const int32_t *cu_seqlens_host, const void *gate, const void *dout,
+                         const float *dS_T, void *dq, void *dk, void *dv, void *dg, void *dbeta,
+                         void *dgate, float *dS0, void *workspace, size_t workspace_bytes,
+                         cudaStream_t stream);
+
+/*
  * Context-parallel prefill across GPUs (KCP, Kimi K3 report digest, section
  * 基础设施): a long sequence is cut into contiguous pieces, one per rank.
  * Over a piece the state map is affine, S_end = M S_start + S_loc, with M the

@@ -248,3 +248,29 @@ def test_state_combine_validation(lib):
     assert lib.kda_state_combine(ctypes.byref(d), A, None, None) == 1
     assert lib.kda_state_combine(ctypes.byref(d), A + 4, S_in, None) == 1     # misaligned
     assert lib.kda_state_combine(ctypes.byref(d), A, A + MB, None) == 1        # S_in inside summaries
+
+
+def test_chunk_bwd_validation(lib):
+    """Rejected on the host before any launch (fake pointers never touched)."""
+    d = _desc(total_tokens=64)
+    cu_host = (ctypes.c_int32 * 2)(0, 64)
+    assert lib.kda_chunk_bwd_workspace_size(ctypes.byref(d), None) == SIZE_MAX
+    need = lib.kda_chunk_bwd_workspace_size(ctypes.byref(d), cu_host)
+    assert need != SIZE_MAX and need % 256 == 0
+    cu_p = ctypes.cast(ctypes.c_void_p(A + 20 * MB), ctypes.POINTER(ctypes.c_int32))
+
+    def bwd(desc=d, cu_h=cu_host, dout=A + 30 * MB, dq=A + 32 * MB, gate=None, dgate=None, S0=None,
+            dS0=None, ws=A + 256 * MB, ws_bytes=1 << 34):
+        return lib.kda_chunk_bwd(ctypes.byref(desc), A, A + 4 * MB, A + 8 * MB, A + 12 * MB, A + 16 * MB,
+                                 S0, cu_p, cu_h, gate, dout, None, dq, A + 34 * MB, A + 36 * MB,
+                                 A + 38 * MB, A + 40 * MB, dgate, dS0, ws, ws_bytes, None)
+    assert bwd(desc=_desc(total_tokens=64, dk=64)) == 2
+    assert bwd(cu_h=None) == 1
+    assert bwd(dout=None) == 1
+    assert bwd(dq=A + 4 * MB + 64) == 1                     # dq inside k
+    assert bwd(gate=A + 50 * MB) == 1                       # gate without dgate
+    assert bwd(S0=A + 60 * MB + 4) == 1                     # S0 not 16-byte aligned
+    assert bwd(dS0=A + 32 * MB) == 1                        # dS0 on dq
+    assert bwd(ws=None) == 3
+    assert bwd(ws_bytes=need - 256) == 3
+    assert bwd(ws=A + 8 * MB) == 1                          # workspace on v

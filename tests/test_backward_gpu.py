@@ -1,0 +1,68 @@
+"""Backward of the prefill (kda_chunk_bwd) against the oracle's fp64 gradients
+(autograd through the token recurrence, itself pinned by finite differences):
+dq, dk, dv, dg, dbeta, dgate and dS0 for L = sum(o * dout) + sum(S_T * dS_T).
+Ragged sequences cover partial chunks and sub-blocks and an empty sequence;
+fp32 I/O runs the CUDA-core forward for the checkpoints, bf16 I/O the
+tensor-core one."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_136_b200 import chunk_bwd, device_status, inputs
+from parity import TOL_BF16, TOL_FP32, rel_max, rel_max_beyond_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _cpu(x):
+    return None if x is None else x.detach().to("cpu")
+
+
+def _run(lengths, H, dtype, seed, gate=True, s0=True, ds_t=True, heads=None):
+    inp = inputs.prefill_inputs(lengths, H=H, dk=128, dv=128, dtype=dtype, device="cuda", seed=seed,
+                                s0_std=0.05 if s0 else None, gate=gate)
+    gen = torch.Generator(device="cuda").manual_seed(seed + 1)
+    dout = torch.randn(inp["v"].shape, generator=gen, device="cuda").to(dtype)
+    N = len(lengths)
+    dS_T = (0.1 * torch.randn((N, H, 128, 128), generator=gen, device="cuda")) if ds_t else None
+    got = chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], dout,
+                    cu_seqlens=inp["cu_seqlens"], cu_seqlens_host=inp["cu_seqlens_host"], S0=inp["S0"],
+                    gate=inp["gate"], dS_T=dS_T)
+    assert device_status() == 0
+    sel = (lambda t: t) if heads is None else (lambda t: None if t is None else t[:, heads].contiguous())
+    ref = oracle.kda_bwd_ref(*(sel(_cpu(inp[n])) for n in ("q", "k", "v", "g", "beta")), sel(_cpu(dout)),
+                             cu_seqlens=np.array(inp["cu_seqlens_host"]), S0=sel(_cpu(inp["S0"])),
+                             gate=sel(_cpu(inp["gate"])), dS_T=sel(_cpu(dS_T)))
+    return {n: sel(t) for n, t in got.items()}, ref
+
+
+def _check(got, ref, dtype):
+    for name in ("dq", "dk", "dv", "dg", "dbeta", "dgate"):
+        if name not in ref:
+            continue
+        if dtype == torch.float32:
+            assert rel_max(got[name], ref[name]) <= TOL_FP32, name
+        else:
+            assert rel_max_beyond_bf16(got[name], ref[name]) <= TOL_BF16, name
+    if "dS0" in ref:
+        assert rel_max(got["dS0"], ref["dS0"]) <= (TOL_FP32 if dtype == torch.float32 else TOL_BF16)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_backward_matches_oracle(dtype):
+    got, ref = _run([150, 0, 70, 64], H=2, dtype=dtype, seed=101)
+    _check(got, ref, dtype)
+
+
+def test_backward_without_gate_s0_or_final_gradient():
+    got, ref = _run([97, 128], H=2, dtype=torch.float32, seed=103, gate=False, s0=False, ds_t=False)
+    _check(got, ref, torch.float32)
+    assert "dgate" not in got
+
+
+def test_backward_full_length_sampled_head():
+    """The bf16 workload's sequence length (4096) and head count; one head is
+    checked against the oracle over the whole sequence."""
+    got, ref = _run([4096], H=32, dtype=torch.bfloat16, seed=107, heads=[5])
+    _check(got, ref, torch.bfloat16)
