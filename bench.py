@@ -531,6 +531,40 @@ def main():
         del sd, xs, Ssp, osp, accd
         torch.cuda.empty_cache()
 
+        # backward of the headline prefill (training): gradients of sum(o * dout)
+        from gated_delta_rule_136_b200 import chunk_bwd
+        xb = inputs.prefill_inputs([T] * B, H=H, dk=DK, dv=DV, device=dev, seed=rank)
+        gen = torch.Generator(device=dev).manual_seed(200 + rank)
+        dout = torch.randn(xb["v"].shape, generator=gen, device=dev).to(torch.bfloat16)
+        runb = lambda: chunk_bwd(xb["q"], xb["k"], xb["v"], xb["g"], xb["beta"], dout,
+                                 cu_seqlens=xb["cu_seqlens"], cu_seqlens_host=xb["cu_seqlens_host"],
+                                 want_dS0=False)
+        for _ in range(2):
+            runb()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 3
+        tw0 = time.time()
+        a.record(stream)
+        for _ in range(reps):
+            runb()
+        b.record(stream)
+        barrier()
+        if sampler:
+            sampler.mark(tw0, time.time())
+        if device_status(dev) != 0:
+            raise RuntimeError("device error word after backward")
+        ms = max_over_ranks(a.elapsed_time(b)) / reps
+        # inputs q, k, g, v, dout and beta read once, dq, dk, dg, dv and dbeta written once
+        byts = B * T * H * (5 * DK * 2 + 2 + 4 * DK * 2 + 2)
+        others[f"backward B={B} T={T} H={H} (gradients of sum(o * dout), bf16)"] = {
+            "tokens": B * T, "ms": ms, "tokens_per_s": world * B * T / (ms / 1e3),
+            "alg_gbs": byts / (ms / 1e3) / 1e9, "roofline_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "note": "forward with 64-token state snapshots, then per (sequence, head) a CUDA-core "
+                    "replay of each chunk and the reverse recurrence"}
+        del xb, dout
+        torch.cuda.empty_cache()
+
         if world > 1:
             # context-parallel prefill (KCP): one 2^20-token sequence, H=32, cut into one
             # piece per rank; the piece summaries cross ranks in one NCCL all-gather

@@ -60,10 +60,31 @@ constexpr int SM_SCAL = SM_RED + 2 * NW * 3 * D;        // [2][NW][2]
 constexpr int SM_FLOATS = SM_SCAL + 2 * NW * 2;
 constexpr size_t SMEM_BYTES = (size_t)SM_FLOATS * sizeof(float);
 
-__device__ __forceinline__ float warp_sum(float x) {
+// Sums x[0..7] over the warp's 32 lanes by halving the vector at each of the
+// first three exchange steps (9 shuffles instead of 40).  On return lane l
+// holds the total of value j(l) = 4 b4 + 2 b3 + b2 (b = the bits of l).
+__device__ __forceinline__ float warp_reduce8(const float (&x)[CPW], int lane) {
+    static_assert(CPW == 8, "eight values per lane");
+    const bool h4 = lane & 16, h3 = lane & 8, h2 = lane & 4;
+    float y[4], z[2];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-    return x;
+    for (int i = 0; i < 4; ++i)
+        y[i] = (h4 ? x[i + 4] : x[i]) + __shfl_xor_sync(0xffffffffu, h4 ? x[i] : x[i + 4], 16);
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+        z[i] = (h3 ? y[i + 2] : y[i]) + __shfl_xor_sync(0xffffffffu, h3 ? y[i] : y[i + 2], 8);
+    float w = (h2 ? z[1] : z[0]) + __shfl_xor_sync(0xffffffffu, h2 ? z[0] : z[1], 4);
+    w += __shfl_xor_sync(0xffffffffu, w, 2);
+    w += __shfl_xor_sync(0xffffffffu, w, 1);
+    return w;
+}
+__device__ __forceinline__ int reduce8_lane(int j) { return ((j >> 2) << 4) | (((j >> 1) & 1) << 3) | ((j & 1) << 2); }
+__device__ __forceinline__ int reduce8_index(int lane) { return ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1); }
+// every lane gets all eight totals
+__device__ __forceinline__ void warp_allreduce8(float (&x)[CPW], int lane) {
+    const float w = warp_reduce8(x, lane);
+#pragma unroll
+    for (int j = 0; j < CPW; ++j) x[j] = __shfl_sync(0xffffffffu, w, reduce8_lane(j));
 }
 
 template <typename TIO>
@@ -143,8 +164,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_kernel(BwdParams p)
                 u[c] = fmaf(s[r][c], kk[r], u[c]);
             }
         }
-#pragma unroll
-        for (int c = 0; c < CPW; ++c) u[c] = warp_sum(u[c]);
+        warp_allreduce8(u, lane);
         const float bt = sm[SM_B + t];
 #pragma unroll
         for (int c = 0; c < CPW; ++c) {
@@ -162,14 +182,15 @@ __global__ void __launch_bounds__(NT, 1) bwd_kernel(BwdParams p)
 #pragma unroll
                 for (int c = 0; c < CPW; ++c) o[c] = fmaf(s[r][c], qq, o[c]);
             }
+            const float ot = warp_reduce8(o, lane);
+            if ((lane & 3) == 0) {               // the eight lanes that hold a total
+                const int c = reduce8_index(lane);
+                sm[SM_OR + t * D + c0 + c] = p.scale * ot;
+            }
+            if (lane < CPW) {
 #pragma unroll
-            for (int c = 0; c < CPW; ++c) o[c] = warp_sum(o[c]);
-            if (lane == 0) {
-#pragma unroll
-                for (int c = 0; c < CPW; ++c) {
-                    sm[SM_U + t * D + c0 + c] = u[c];
-                    sm[SM_OR + t * D + c0 + c] = p.scale * o[c];
-                }
+                for (int c = 0; c < CPW; ++c)
+                    if (lane == c) sm[SM_U + t * D + c0 + c] = u[c];
             }
         }
     };
@@ -231,8 +252,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_kernel(BwdParams p)
                         rr[c] = fmaf(dS[r][c], kk[r], rr[c]);
                     }
                 }
-#pragma unroll
-                for (int c = 0; c < CPW; ++c) rr[c] = warp_sum(rr[c]);
+                warp_allreduce8(rr, lane);
                 float *red = sm + SM_RED + par * (NW * 3 * D) + w * 3 * D;
                 const float *Sprev = scr_st + (int64_t)t * D * D;
 #pragma unroll
