@@ -38,6 +38,7 @@ B, T, H, DK, DV = 8, 4096, 32, 128, 128
 CHUNK_ALG = 64
 # workload (decode)
 DEC_B, DEC_H, DEC_STEPS = 512, 64, 1000
+EXTRA_WORKLOADS = ("varlen", "long", "snapshots", "spec", "backward", "kcp")
 
 
 def flops_per_token_head(dk=DK, dv=DV, C=CHUNK_ALG):
@@ -60,6 +61,10 @@ PROFILED_TRAFFIC = {
                               "profile": "profiles/chunk_tc_kernel_prefill_4x4096x16.md"},
     "csrc/kda_decode.cuh": {"sha1": "8e75484b34f3", "bytes_per_head_step": (273.707520e6 + 212.401408e6) / 4096,
                             "profile": "profiles/decode_kernel_64x64.md"},
+    # speculative verify (4 draft tokens) + commit (3) at batch 128 x 64 heads: per head and round
+    "csrc/kda_spec.cuh": {"sha1": "5f78f5eaf7b5",
+                          "bytes_per_head_round": (579.116800e6 + 4.305920e6 + 555.884544e6 + 477.843968e6) / 8192,
+                          "profile": "profiles/spec_kernel_verify_commit_128x64.md"},
 }
 
 
@@ -242,13 +247,20 @@ def main():
     ap.add_argument("--heads", type=int, default=H)
     ap.add_argument("--decode-batch", type=int, default=DEC_B)
     ap.add_argument("--decode-steps", type=int, default=DEC_STEPS)
+    ap.add_argument("--extra", default="",
+                    help="comma-separated extra workloads to time: " + ", ".join(EXTRA_WORKLOADS))
     ap.add_argument("--all-workloads", action="store_true",
                     help="also time the varlen (64 x [512, 32768] x 64 heads) and the "
                          "1M-token x 32-head floor-stress prefill, the headline prefill "
-                         "with state snapshots every 512 tokens, and speculative-decode "
-                         "verify/commit rounds")
+                         "with state snapshots every 512 tokens, speculative-decode "
+                         "verify/commit rounds, the backward of the headline prefill and, "
+                         "with more than one rank, the context-parallel prefill")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    extras = set(EXTRA_WORKLOADS) if args.all_workloads else {x for x in args.extra.split(",") if x}
+    if extras - set(EXTRA_WORKLOADS):
+        ap.error(f"--extra: unknown workload(s) {sorted(extras - set(EXTRA_WORKLOADS))}; "
+                 f"choose from {', '.join(EXTRA_WORKLOADS)}")
     B, T, H = args.batch, args.seqlen, args.heads
     DEC_B, DEC_STEPS = args.decode_batch, args.decode_steps
     if args.impl == "reference":
@@ -412,7 +424,7 @@ def main():
         torch.cuda.empty_cache()
 
     others = None
-    if args.all_workloads:
+    if extras:
         others = {}
         cases = {
             "varlen 64 sequences, lengths U[512, 32768], H=64, S0 ~ N(0, 0.02)":
@@ -421,6 +433,8 @@ def main():
             "1 sequence x 2^20 tokens, H=32, g ~ -5 U(0.8, 1)":
                 dict(lengths=[1 << 20], H=32, s0_std=None, g_mode="floor_stress"),
         }
+        keys = dict(zip(cases, ("varlen", "long")))
+        cases = {name: c for name, c in cases.items() if keys[name] in extras}
         for name, c in cases.items():
             w = inputs.prefill_inputs(c["lengths"], H=c["H"], dk=DK, dv=DV, device=dev, seed=rank,
                                       s0_std=c["s0_std"], g_mode=c["g_mode"])
@@ -455,117 +469,122 @@ def main():
             del w, ow, Sw, wsw
             torch.cuda.empty_cache()
 
-        # the headline prefill with state snapshots every 512 tokens (prefix-cache hook)
-        from gated_delta_rule_136_b200 import chunk_fwd_snapshots
-        w = inputs.prefill_inputs([T] * B, H=H, dk=DK, dv=DV, device=dev, seed=rank)
-        interval = 512
-        run = lambda: chunk_fwd_snapshots(w["q"], w["k"], w["v"], w["g"], w["beta"], interval,
-                                          cu_seqlens=w["cu_seqlens"],
-                                          cu_seqlens_host=w["cu_seqlens_host"])
-        for _ in range(2):
-            run()
-        barrier()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 5
-        tw0 = time.time()
-        a.record(stream)
-        for _ in range(reps):
-            run()
-        b.record(stream)
-        barrier()
-        if sampler:
-            sampler.mark(tw0, time.time())
-        if device_status(dev) != 0:
-            raise RuntimeError("device error word after the snapshot prefill")
-        ms = max_over_ranks(a.elapsed_time(b)) / reps
-        nsnap = B * (T // interval)
-        byts = B * T * H * bytes_per_token_head() + B * H * DK * DV * 4 + nsnap * H * DK * DV * 4
-        others[f"prefill B={B} T={T} H={H} with state snapshots every {interval} tokens"] = {
-            "tokens": B * T, "ms": ms, "tokens_per_s": world * B * T / (ms / 1e3),
-            "snapshot_bytes": nsnap * H * DK * DV * 4, "alg_gbs": byts / (ms / 1e3) / 1e9,
-            "roofline_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-            "note": "timed through the Python binding, which allocates the snapshot buffer and "
-                    "uploads the slot table on every call"}
-        del w
-        torch.cuda.empty_cache()
+        if "snapshots" in extras:
+            # the headline prefill with state snapshots every 512 tokens (prefix-cache hook)
+            from gated_delta_rule_136_b200 import chunk_fwd_snapshots
+            w = inputs.prefill_inputs([T] * B, H=H, dk=DK, dv=DV, device=dev, seed=rank)
+            interval = 512
+            run = lambda: chunk_fwd_snapshots(w["q"], w["k"], w["v"], w["g"], w["beta"], interval,
+                                              cu_seqlens=w["cu_seqlens"],
+                                              cu_seqlens_host=w["cu_seqlens_host"])
+            for _ in range(2):
+                run()
+            barrier()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 5
+            tw0 = time.time()
+            a.record(stream)
+            for _ in range(reps):
+                run()
+            b.record(stream)
+            barrier()
+            if sampler:
+                sampler.mark(tw0, time.time())
+            if device_status(dev) != 0:
+                raise RuntimeError("device error word after the snapshot prefill")
+            ms = max_over_ranks(a.elapsed_time(b)) / reps
+            nsnap = B * (T // interval)
+            byts = B * T * H * bytes_per_token_head() + B * H * DK * DV * 4 + nsnap * H * DK * DV * 4
+            others[f"prefill B={B} T={T} H={H} with state snapshots every {interval} tokens"] = {
+                "tokens": B * T, "ms": ms, "tokens_per_s": world * B * T / (ms / 1e3),
+                "snapshot_bytes": nsnap * H * DK * DV * 4, "alg_gbs": byts / (ms / 1e3) / 1e9,
+                "roofline_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                "note": "timed through the Python binding, which allocates the snapshot buffer and "
+                        "uploads the slot table on every call"}
+            del w
+            torch.cuda.empty_cache()
 
-        # speculative decode: verify D = 4 draft tokens, commit 3, per round (decode batch)
-        from gated_delta_rule_136_b200 import spec_commit, spec_verify
-        Dd = 4
-        sd = inputs.prefill_inputs([Dd] * DEC_B, H=DEC_H, dk=DK, dv=DV, device=dev, seed=rank,
-                                   s0_std=0.02, gate=True)
-        xs = {n: sd[n].view(DEC_B, Dd, *sd[n].shape[1:]) for n in ("q", "k", "v", "g", "beta", "gate")}
-        Ssp = sd["S0"]
-        osp = torch.empty_like(xs["v"])
-        accd = torch.full((DEC_B,), 3, dtype=torch.int32, device=dev)
+        if "spec" in extras:
+            # speculative decode: verify D = 4 draft tokens, commit 3, per round (decode batch)
+            from gated_delta_rule_136_b200 import spec_commit, spec_verify
+            Dd = 4
+            sd = inputs.prefill_inputs([Dd] * DEC_B, H=DEC_H, dk=DK, dv=DV, device=dev, seed=rank,
+                                       s0_std=0.02, gate=True)
+            xs = {n: sd[n].view(DEC_B, Dd, *sd[n].shape[1:]) for n in ("q", "k", "v", "g", "beta", "gate")}
+            Ssp = sd["S0"]
+            osp = torch.empty_like(xs["v"])
+            accd = torch.full((DEC_B,), 3, dtype=torch.int32, device=dev)
 
-        def spec_round():
-            spec_verify(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], Ssp, gate=xs["gate"], out=osp)
-            spec_commit(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], Ssp, accd)
+            def spec_round():
+                spec_verify(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], Ssp, gate=xs["gate"], out=osp)
+                spec_commit(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], Ssp, accd)
 
-        for _ in range(args.warmup):
-            spec_round()
-        barrier()
-        rounds = 50
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        tw0 = time.time()
-        a.record(stream)
-        for _ in range(rounds):
-            spec_round()
-        b.record(stream)
-        barrier()
-        if sampler:
-            sampler.mark(tw0, time.time())
-        if device_status(dev) != 0:
-            raise RuntimeError("device error word after speculative decode")
-        ms = max_over_ranks(a.elapsed_time(b)) / rounds
-        heads = DEC_B * DEC_H
-        byts = heads * (3 * DK * DV * 4 + Dd * (2 * (3 * DK + DV + 1) + 2 * DV + 2 * DV)
-                        + 3 * 2 * (3 * DK + DV + 1))
-        others[f"speculative decode batch={DEC_B} H={DEC_H}: verify {Dd} draft tokens, commit 3"] = {
-            "rounds_per_s": world * 1e3 / ms, "ms_per_round": ms,
-            "verified_tokens_per_s": world * DEC_B * Dd / (ms / 1e3),
-            "alg_gbs": byts / (ms / 1e3) / 1e9, "roofline_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-            "note": "the state crosses HBM three times per round (verify read, commit read and "
-                    "write) instead of twice per token"}
-        del sd, xs, Ssp, osp, accd
-        torch.cuda.empty_cache()
+            for _ in range(args.warmup):
+                spec_round()
+            barrier()
+            rounds = 50
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            tw0 = time.time()
+            a.record(stream)
+            for _ in range(rounds):
+                spec_round()
+            b.record(stream)
+            barrier()
+            if sampler:
+                sampler.mark(tw0, time.time())
+            if device_status(dev) != 0:
+                raise RuntimeError("device error word after speculative decode")
+            ms = max_over_ranks(a.elapsed_time(b)) / rounds
+            heads = DEC_B * DEC_H
+            byts = heads * (3 * DK * DV * 4 + Dd * (2 * (3 * DK + DV + 1) + 2 * DV + 2 * DV)
+                            + 3 * 2 * (3 * DK + DV + 1))
+            others[f"speculative decode batch={DEC_B} H={DEC_H}: verify {Dd} draft tokens, commit 3"] = {
+                "rounds_per_s": world * 1e3 / ms, "ms_per_round": ms,
+                "verified_tokens_per_s": world * DEC_B * Dd / (ms / 1e3),
+                "alg_gbs": byts / (ms / 1e3) / 1e9, "roofline_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                "alg_bytes_per_round": byts,
+                "traffic": profiled_traffic("csrc/kda_spec.cuh", "bytes_per_head_round", heads),
+                "note": "the state crosses HBM three times per round (verify read, commit read and "
+                        "write) instead of twice per token"}
+            del sd, xs, Ssp, osp, accd
+            torch.cuda.empty_cache()
 
-        # backward of the headline prefill (training): gradients of sum(o * dout)
-        from gated_delta_rule_136_b200 import chunk_bwd
-        xb = inputs.prefill_inputs([T] * B, H=H, dk=DK, dv=DV, device=dev, seed=rank)
-        gen = torch.Generator(device=dev).manual_seed(200 + rank)
-        dout = torch.randn(xb["v"].shape, generator=gen, device=dev).to(torch.bfloat16)
-        runb = lambda: chunk_bwd(xb["q"], xb["k"], xb["v"], xb["g"], xb["beta"], dout,
-                                 cu_seqlens=xb["cu_seqlens"], cu_seqlens_host=xb["cu_seqlens_host"],
-                                 want_dS0=False)
-        for _ in range(2):
-            runb()
-        barrier()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 3
-        tw0 = time.time()
-        a.record(stream)
-        for _ in range(reps):
-            runb()
-        b.record(stream)
-        barrier()
-        if sampler:
-            sampler.mark(tw0, time.time())
-        if device_status(dev) != 0:
-            raise RuntimeError("device error word after backward")
-        ms = max_over_ranks(a.elapsed_time(b)) / reps
-        # inputs q, k, g, v, dout and beta read once, dq, dk, dg, dv and dbeta written once
-        byts = B * T * H * (5 * DK * 2 + 2 + 4 * DK * 2 + 2)
-        others[f"backward B={B} T={T} H={H} (gradients of sum(o * dout), bf16)"] = {
-            "tokens": B * T, "ms": ms, "tokens_per_s": world * B * T / (ms / 1e3),
-            "alg_gbs": byts / (ms / 1e3) / 1e9, "roofline_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-            "note": "forward with 64-token state snapshots, then per (sequence, head) a CUDA-core "
-                    "replay of each chunk and the reverse recurrence"}
-        del xb, dout
-        torch.cuda.empty_cache()
+        if "backward" in extras:
+            # backward of the headline prefill (training): gradients of sum(o * dout)
+            from gated_delta_rule_136_b200 import chunk_bwd
+            xb = inputs.prefill_inputs([T] * B, H=H, dk=DK, dv=DV, device=dev, seed=rank)
+            gen = torch.Generator(device=dev).manual_seed(200 + rank)
+            dout = torch.randn(xb["v"].shape, generator=gen, device=dev).to(torch.bfloat16)
+            runb = lambda: chunk_bwd(xb["q"], xb["k"], xb["v"], xb["g"], xb["beta"], dout,
+                                     cu_seqlens=xb["cu_seqlens"], cu_seqlens_host=xb["cu_seqlens_host"],
+                                     want_dS0=False)
+            for _ in range(2):
+                runb()
+            barrier()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 3
+            tw0 = time.time()
+            a.record(stream)
+            for _ in range(reps):
+                runb()
+            b.record(stream)
+            barrier()
+            if sampler:
+                sampler.mark(tw0, time.time())
+            if device_status(dev) != 0:
+                raise RuntimeError("device error word after backward")
+            ms = max_over_ranks(a.elapsed_time(b)) / reps
+            # inputs q, k, g, v, dout and beta read once, dq, dk, dg, dv and dbeta written once
+            byts = B * T * H * (5 * DK * 2 + 2 + 4 * DK * 2 + 2)
+            others[f"backward B={B} T={T} H={H} (gradients of sum(o * dout), bf16)"] = {
+                "tokens": B * T, "ms": ms, "tokens_per_s": world * B * T / (ms / 1e3),
+                "alg_gbs": byts / (ms / 1e3) / 1e9, "roofline_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                "note": "forward with 64-token state snapshots, then per (sequence, head) a CUDA-core "
+                        "replay of each chunk and the reverse recurrence"}
+            del xb, dout
+            torch.cuda.empty_cache()
 
-        if world > 1:
+        if world > 1 and "kcp" in extras:
             # context-parallel prefill (KCP): one 2^20-token sequence, H=32, cut into one
             # piece per rank; the piece summaries cross ranks in one NCCL all-gather
             from gated_delta_rule_136_b200 import kcp_chunk_fwd, split_pieces
