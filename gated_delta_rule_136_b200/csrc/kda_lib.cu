@@ -929,3 +929,200 @@ extern "C" kda_status kda_chunk_fwd_noalloc(const kda_fwd_desc *desc, const void
     e = launch_prefill(d, q, k, v, g, beta, S0, cu_seqlens, seq_order, gate, o, S_T, kda::SnapOut{nullptr, nullptr, 0, 64}, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------------------
+// Prefill from and to host memory (kda_chunk_fwd_host).  The batch is cut
+// into groups of whole sequences; the host-to-device copy of group i+1, the
+// prefill of group i and the device-to-host copy of group i-1 run on three
+// streams (the two copy engines and the SMs), with input and output slots
+// double-buffered in the caller's device workspace.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kHostGroups = 8;
+
+struct HostPipe {
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t entry = nullptr, in_ready[2] = {}, computed[2] = {}, out_free[2] = {};
+};
+std::mutex g_pipe_mutex;          // held while a call enqueues its work
+HostPipe g_pipe[kMaxDevices];
+
+cudaError_t host_pipe(HostPipe **out) {   // caller holds g_pipe_mutex
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    HostPipe &p = g_pipe[dev];
+    if (!p.h2d) {
+        HostPipe n;
+        if ((e = cudaStreamCreateWithFlags(&n.h2d, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        if ((e = cudaStreamCreateWithFlags(&n.d2h, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        cudaEvent_t *evs[] = {&n.entry, &n.in_ready[0], &n.in_ready[1], &n.computed[0], &n.computed[1],
+                              &n.out_free[0], &n.out_free[1]};
+        for (cudaEvent_t *ev : evs)
+            if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+        p = n;
+    }
+    *out = &p;
+    return cudaSuccess;
+}
+
+struct HostGroup {
+    int32_t s0, s1;     // sequences [s0, s1)
+    int64_t t0, t1;     // tokens [t0, t1)
+    size_t cu_off;      // this group's relative cu_seqlens in the cu region (entries)
+};
+
+struct HostLayout {
+    std::vector<HostGroup> groups;
+    std::vector<int32_t> cu_rel;                 // every group's cu_seqlens, relative to its start
+    int64_t tmax = 0, smax = 0;
+    size_t cu = 0, in[2] = {}, out[2] = {}, fws = 0, fws_bytes = 0, total = 0;
+    size_t off_q = 0, off_k = 0, off_g = 0, off_v = 0, off_b = 0, off_z = 0, off_s0 = 0, in_bytes = 0;
+    size_t off_o = 0, off_st = 0, out_bytes = 0;
+};
+
+kda_fwd_desc group_desc(const kda_fwd_desc &d, const HostGroup &gr) {
+    kda_fwd_desc g = d;
+    g.total_tokens = gr.t1 - gr.t0;
+    g.num_seqs = gr.s1 - gr.s0;
+    return g;
+}
+
+HostLayout host_layout(const kda_fwd_desc &d, const int32_t *cu, bool gate, bool s0, bool st) {
+    HostLayout w;
+    const int32_t N = d.num_seqs;
+    const int G = std::min<int32_t>(N, kHostGroups);
+    const int64_t T = d.total_tokens;
+    int32_t s = 0;
+    for (int gi = 0; gi < G; ++gi) {
+        int32_t e = s + 1;
+        const int64_t target = T * (gi + 1) / G;
+        while (e < N - (G - 1 - gi) && cu[e] < target) ++e;
+        if (gi == G - 1) e = N;
+        w.groups.push_back(HostGroup{s, e, cu[s], cu[e], w.cu_rel.size()});
+        for (int32_t n = s; n <= e; ++n) w.cu_rel.push_back(cu[n] - cu[s]);
+        w.tmax = std::max<int64_t>(w.tmax, (int64_t)cu[e] - cu[s]);
+        w.smax = std::max<int64_t>(w.smax, e - s);
+        s = e;
+    }
+    const size_t esz = d.io_dtype == KDA_BF16 ? 2 : 4, H = (size_t)d.num_heads;
+    const size_t tm = (size_t)w.tmax, sm = (size_t)w.smax, DKV = (size_t)d.dk * d.dv * 4;
+    size_t o = 0;
+    w.off_q = o; o += align256(tm * H * d.dk * esz);
+    w.off_k = o; o += align256(tm * H * d.dk * esz);
+    w.off_g = o; o += align256(tm * H * d.dk * esz);
+    w.off_v = o; o += align256(tm * H * d.dv * esz);
+    w.off_b = o; o += align256(tm * H * esz);
+    w.off_z = o; o += gate ? align256(tm * H * d.dv * esz) : 0;
+    w.off_s0 = o; o += s0 ? align256(sm * H * DKV) : 0;
+    w.in_bytes = o;
+    o = 0;
+    w.off_o = o; o += align256(tm * H * d.dv * esz);
+    w.off_st = o; o += st ? align256(sm * H * DKV) : 0;
+    w.out_bytes = o;
+    for (const HostGroup &gr : w.groups) {
+        const kda_fwd_desc gd = group_desc(d, gr);
+        w.fws_bytes = std::max(w.fws_bytes, fwd_workspace_bytes(&gd, w.cu_rel.data() + gr.cu_off));
+    }
+    size_t off = 0;
+    w.cu = off;     off += align256(sizeof(int32_t) * w.cu_rel.size());
+    w.in[0] = off;  off += w.in_bytes;
+    w.in[1] = off;  off += w.in_bytes;
+    w.out[0] = off; off += w.out_bytes;
+    w.out[1] = off; off += w.out_bytes;
+    w.fws = off;    off += align256(w.fws_bytes);
+    w.total = off;
+    return w;
+}
+
+}  // namespace
+
+extern "C" size_t kda_chunk_fwd_host_workspace_size(const kda_fwd_desc *desc, const int32_t *cu_seqlens_host,
+                                                    int32_t with_gate, int32_t with_S0, int32_t with_S_T) {
+    if (validate_fwd_desc(desc) != KDA_OK || !cu_seqlens_host) return SIZE_MAX;
+    if (validate_host_seqlens(desc, cu_seqlens_host) != KDA_OK) return SIZE_MAX;
+    return host_layout(*desc, cu_seqlens_host, with_gate != 0, with_S0 != 0, with_S_T != 0).total;
+}
+
+extern "C" kda_status kda_chunk_fwd_host(const kda_fwd_desc *desc, const void *q, const void *k,
+                                         const void *v, const void *g, const void *beta, const float *S0,
+                                         const int32_t *cu_seqlens_host, const void *gate, void *o,
+                                         float *S_T, void *workspace, size_t workspace_bytes,
+                                         cudaStream_t stream) {
+    kda_status st = validate_fwd_desc(desc);
+    if (st != KDA_OK) return st;
+    const kda_fwd_desc &d = *desc;
+    if (!cu_seqlens_host) return KDA_ERR_INVALID_ARG;
+    if ((st = validate_host_seqlens(desc, cu_seqlens_host)) != KDA_OK) return st;
+    if (d.total_tokens > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
+    const HostLayout w = host_layout(d, cu_seqlens_host, gate != nullptr, S0 != nullptr, S_T != nullptr);
+    if (!workspace || workspace_bytes < w.total || reinterpret_cast<uintptr_t>(workspace) % 256 != 0)
+        return KDA_ERR_WORKSPACE;
+
+    std::lock_guard<std::mutex> lock(g_pipe_mutex);
+    HostPipe *pp = nullptr;
+    if (host_pipe(&pp) != cudaSuccess) return KDA_ERR_CUDA;
+    HostPipe &P = *pp;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    const size_t esz = d.io_dtype == KDA_BF16 ? 2 : 4, H = (size_t)d.num_heads;
+    const size_t rk = H * d.dk * esz, rv = H * d.dv * esz, rb = H * esz;      // bytes per token row
+    const size_t rs = H * (size_t)d.dk * d.dv * sizeof(float);               // bytes per sequence state
+    int32_t *cu_dev = reinterpret_cast<int32_t *>(ws + w.cu);
+    auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+    auto cp = [](void *dst, const void *src, size_t n, cudaMemcpyKind kind, cudaStream_t s) {
+        return n == 0 ? cudaSuccess : cudaMemcpyAsync(dst, src, n, kind, s);
+    };
+    // every group's relative cu_seqlens, then the copy streams join the caller's stream
+    if (!ok(cudaMemcpyAsync(cu_dev, w.cu_rel.data(), w.cu_rel.size() * sizeof(int32_t), cudaMemcpyHostToDevice,
+                            stream)) ||
+        !ok(cudaEventRecord(P.entry, stream)) || !ok(cudaStreamWaitEvent(P.h2d, P.entry, 0)) ||
+        !ok(cudaStreamWaitEvent(P.d2h, P.entry, 0)))
+        return KDA_ERR_CUDA;
+    const char *cq = static_cast<const char *>(q), *ck = static_cast<const char *>(k);
+    const char *cg = static_cast<const char *>(g), *cv = static_cast<const char *>(v);
+    const char *cb = static_cast<const char *>(beta), *cz = static_cast<const char *>(gate);
+    const char *cs0 = reinterpret_cast<const char *>(S0);
+    char *co = static_cast<char *>(o), *cst = reinterpret_cast<char *>(S_T);
+    const int G = (int)w.groups.size();
+    for (int i = 0; i < G; ++i) {
+        const HostGroup &gr = w.groups[i];
+        const int sl = i & 1;
+        unsigned char *in = ws + w.in[sl], *out = ws + w.out[sl];
+        const size_t nt = (size_t)(gr.t1 - gr.t0), ns = (size_t)(gr.s1 - gr.s0);
+        const size_t t0 = (size_t)gr.t0, s0 = (size_t)gr.s0;
+        // inputs of group i, once the prefill of group i-2 has consumed the slot
+        if (i >= 2 && !ok(cudaStreamWaitEvent(P.h2d, P.computed[sl], 0))) return KDA_ERR_CUDA;
+        if (!ok(cp(in + w.off_q, cq + t0 * rk, nt * rk, cudaMemcpyHostToDevice, P.h2d)) ||
+            !ok(cp(in + w.off_k, ck + t0 * rk, nt * rk, cudaMemcpyHostToDevice, P.h2d)) ||
+            !ok(cp(in + w.off_g, cg + t0 * rk, nt * rk, cudaMemcpyHostToDevice, P.h2d)) ||
+            !ok(cp(in + w.off_v, cv + t0 * rv, nt * rv, cudaMemcpyHostToDevice, P.h2d)) ||
+            !ok(cp(in + w.off_b, cb + t0 * rb, nt * rb, cudaMemcpyHostToDevice, P.h2d)) ||
+            (gate && !ok(cp(in + w.off_z, cz + t0 * rv, nt * rv, cudaMemcpyHostToDevice, P.h2d))) ||
+            (S0 && !ok(cp(in + w.off_s0, cs0 + s0 * rs, ns * rs, cudaMemcpyHostToDevice, P.h2d))) ||
+            !ok(cudaEventRecord(P.in_ready[sl], P.h2d)))
+            return KDA_ERR_CUDA;
+        // the prefill of group i, once its inputs are in and group i-2's outputs are out
+        if (!ok(cudaStreamWaitEvent(stream, P.in_ready[sl], 0)) ||
+            (i >= 2 && !ok(cudaStreamWaitEvent(stream, P.out_free[sl], 0))))
+            return KDA_ERR_CUDA;
+        const kda_fwd_desc gd = group_desc(d, gr);
+        st = chunk_fwd_impl(&gd, nullptr, in + w.off_q, in + w.off_k, in + w.off_v, in + w.off_g, in + w.off_b,
+                            S0 ? reinterpret_cast<const float *>(in + w.off_s0) : nullptr, cu_dev + gr.cu_off,
+                            w.cu_rel.data() + gr.cu_off, gate ? in + w.off_z : nullptr, out + w.off_o,
+                            S_T ? reinterpret_cast<float *>(out + w.off_st) : nullptr, ws + w.fws, w.fws_bytes,
+                            stream);
+        if (st != KDA_OK) return st;
+        if (!ok(cudaEventRecord(P.computed[sl], stream))) return KDA_ERR_CUDA;
+        // the outputs of group i
+        if (!ok(cudaStreamWaitEvent(P.d2h, P.computed[sl], 0)) ||
+            !ok(cp(co + t0 * rv, out + w.off_o, nt * rv, cudaMemcpyDeviceToHost, P.d2h)) ||
+            (S_T && !ok(cp(cst + s0 * rs, out + w.off_st, ns * rs, cudaMemcpyDeviceToHost, P.d2h))) ||
+            !ok(cudaEventRecord(P.out_free[sl], P.d2h)))
+            return KDA_ERR_CUDA;
+    }
+    // the caller's stream covers the last copies (the copy streams are in order)
+    if (G > 0 && !ok(cudaStreamWaitEvent(stream, P.out_free[(G - 1) & 1], 0))) return KDA_ERR_CUDA;
+    return KDA_OK;
+}

@@ -29,7 +29,8 @@ EXPORTED_SYMBOLS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode
                     "kda_chunk_fwd_noalloc", "kda_selftest_bounded_wait",
                     "kda_chunk_fwd_snapshots", "kda_spec_verify", "kda_spec_commit",
                     "kda_segment_summary_workspace_size", "kda_segment_summary",
-                    "kda_state_combine", "kda_chunk_bwd_workspace_size", "kda_chunk_bwd")
+                    "kda_state_combine", "kda_chunk_bwd_workspace_size", "kda_chunk_bwd",
+                    "kda_chunk_fwd_host_workspace_size", "kda_chunk_fwd_host")
 NOALLOC_MAX_SEQS = 65536   # KDA_NOALLOC_MAX_SEQS in include/kda.h
 
 
@@ -124,6 +125,12 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.kda_chunk_bwd.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, vp, vp, vp, i32p, i32p, vp,
                                       vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         lib.kda_chunk_bwd.restype = ctypes.c_int
+        lib.kda_chunk_fwd_host_workspace_size.argtypes = [ctypes.POINTER(FwdDesc), i32p, ctypes.c_int32,
+                                                          ctypes.c_int32, ctypes.c_int32]
+        lib.kda_chunk_fwd_host_workspace_size.restype = sz
+        lib.kda_chunk_fwd_host.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, vp, vp, vp, i32p, vp, vp,
+                                           vp, vp, sz, vp]
+        lib.kda_chunk_fwd_host.restype = ctypes.c_int
         lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_int32, vp]
         lib.kda_selftest_bounded_wait.restype = ctypes.c_int
         _lib = lib
@@ -442,6 +449,58 @@ def state_combine(summaries, out=None):
     if st != KDA_OK:
         raise KDAError(st, "kda_state_combine")
     return S_in
+
+
+def chunk_fwd_host(q, k, v, g, beta, cu_seqlens_host, S0=None, gate=None, scale=None,
+                   g_floor: float = -5.0, out=None, final_state_out=None, output_final_state=True,
+                   device=None, workspace=None):
+    """``kda_chunk_fwd_host``: the prefill of :func:`chunk_fwd` with inputs
+    and outputs in host memory (CPU tensors, page-locked for the copies to
+    overlap the compute), pipelined over groups of sequences.  Returns
+    ``(o, S_T)`` as CPU tensors once the call's stream has been synchronised."""
+    if not torch.cuda.is_available():
+        raise RuntimeError("the KDA library needs a CUDA GPU (sm_100a); none is available")
+    lib = load_library()
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    cu_host = [int(x) for x in cu_seqlens_host]
+    N = len(cu_host) - 1
+    cpu = torch.device("cpu")
+    for name, t, shape in (("q", q, (T, H, dk)), ("k", k, (T, H, dk)), ("g", g, (T, H, dk)),
+                           ("v", v, (T, H, dv)), ("beta", beta, (T, H))):
+        if t.device != cpu or t.dtype != q.dtype or tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CPU tensor of shape {shape} and dtype {q.dtype}")
+    if gate is not None and (gate.device != cpu or tuple(gate.shape) != (T, H, dv) or not gate.is_contiguous()):
+        raise ValueError("gate must be a contiguous CPU tensor of v's shape")
+    if S0 is not None and (S0.device != cpu or S0.dtype != torch.float32 or tuple(S0.shape) != (N, H, dk, dv)
+                           or not S0.is_contiguous()):
+        raise ValueError("S0 must be a contiguous fp32 CPU tensor [N,H,dk,dv]")
+    o = out if out is not None else torch.empty((T, H, dv), dtype=q.dtype, pin_memory=True)
+    S_T = None
+    if output_final_state:
+        S_T = (final_state_out if final_state_out is not None
+               else torch.empty((N, H, dk, dv), dtype=torch.float32, pin_memory=True))
+    desc = FwdDesc(total_tokens=T, num_seqs=N, num_heads=H, dk=dk, dv=dv, io_dtype=_io_dtype(q),
+                   scale=float(dk ** -0.5 if scale is None else scale), g_floor=float(g_floor),
+                   chunk=0, max_seqlen=0)
+    cu_h = (ctypes.c_int32 * (N + 1))(*cu_host)
+    ws_bytes = lib.kda_chunk_fwd_host_workspace_size(ctypes.byref(desc), cu_h, int(gate is not None),
+                                                     int(S0 is not None), int(S_T is not None))
+    if ws_bytes == ctypes.c_size_t(-1).value:
+        raise KDAError(1, "kda_chunk_fwd_host_workspace_size")
+    ws = workspace
+    if ws is None or ws.numel() < ws_bytes:
+        ws = torch.empty(max(int(ws_bytes), 256), dtype=torch.uint8, device=device)
+    with torch.cuda.device(device):
+        stream = torch.cuda.current_stream(device)
+        st = lib.kda_chunk_fwd_host(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                    _ptr(S0), cu_h, _ptr(gate), _ptr(o), _ptr(S_T), _ptr(ws), ws.numel(),
+                                    ctypes.c_void_p(stream.cuda_stream))
+        if st != KDA_OK:
+            raise KDAError(st, "kda_chunk_fwd_host")
+        stream.synchronize()
+    return o, S_T
 
 
 def chunk_bwd(q, k, v, g, beta, dout, cu_seqlens=None, cu_seqlens_host=None, S0=None, gate=None,

@@ -268,6 +268,29 @@ kda_status kda_chunk_fwd_snapshots(const kda_fwd_desc *desc, const kda_snapshots
                                    cudaStream_t stream);
 
 /*
+ * kda_chunk_fwd from and to HOST memory: q, k, v, g, beta, gate, S0 (inputs)
+ * and o, S_T (outputs) are host pointers in the layouts of kda_chunk_fwd;
+ * cu_seqlens_host (host) is required.  The batch is cut into up to 8 groups
+ * of whole sequences and pipelined over three streams: the host-to-device
+ * copy of group i+1 and the device-to-host copy of group i-1 overlap the
+ * prefill of group i on `stream`.  Host buffers should be page-locked
+ * (cudaHostAlloc / cudaHostRegister) for the copies to overlap; pageable
+ * ones work but serialise.  The device workspace (256-byte aligned) holds two
+ * input and two output slots and the prefill's own workspace:
+ * kda_chunk_fwd_host_workspace_size(desc, cu_seqlens_host, with_gate,
+ * with_S0, with_S_T) bytes.  When the call returns the work is enqueued;
+ * synchronising `stream` waits for every copy.  Calls on one device are
+ * serialised while they enqueue (they share two copy streams).  Errors as
+ * kda_chunk_fwd; KDA_ERR_WORKSPACE for a short or misaligned workspace.
+ */
+size_t kda_chunk_fwd_host_workspace_size(const kda_fwd_desc *desc, const int32_t *cu_seqlens_host,
+                                         int32_t with_gate, int32_t with_S0, int32_t with_S_T);
+kda_status kda_chunk_fwd_host(const kda_fwd_desc *desc, const void *q, const void *k, const void *v,
+                              const void *g, const void *beta, const float *S0,
+                              const int32_t *cu_seqlens_host, const void *gate, void *o, float *S_T,
+                              void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Backward of the prefill (training; the report digest's FlashKDA serves
  * training and prefill, section 基础设施): the gradients of
  * L = sum(o * dout) + sum(S_T * dS_T) through the recurrence of

@@ -274,3 +274,25 @@ def test_chunk_bwd_validation(lib):
     assert bwd(ws=None) == 3
     assert bwd(ws_bytes=need - 256) == 3
     assert bwd(ws=A + 8 * MB) == 1                          # workspace on v
+
+
+def test_chunk_fwd_host_validation(lib):
+    """Rejected on the host before any copy or launch (fake pointers never touched)."""
+    d = _desc(num_seqs=2, total_tokens=10)
+    cu_host = (ctypes.c_int32 * 3)(0, 4, 10)
+    assert lib.kda_chunk_fwd_host_workspace_size(ctypes.byref(_desc(num_heads=0)), cu_host, 0, 0, 1) == SIZE_MAX
+    assert lib.kda_chunk_fwd_host_workspace_size(ctypes.byref(d), None, 0, 0, 1) == SIZE_MAX
+    full = lib.kda_chunk_fwd_host_workspace_size(ctypes.byref(d), cu_host, 1, 1, 1)
+    need = lib.kda_chunk_fwd_host_workspace_size(ctypes.byref(d), cu_host, 0, 0, 0)   # as called below
+    assert need != SIZE_MAX and need % 256 == 0 and full > need
+
+    def host(desc=d, cu_h=cu_host, ws=A + 256 * MB, ws_bytes=need, o=A + 24 * MB):
+        return lib.kda_chunk_fwd_host(ctypes.byref(desc), A, A + 4 * MB, A + 8 * MB, A + 12 * MB, A + 16 * MB,
+                                      None, cu_h, None, o, None, ws, ws_bytes, None)
+    assert host(cu_h=None) == 1
+    assert host(cu_h=(ctypes.c_int32 * 3)(0, 4, 9)) == 1          # disagrees with total_tokens
+    assert host(o=None) == 1
+    assert host(desc=_desc(num_seqs=2, total_tokens=10, io_dtype=5)) == 1
+    assert host(ws=None) == 3
+    assert host(ws_bytes=need - 256) == 3
+    assert host(ws=A + 256 * MB + 64) == 3                           # not 256-byte aligned

@@ -101,3 +101,24 @@ def test_long_draft_without_gate(D, dk, dv, dtype):
         assert rel_max_beyond_bf16(o.view(B * D, H, dv), o_ref) <= TOL_BF16
         assert rel_max(S, S_ref) <= TOL_BF16
     assert device_status() == 0
+
+
+def test_full_size_sampled():
+    """The bench's launch: 512 sequences x 64 heads, 4 draft tokens verified,
+    3 committed; sampled (sequence, head) pairs against the oracle."""
+    B, D, H, d = 512, 4, 64, 128
+    inp, x, S = _draft(B, D, H, d, torch.bfloat16, seed=59)
+    S_before = S.clone()
+    o = spec_verify(x["q"], x["k"], x["v"], x["g"], x["beta"], S, gate=x["gate"])
+    spec_commit(x["q"], x["k"], x["v"], x["g"], x["beta"], S,
+                torch.full((B,), 3, dtype=torch.int32, device="cuda"))
+    assert device_status() == 0
+    for b, h in ((0, 0), (137, 21), (511, 63), (300, 5)):
+        sl = slice(b * D, (b + 1) * D)
+        cut = lambda t, n=None: _cpu(t[sl, h:h + 1]) if n is None else _cpu(t[sl][:n, h:h + 1])
+        o_ref, _ = oracle.kda_fwd_ref(*(cut(inp[n]) for n in ("q", "k", "v", "g", "beta")),
+                                      S0=_cpu(S_before[b:b + 1, h:h + 1]), gate=cut(inp["gate"]))
+        assert rel_max_beyond_bf16(o[b, :, h:h + 1], o_ref) <= TOL_BF16
+        _, S_ref = oracle.kda_fwd_ref(*(cut(inp[n], 3) for n in ("q", "k", "v", "g", "beta")),
+                                      S0=_cpu(S_before[b:b + 1, h:h + 1]))
+        assert rel_max(S[b:b + 1, h:h + 1], S_ref) <= TOL_BF16
