@@ -65,6 +65,9 @@ PROFILED_TRAFFIC = {
     "csrc/kda_spec.cuh": {"sha1": "5f78f5eaf7b5",
                           "bytes_per_head_round": (579.116800e6 + 4.305920e6 + 555.884544e6 + 477.843968e6) / 8192,
                           "profile": "profiles/spec_kernel_verify_commit_128x64.md"},
+    # backward kernel at 2 x 1024 x 16 (bf16): per token-head (the forward with snapshots not included)
+    "csrc/kda_bwd.cuh": {"sha1": "efb7c2732829", "bytes_per_token_head": (74.357504e6 + 29.543424e6) / 32768,
+                         "profile": "profiles/bwd_kernel_2x1024x16.md"},
 }
 
 
@@ -578,6 +581,8 @@ def main():
             others[f"backward B={B} T={T} H={H} (gradients of sum(o * dout), bf16)"] = {
                 "tokens": B * T, "ms": ms, "tokens_per_s": world * B * T / (ms / 1e3),
                 "alg_gbs": byts / (ms / 1e3) / 1e9, "roofline_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                "alg_bytes": byts,
+                "traffic_bwd_kernel": profiled_traffic("csrc/kda_bwd.cuh", "bytes_per_token_head", B * T * H),
                 "note": "forward with 64-token state snapshots, then per (sequence, head) a CUDA-core "
                         "replay of each chunk and the reverse recurrence"}
             del xb, dout
