@@ -588,6 +588,38 @@ def main():
             del xb, dout
             torch.cuda.empty_cache()
 
+        if "kcp" in extras:
+            # one rank's KCP summary: a 2^20 / 8-token piece, H=32, state from zero and
+            # transition product (a middle rank of eight), on this GPU alone
+            from gated_delta_rule_136_b200 import segment_summary
+            Lp, Hp = (1 << 20) // 8, 32
+            wp = inputs.prefill_inputs([Lp], H=Hp, dk=DK, dv=DV, device=dev, seed=300 + rank,
+                                       g_mode="floor_stress")
+            runs = lambda: segment_summary(wp["q"], wp["k"], wp["v"], wp["g"], wp["beta"], wp["cu_seqlens"],
+                                           wp["cu_seqlens_host"], with_M=True)
+            for _ in range(2):
+                runs()
+            barrier()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 3
+            tw0 = time.time()
+            a.record(stream)
+            for _ in range(reps):
+                runs()
+            b.record(stream)
+            barrier()
+            if sampler:
+                sampler.mark(tw0, time.time())
+            if device_status(dev) != 0:
+                raise RuntimeError("device error word after the piece summary")
+            ms = max_over_ranks(a.elapsed_time(b)) / reps
+            others[f"KCP piece summary: {Lp} tokens x H={Hp} (S_loc and M), one rank"] = {
+                "tokens": Lp, "ms": ms, "tokens_per_s": world * Lp / (ms / 1e3),
+                "note": "two chains per (piece, head), cut into sub-segments folded by the scan kernel "
+                        "when the chains are fewer than the SMs"}
+            del wp
+            torch.cuda.empty_cache()
+
         if world > 1 and "kcp" in extras:
             # context-parallel prefill (KCP): one 2^20-token sequence, H=32, cut into one
             # piece per rank; the piece summaries cross ranks in one NCCL all-gather

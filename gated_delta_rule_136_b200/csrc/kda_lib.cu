@@ -89,8 +89,8 @@ kda_status validate_host_seqlens(const kda_fwd_desc *d, const int32_t *cu) {
 // ---------------------------------------------------------------- long-sequence split
 // When there are fewer (sequence, head) units than SMs, long sequences are cut
 // into segments so that the tensor-core prefill still fills the GPU (needs
-// cu_seqlens_host).  KDA_SEGMENTS=<P> forces P segments per sequence (tuning
-// and tests).
+// cu_seqlens_host).  KDA_SEGMENTS=<P> forces P segments per sequence, and
+// KDA_SEGMENTS=1 disables the split (tuning and tests).
 constexpr int64_t kMinSegTokens = 1024;
 
 int device_sm_count() {
@@ -133,7 +133,7 @@ SegPlan plan_segments(const kda_fwd_desc &d, const int32_t *cu) {
     // U P units, each of ceil(C / P) chunks.  Take the best P, and split only
     // if it saves at least 10 %.
     int64_t best_p = 1;
-    if (forced <= 1 && units < sms) {
+    if (forced < 1 && units < sms) {          // KDA_SEGMENTS=1: no split
         int64_t cmax = 0;
         for (int32_t n = 0; n < N; ++n) cmax = std::max<int64_t>(cmax, ((int64_t)cu[n + 1] - cu[n] + 63) / 64);
         auto waves = [&](int64_t x) { return (x + sms - 1) / sms; };
@@ -316,7 +316,7 @@ cudaError_t launch_split(const kda_fwd_desc &d, const SegPlan &pl, const int32_t
     std::vector<kda::ScanJob> jobs;
     p1.reserve((size_t)pl.pass1_units);
     p2.reserve((size_t)pl.pass2_units);
-    size_t blk = 0;   // next (sequence, head) matrix block, each P x 3 x D^2 floats
+    size_t mat_off = 0;   // floats used so far: each split (sequence, head) takes P x 3 x D^2, P per sequence
     for (int32_t n = 0; n < N; ++n) {
         const int64_t t0 = cu[n], t1 = cu[n + 1];
         const int32_t P = pl.nseg[n];
@@ -328,8 +328,8 @@ cudaError_t launch_split(const kda_fwd_desc &d, const SegPlan &pl, const int32_t
                 p2.push_back(TcUnit{t0, t1, s0, st, h, kda::tck::UNIT_STORE_O, n, t0});
                 continue;
             }
-            float *base = mats + blk * (size_t)P * 3u * DD;
-            ++blk;
+            float *base = mats + mat_off;
+            mat_off += (size_t)P * 3u * DD;
             auto Sloc = [&](int32_t sp) { return base + ((size_t)sp * 3u + 0u) * DD; };
             auto Mp = [&](int32_t sp) { return base + ((size_t)sp * 3u + 1u) * DD; };
             auto Sin = [&](int32_t sp) { return base + ((size_t)sp * 3u + 2u) * DD; };
@@ -343,7 +343,7 @@ cudaError_t launch_split(const kda_fwd_desc &d, const SegPlan &pl, const int32_t
                 p2.push_back(TcUnit{a, b, sp == 0 ? s0 : Sin(sp), sp + 1 == P ? st : nullptr, h,
                                     kda::tck::UNIT_STORE_O, n, t0});
             }
-            jobs.push_back(kda::ScanJob{Sloc(0), Mp(0), Sin(0), (int64_t)(3u * DD), P, nullptr});
+            jobs.push_back(kda::ScanJob{Sloc(0), Mp(0), Sin(0), (int64_t)(3u * DD), P, nullptr, 0});
         }
     }
     auto longest_first = [](const TcUnit &x, const TcUnit &y) {
@@ -714,9 +714,81 @@ kda_status kda_chunk_bwd(const kda_fwd_desc *desc, const void *q, const void *k,
 }
 
 // ---------------------------------------------------------------- context parallel (KCP)
-size_t kda_segment_summary_workspace_size(const kda_fwd_desc *desc) {
-    if (validate_fwd_desc(desc) != KDA_OK) return SIZE_MAX;
-    return align256(2u * sizeof(kda::tck::TcUnit) * (size_t)desc->num_seqs * (size_t)desc->num_heads);
+namespace {
+// Sub-segments per piece for the summary: the chains (S_loc, and M where
+// asked) of every (sequence, head) are cut like the prefill's long-sequence
+// split when they are fewer than the SMs, then folded by the scan kernel.
+struct SummaryPlan {
+    std::vector<int32_t> nseg;      // sub-segments per sequence
+    std::vector<int64_t> seglen;    // tokens per sub-segment (multiple of 64)
+    int64_t mat_blocks = 0;         // (sequence, head, sub-segment) entries of the split buffers
+    int64_t jobs = 0, units = 0;
+};
+
+SummaryPlan plan_summary(const kda_fwd_desc &d, const int32_t *cu, bool with_M) {
+    SummaryPlan pl;
+    const int32_t N = d.num_seqs, H = d.num_heads;
+    pl.nseg.assign(N, 1);
+    pl.seglen.assign(N, 0);
+    const int64_t chains = (int64_t)N * H * (with_M ? 2 : 1);
+    const char *env = std::getenv("KDA_SEGMENTS");
+    const int forced = env ? std::atoi(env) : 0;
+    const int sms = device_sm_count();
+    int64_t best_p = 1;
+    if (forced < 1 && chains < sms) {         // KDA_SEGMENTS=1: no split
+        int64_t cmax = 0;
+        for (int32_t n = 0; n < N; ++n) cmax = std::max<int64_t>(cmax, ((int64_t)cu[n + 1] - cu[n] + 63) / 64);
+        auto waves = [&](int64_t x) { return (x + sms - 1) / sms; };
+        const int64_t t1 = waves(chains) * cmax;
+        int64_t best_t = t1;
+        for (int64_t P = 2; P <= 64 && P * kMinSegTokens / 64 <= cmax; ++P) {
+            // every sub-segment needs both chains (M for the fold), plus the folds
+            const int64_t t = waves((int64_t)N * H * 2 * P) * ((cmax + P - 1) / P) + P;
+            if (t < best_t) { best_t = t; best_p = P; }
+        }
+        if (best_t * 10 > t1 * 9) best_p = 1;
+    }
+    for (int32_t n = 0; n < N; ++n) {
+        const int64_t L = (int64_t)cu[n + 1] - cu[n];
+        int64_t P = forced > 1 ? std::min<int64_t>(forced, L / 128)
+                               : (best_p > 1 ? std::min<int64_t>(best_p, L / kMinSegTokens) : 1);
+        if (P >= 2) {
+            const int64_t seg = ((L + P - 1) / P + 63) / 64 * 64;
+            P = (L + seg - 1) / seg;
+        }
+        if (P >= 2) {
+            pl.nseg[n] = (int32_t)P;
+            pl.seglen[n] = ((L + P - 1) / P + 63) / 64 * 64;
+            pl.mat_blocks += (int64_t)H * P;
+            pl.jobs += (int64_t)H * (with_M ? 2 : 1);
+            pl.units += (int64_t)H * 2 * P;
+        } else {
+            pl.units += (int64_t)H * (with_M ? 2 : 1);
+        }
+    }
+    return pl;
+}
+
+struct SummaryLayout {
+    size_t units = 0, jobs = 0, mats = 0, total = 0;
+};
+
+SummaryLayout summary_layout(const SummaryPlan &pl) {
+    SummaryLayout w;
+    size_t off = 0;
+    w.units = off; off += align256(sizeof(kda::tck::TcUnit) * (size_t)std::max<int64_t>(pl.units, 1));
+    w.jobs = off;  off += align256(sizeof(kda::ScanJob) * (size_t)std::max<int64_t>(pl.jobs, 1));
+    w.mats = off;  off += align256((size_t)pl.mat_blocks * 2u * 128u * 128u * sizeof(float));
+    w.total = off;
+    return w;
+}
+}  // namespace
+
+size_t kda_segment_summary_workspace_size(const kda_fwd_desc *desc, const int32_t *cu_seqlens_host,
+                                          int32_t with_M) {
+    if (validate_fwd_desc(desc) != KDA_OK || !cu_seqlens_host) return SIZE_MAX;
+    if (validate_host_seqlens(desc, cu_seqlens_host) != KDA_OK) return SIZE_MAX;
+    return summary_layout(plan_summary(*desc, cu_seqlens_host, with_M != 0)).total;
 }
 
 kda_status kda_segment_summary(const kda_fwd_desc *desc, const void *q, const void *k,
@@ -734,6 +806,8 @@ kda_status kda_segment_summary(const kda_fwd_desc *desc, const void *q, const vo
     if ((st = validate_host_seqlens(desc, cu_seqlens_host)) != KDA_OK) return st;
     for (const void *ptr : {q, k, v, g})      // moved by TMA
         if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return KDA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(S_loc) % 16 != 0 || reinterpret_cast<uintptr_t>(M) % 16 != 0)
+        return KDA_ERR_INVALID_ARG;            // written by the scan kernel as float4
 
     const int32_t N = d.num_seqs, H = d.num_heads;
     const int64_t T = d.total_tokens, DD = 128 * 128;
@@ -745,40 +819,71 @@ kda_status kda_segment_summary(const kda_fwd_desc *desc, const void *q, const vo
     for (const Range &r : ins)
         if (overlaps(rl, r) || overlaps(rm, r)) return KDA_ERR_INVALID_ARG;
     if (overlaps(rl, rm)) return KDA_ERR_INVALID_ARG;
-    const size_t need = kda_segment_summary_workspace_size(desc);
-    if (!workspace || workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256 != 0)
+    const SummaryPlan pl = plan_summary(d, cu_seqlens_host, M != nullptr);
+    const SummaryLayout w = summary_layout(pl);
+    if (!workspace || workspace_bytes < w.total || reinterpret_cast<uintptr_t>(workspace) % 256 != 0)
         return KDA_ERR_WORKSPACE;
-    const Range rw = range_of(workspace, (int64_t)need);
+    const Range rw = range_of(workspace, (int64_t)w.total);
     for (const Range &r : ins)
         if (overlaps(rw, r)) return KDA_ERR_INVALID_ARG;
     if (overlaps(rw, rl) || overlaps(rw, rm)) return KDA_ERR_INVALID_ARG;
 
-    // one chain per (sequence, head) for S_loc, one more for M: the M chain
-    // starts from the identity with v taken as zero
+    // chains: unsplit pieces write S_loc (and M) directly; a split piece runs
+    // both chains per sub-segment into the workspace, and the scan folds them
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    float *mats = reinterpret_cast<float *>(ws + w.mats);
     std::vector<TcUnit> units;
-    units.reserve((size_t)N * H * (M ? 2 : 1));
+    std::vector<kda::ScanJob> jobs;
+    units.reserve((size_t)pl.units);
+    size_t mat_off = 0;   // floats used so far: each split (sequence, head) takes P x 2 x D^2, P per sequence
     for (int32_t n = 0; n < N; ++n) {
+        const int64_t a0 = cu_seqlens_host[n], a1 = cu_seqlens_host[n + 1];
+        const int32_t P = pl.nseg[n];
         for (int32_t h = 0; h < H; ++h) {
             const int64_t u = (int64_t)n * H + h;
-            units.push_back(TcUnit{cu_seqlens_host[n], cu_seqlens_host[n + 1], S0 ? S0 + u * DD : nullptr,
-                                   S_loc + u * DD, h, 0, n, cu_seqlens_host[n]});
-            if (M)
-                units.push_back(TcUnit{cu_seqlens_host[n], cu_seqlens_host[n + 1], nullptr, M + u * DD, h,
-                                       kda::tck::UNIT_ZERO_V | kda::tck::UNIT_S0_IDENTITY, n,
-                                       cu_seqlens_host[n]});
+            const float *s0 = S0 ? S0 + u * DD : nullptr;
+            if (P == 1) {
+                units.push_back(TcUnit{a0, a1, s0, S_loc + u * DD, h, 0, n, a0});
+                if (M)
+                    units.push_back(TcUnit{a0, a1, nullptr, M + u * DD, h,
+                                           kda::tck::UNIT_ZERO_V | kda::tck::UNIT_S0_IDENTITY, n, a0});
+                continue;
+            }
+            float *Lb = mats + mat_off;                        // [P] S_loc, then [P] M
+            float *Mb = Lb + (size_t)P * DD;
+            mat_off += (size_t)P * 2u * DD;
+            for (int32_t sp = 0; sp < P; ++sp) {
+                const int64_t b0 = a0 + (int64_t)sp * pl.seglen[n];
+                const int64_t b1 = std::min<int64_t>(a1, b0 + pl.seglen[n]);
+                units.push_back(TcUnit{b0, b1, sp == 0 ? s0 : nullptr, Lb + sp * DD, h, 0, n, a0});
+                units.push_back(TcUnit{b0, b1, nullptr, Mb + sp * DD, h,
+                                       kda::tck::UNIT_ZERO_V | kda::tck::UNIT_S0_IDENTITY, n, a0});
+            }
+            jobs.push_back(kda::ScanJob{Lb, Mb, nullptr, DD, P + 1, S_loc + u * DD, 0});
+            if (M) jobs.push_back(kda::ScanJob{Mb, Mb, nullptr, DD, P + 1, M + u * DD, 1});
         }
     }
     std::stable_sort(units.begin(), units.end(), [](const TcUnit &x, const TcUnit &y) {
         return (x.t_end - x.t_begin) > (y.t_end - y.t_begin);
     });
-    TcUnit *du = static_cast<TcUnit *>(workspace);
+    TcUnit *du = reinterpret_cast<TcUnit *>(ws + w.units);
     if (cudaMemcpyAsync(du, units.data(), units.size() * sizeof(TcUnit), cudaMemcpyHostToDevice,
                         stream) != cudaSuccess)
         return KDA_ERR_CUDA;
     kda::tck::TcParams tp{beta, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, H, d.scale,
                           d.g_floor, du, kda::SnapOut{nullptr, nullptr, 0, 64}};
-    return launch_tc_units(d, q, k, v, g, tp, (int64_t)units.size(), stream) == cudaSuccess ? KDA_OK
-                                                                                           : KDA_ERR_CUDA;
+    if (launch_tc_units(d, q, k, v, g, tp, (int64_t)units.size(), stream) != cudaSuccess) return KDA_ERR_CUDA;
+    if (jobs.empty()) return KDA_OK;
+    kda::ScanJob *dj = reinterpret_cast<kda::ScanJob *>(ws + w.jobs);
+    if (cudaMemcpyAsync(dj, jobs.data(), jobs.size() * sizeof(kda::ScanJob), cudaMemcpyHostToDevice,
+                        stream) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    const size_t scan_smem = 2u * (size_t)DD * sizeof(float);
+    if (cudaFuncSetAttribute(kda::segment_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)scan_smem) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    kda::segment_scan_kernel<<<(unsigned)jobs.size(), 256, scan_smem, stream>>>(dj);
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 kda_status kda_state_combine(const kda_combine_desc *desc, const float *summaries, float *S_in,

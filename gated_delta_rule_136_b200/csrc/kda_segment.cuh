@@ -25,6 +25,7 @@ struct ScanJob {
     int64_t stride;       // floats between consecutive segments' matrices
     int32_t num_segments;
     float *S_last;        // if not null: S_in(P-1) is also written here
+    int32_t product;      // 1: S_loc is read for segment 0 only, so S_in(P-1) = M_{P-2} ... M_1 S_loc,0
 };
 
 // One CTA (256 threads) per (sequence, head).  dk = dv = 128; thread (v, half)
@@ -52,7 +53,7 @@ __device__ __forceinline__ void scan_one(const ScanJob &job)
         float acc[64];
         const float *Sl = job.S_loc + seg * job.stride;
 #pragma unroll
-        for (int r = 0; r < 64; ++r) acc[r] = Sl[(half * 64 + r) * D + v];
+        for (int r = 0; r < 64; ++r) acc[r] = job.product ? 0.0f : Sl[(half * 64 + r) * D + v];
         for (int c4 = 0; c4 < D; c4 += 4) {
             const float s0 = Ss[(c4 + 0) * D + v], s1 = Ss[(c4 + 1) * D + v];
             const float s2 = Ss[(c4 + 2) * D + v], s3 = Ss[(c4 + 3) * D + v];
@@ -89,7 +90,7 @@ __global__ void __launch_bounds__(256) state_combine_kernel(const float *summari
     constexpr int64_t DD = 128 * 128;
     const int64_t u = blockIdx.x;
     scan_one(ScanJob{summaries + u * DD, summaries + (units + u) * DD, nullptr, 2 * units * DD,
-                     num_summaries + 1, S_in + u * DD});
+                     num_summaries + 1, S_in + u * DD, 0});
 }
 
 }  // namespace kda

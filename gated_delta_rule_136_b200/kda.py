@@ -113,7 +113,7 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.kda_spec_verify.restype = ctypes.c_int
         lib.kda_spec_commit.argtypes = [ctypes.POINTER(SpecDesc), vp, vp, vp, vp, vp, vp, vp, vp]
         lib.kda_spec_commit.restype = ctypes.c_int
-        lib.kda_segment_summary_workspace_size.argtypes = [ctypes.POINTER(FwdDesc)]
+        lib.kda_segment_summary_workspace_size.argtypes = [ctypes.POINTER(FwdDesc), i32p, ctypes.c_int32]
         lib.kda_segment_summary_workspace_size.restype = sz
         lib.kda_segment_summary.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, vp, vp, vp, i32p,
                                             i32p, vp, vp, vp, sz, vp]
@@ -411,14 +411,14 @@ def segment_summary(q, k, v, g, beta, cu_seqlens, cu_seqlens_host, S0=None, with
     desc = FwdDesc(total_tokens=T, num_seqs=N, num_heads=H, dk=dk, dv=dv, io_dtype=_io_dtype(q),
                    scale=float(dk ** -0.5 if scale is None else scale), g_floor=float(g_floor),
                    chunk=0, max_seqlen=0)
-    ws_bytes = lib.kda_segment_summary_workspace_size(ctypes.byref(desc))
+    cu_h = (ctypes.c_int32 * (N + 1))(*cu_host)
+    ws_bytes = lib.kda_segment_summary_workspace_size(ctypes.byref(desc), cu_h, int(with_M))
     if ws_bytes == ctypes.c_size_t(-1).value:
         raise KDAError(1, "kda_segment_summary_workspace_size")
     ws = torch.empty(max(int(ws_bytes), 256), dtype=torch.uint8, device=device)
     summ = torch.empty((2, N, H, dk, dv), dtype=torch.float32, device=device)
     if not with_M:
         summ[1].zero_()
-    cu_h = (ctypes.c_int32 * (N + 1))(*cu_host)
     with torch.cuda.device(device):
         st = lib.kda_segment_summary(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
                                      _ptr(S0), ctypes.cast(_ptr(cu_seqlens), ctypes.POINTER(ctypes.c_int32)),

@@ -340,14 +340,18 @@ kda_status kda_chunk_bwd(const kda_fwd_desc *desc, const void *q, const void *k,
  *   M     [num_seqs][num_heads][dk][dk] fp32, device: the transition product,
  *         or NULL to skip it (the first piece of a sequence needs none).
  * cu_seqlens_host (num_seqs + 1 int32, host) is required: the work list is
- * built on the host.  The workspace (device, 256-byte aligned) must hold
- * kda_segment_summary_workspace_size(desc) bytes.  Covers bf16 I/O with
- * dk = dv = 128 (the tensor-core kernel), else KDA_ERR_UNSUPPORTED.
+ * built on the host.  When the chains are fewer than the SMs, long pieces are
+ * cut into sub-segments whose summaries the scan kernel folds (the same
+ * decomposition one level down).  The workspace (device, 256-byte aligned)
+ * must hold kda_segment_summary_workspace_size(desc, cu_seqlens_host,
+ * M != NULL) bytes.  S_loc and M must be 16-byte aligned.  Covers bf16 I/O
+ * with dk = dv = 128 (the tensor-core kernel), else KDA_ERR_UNSUPPORTED.
  * KDA_ERR_INVALID_ARG for a bad descriptor, null or overlapping buffers or
  * bad host seqlens; KDA_ERR_WORKSPACE for a short workspace.  Asynchronous on
  * `stream`.
  */
-size_t kda_segment_summary_workspace_size(const kda_fwd_desc *desc);
+size_t kda_segment_summary_workspace_size(const kda_fwd_desc *desc, const int32_t *cu_seqlens_host,
+                                          int32_t with_M);
 kda_status kda_segment_summary(const kda_fwd_desc *desc, const void *q, const void *k,
                                const void *v, const void *g, const void *beta, const float *S0,
                                const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,

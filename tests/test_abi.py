@@ -212,8 +212,10 @@ def _summary(lib, desc, S_loc=A + 40 * MB, M=A + 48 * MB, S0=None, cu_host=None,
 def test_segment_summary_validation(lib):
     """Rejected on the host before any launch (fake pointers never touched)."""
     d = _desc()
-    assert lib.kda_segment_summary_workspace_size(ctypes.byref(_desc(num_heads=0))) == SIZE_MAX
-    assert lib.kda_segment_summary_workspace_size(ctypes.byref(d)) % 256 == 0
+    cu1 = (ctypes.c_int32 * 2)(0, 64)
+    assert lib.kda_segment_summary_workspace_size(ctypes.byref(_desc(num_heads=0)), cu1, 1) == SIZE_MAX
+    assert lib.kda_segment_summary_workspace_size(ctypes.byref(d), None, 1) == SIZE_MAX
+    assert lib.kda_segment_summary_workspace_size(ctypes.byref(d), cu1, 1) % 256 == 0
     assert _summary(lib, _desc(io_dtype=kda.KDA_FP32)) == 2          # tensor-core shape only
     assert _summary(lib, _desc(dk=64)) == 2
     assert _summary(lib, _desc(chunk=16)) == 2

@@ -112,3 +112,41 @@ def test_single_rank_is_plain_prefill():
     o2, S2 = chunk_fwd(*args, S0=inp["S0"], cu_seqlens=inp["cu_seqlens"],
                        cu_seqlens_host=inp["cu_seqlens_host"])
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+def _summary_with_segments(inp, S0, segments):
+    import os
+    old = os.environ.get("KDA_SEGMENTS")
+    try:
+        if segments is None:
+            os.environ.pop("KDA_SEGMENTS", None)
+        else:
+            os.environ["KDA_SEGMENTS"] = str(segments)
+        return segment_summary(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["cu_seqlens"],
+                               inp["cu_seqlens_host"], S0=S0)
+    finally:
+        if old is None:
+            os.environ.pop("KDA_SEGMENTS", None)
+        else:
+            os.environ["KDA_SEGMENTS"] = old
+
+
+@pytest.mark.parametrize("lengths,segments", [([1000, 300], 3), ([300, 1000], 3), ([8192], None)])
+def test_split_summary_matches_oracle_and_unsplit(lengths, segments):
+    """Pieces cut into sub-segments (forced, or chosen because the chains are
+    fewer than the SMs) and folded by the scan: S_loc and M as the oracle's
+    and as the one-chain summary's."""
+    inp = inputs.prefill_inputs(lengths, H=2, dk=128, dv=128, device="cuda", seed=67, s0_std=0.05,
+                                g_mode="floor_stress")
+    split = _summary_with_segments(inp, inp["S0"], segments)
+    whole = _summary_with_segments(inp, inp["S0"], 1)
+    cu = np.array(inp["cu_seqlens_host"])
+    q, k, v, g, beta = (_cpu(inp[n]) for n in ("q", "k", "v", "g", "beta"))
+    _, S_loc = oracle.kda_fwd_ref(q, k, v, g, beta, cu_seqlens=cu, S0=_cpu(inp["S0"]))
+    eye = np.broadcast_to(np.eye(128), (len(lengths), 2, 128, 128)).copy()
+    _, M = oracle.kda_fwd_ref(q, k, torch.zeros_like(v), g, beta, cu_seqlens=cu, S0=eye)
+    for got in (split, whole):
+        assert rel_max(got[0], S_loc) <= TOL_BF16
+        assert rel_max(got[1], M) <= TOL_BF16
+    assert rel_max(split[0], whole[0].cpu()) <= TOL_BF16 and rel_max(split[1], whole[1].cpu()) <= TOL_BF16
+    assert device_status() == 0

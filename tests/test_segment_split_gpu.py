@@ -80,6 +80,17 @@ def test_varlen_only_long_sequences_split():
     assert torch.equal(S_s[3], inp["S0"][3])
 
 
+def test_split_with_different_segment_counts():
+    """Sequences cut into different numbers of segments (2 for 300 tokens, 3
+    for 1300 under a forced 3), the smaller count first: each (sequence,
+    head) takes its own P segments of the split buffers."""
+    inp = inputs.prefill_inputs([300, 1300], H=3, dk=128, dv=128, device="cuda", seed=49, s0_std=0.05)
+    o_s, S_s = _run(inp, segments=3)
+    o_ref, S_ref = _oracle(inp)
+    assert rel_max_beyond_bf16(o_s, o_ref) <= TOL_BF16 and rel_max(S_s, S_ref) <= TOL_BF16
+    assert device_status() == 0
+
+
 def test_long_sequence_default_policy_floor_stress():
     """1 sequence x 32 heads x 65536 tokens, decay near the floor: fewer units
     than SMs, so the default policy splits; two heads checked in full."""
