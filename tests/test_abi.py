@@ -298,3 +298,39 @@ def test_chunk_fwd_host_validation(lib):
     assert host(ws=None) == 3
     assert host(ws_bytes=need - 256) == 3
     assert host(ws=A + 256 * MB + 64) == 3                           # not 256-byte aligned
+
+
+def _in_subprocess_env(env, code):
+    """Run `code` (prints one integer) with extra environment variables: the
+    planners read KDA_SEGMENTS when they run, so each case gets a fresh process."""
+    import subprocess
+    import sys
+    out = subprocess.run([sys.executable, "-c", code], env={**os.environ, **env}, capture_output=True,
+                         text=True, check=True, cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    return int(out.stdout.strip().splitlines()[-1])
+
+
+_SUMMARY_WS = """
+import ctypes
+from gated_delta_rule_136_b200 import kda
+lib = kda.load_library()
+lengths = {lengths}
+cu = [0]
+for L in lengths: cu.append(cu[-1] + L)
+d = kda.FwdDesc(total_tokens=cu[-1], num_seqs=len(lengths), num_heads={H}, dk=128, dv=128, io_dtype=kda.KDA_BF16,
+                scale=0.088, g_floor=-5.0, chunk=0, max_seqlen=0)
+print(lib.kda_segment_summary_workspace_size(ctypes.byref(d), (ctypes.c_int32 * len(cu))(*cu), 1))
+"""
+
+
+def test_summary_split_plan_sizes():
+    """Host planning of the piece summary (no GPU: 148 SMs assumed).  A long
+    piece with few heads is split (its sub-segment matrices need workspace);
+    KDA_SEGMENTS=1 keeps one chain; forced counts that differ per sequence
+    are sized by their sum."""
+    DD = 128 * 128 * 4
+    auto = _in_subprocess_env({}, _SUMMARY_WS.format(lengths=[131072], H=32))
+    whole = _in_subprocess_env({"KDA_SEGMENTS": "1"}, _SUMMARY_WS.format(lengths=[131072], H=32))
+    assert whole < DD and auto >= 32 * 2 * 2 * DD                  # at least 2 sub-segments each
+    mixed = _in_subprocess_env({"KDA_SEGMENTS": "3"}, _SUMMARY_WS.format(lengths=[300, 1300], H=3))
+    assert mixed >= (3 * 2 + 3 * 3) * 2 * DD                        # P = 2 and 3, S_loc and M each
