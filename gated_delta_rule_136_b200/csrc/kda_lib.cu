@@ -615,17 +615,36 @@ BwdLayout bwd_layout(const kda_fwd_desc &d, const int32_t *cu) {
     BwdLayout w;
     for (int32_t n = 0; n < d.num_seqs; ++n) w.slots += ((int64_t)cu[n + 1] - cu[n]) / kda::bwd::CH;
     const size_t esz = d.io_dtype == KDA_BF16 ? 2 : 4;
-    const size_t DD = (size_t)kda::bwd::D * kda::bwd::D;
+    const size_t DD = (size_t)d.dk * d.dv;
     size_t off = 0;
     w.base = off;    off += align256(sizeof(int64_t) * (size_t)(d.num_seqs + 1));
     w.states = off;  off += align256((size_t)w.slots * d.num_heads * DD * sizeof(float));
-    w.o = off;       off += align256((size_t)d.total_tokens * d.num_heads * kda::bwd::D * esz);
+    w.o = off;       off += align256((size_t)d.total_tokens * d.num_heads * d.dv * esz);
     w.fws_bytes = fwd_workspace_bytes(&d, cu);
     w.fws = off;     off += align256(w.fws_bytes);
-    w.scratch = off; off += align256((size_t)d.num_seqs * d.num_heads * kda::bwd::SCRATCH_FLOATS * sizeof(float));
+    w.scratch = off; off += align256((size_t)d.num_seqs * d.num_heads * kda::bwd::scratch_floats(d.dk, d.dv) * sizeof(float));
     w.total = off;
     return w;
 }
+extern "C++" {
+template <int DK, int DV, typename TIO>
+cudaError_t launch_bwd(const kda::bwd::BwdParams &bp, int64_t units, cudaStream_t stream) {
+    using SM = kda::bwd::BwdSmem<DK, DV>;
+    auto kern = kda::bwd::bwd_kernel<DK, DV, TIO>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::BYTES);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)units, kda::bwd::NT, SM::BYTES, stream>>>(bp);
+    return cudaGetLastError();
+}
+
+template <typename TIO>
+cudaError_t dispatch_bwd(int dk, int dv, const kda::bwd::BwdParams &bp, int64_t units, cudaStream_t stream) {
+    if (dk == 128 && dv == 128) return launch_bwd<128, 128, TIO>(bp, units, stream);
+    if (dk == 128 && dv == 64) return launch_bwd<128, 64, TIO>(bp, units, stream);
+    if (dk == 64 && dv == 128) return launch_bwd<64, 128, TIO>(bp, units, stream);
+    return launch_bwd<64, 64, TIO>(bp, units, stream);
+}
+}  // extern "C++"
 }  // namespace
 
 size_t kda_chunk_bwd_workspace_size(const kda_fwd_desc *desc, const int32_t *cu_seqlens_host) {
@@ -643,7 +662,6 @@ kda_status kda_chunk_bwd(const kda_fwd_desc *desc, const void *q, const void *k,
     kda_status st = validate_fwd_desc(desc);
     if (st != KDA_OK) return st;
     const kda_fwd_desc &d = *desc;
-    if (d.dk != kda::bwd::D || d.dv != kda::bwd::D) return KDA_ERR_UNSUPPORTED;
     if (!cu_seqlens || !cu_seqlens_host) return KDA_ERR_INVALID_ARG;
     if ((st = validate_host_seqlens(desc, cu_seqlens_host)) != KDA_OK) return st;
     const bool any = d.total_tokens > 0;
@@ -656,14 +674,15 @@ kda_status kda_chunk_bwd(const kda_fwd_desc *desc, const void *q, const void *k,
                             static_cast<const void *>(dS0)})   // moved as float4
         if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return KDA_ERR_INVALID_ARG;
     const size_t esz = d.io_dtype == KDA_BF16 ? 2 : 4;
-    const int64_t T = d.total_tokens, DD = (int64_t)kda::bwd::D * kda::bwd::D;
-    const int64_t nk = T * H * 128 * (int64_t)esz, nb = T * H * (int64_t)esz, ns = (int64_t)N * H * DD * 4;
-    const Range ins[] = {range_of(q, nk), range_of(k, nk), range_of(g, nk), range_of(v, nk),
-                         range_of(beta, nb), range_of(gate, gate ? nk : 0), range_of(dout, nk),
+    const int64_t T = d.total_tokens, DD = (int64_t)d.dk * d.dv;
+    const int64_t nk = T * H * d.dk * (int64_t)esz, nv = T * H * d.dv * (int64_t)esz;
+    const int64_t nb = T * H * (int64_t)esz, ns = (int64_t)N * H * DD * 4;
+    const Range ins[] = {range_of(q, nk), range_of(k, nk), range_of(g, nk), range_of(v, nv),
+                         range_of(beta, nb), range_of(gate, gate ? nv : 0), range_of(dout, nv),
                          range_of(S0, S0 ? ns : 0), range_of(dS_T, dS_T ? ns : 0),
                          range_of(cu_seqlens, 4 * (int64_t)(N + 1))};
-    const Range outs[] = {range_of(dq, nk), range_of(dk, nk), range_of(dv, nk), range_of(dg, nk),
-                          range_of(dbeta, nb), range_of(dgate, gate ? nk : 0), range_of(dS0, dS0 ? ns : 0)};
+    const Range outs[] = {range_of(dq, nk), range_of(dk, nk), range_of(dv, nv), range_of(dg, nk),
+                          range_of(dbeta, nb), range_of(dgate, gate ? nv : 0), range_of(dS0, dS0 ? ns : 0)};
     for (const Range &a : outs) {
         for (const Range &b : ins)
             if (overlaps(a, b)) return KDA_ERR_INVALID_ARG;
@@ -705,11 +724,9 @@ kda_status kda_chunk_bwd(const kda_fwd_desc *desc, const void *q, const void *k,
     kda::bwd::BwdParams bp{q, k, v, g, beta, gate, dout, S0, dS_T, cu_seqlens, states, base_dev,
                            reinterpret_cast<float *>(ws + w.scratch), dq, dk, dv, dg, dbeta, dgate, dS0,
                            H, d.scale, d.g_floor};
-    auto kern = d.io_dtype == KDA_BF16 ? kda::bwd::bwd_kernel<__nv_bfloat16> : kda::bwd::bwd_kernel<float>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kda::bwd::SMEM_BYTES) != cudaSuccess)
-        return KDA_ERR_CUDA;
-    kern<<<(unsigned)((int64_t)N * H), kda::bwd::NT, kda::bwd::SMEM_BYTES, stream>>>(bp);
+    const cudaError_t e = d.io_dtype == KDA_BF16 ? dispatch_bwd<__nv_bfloat16>(d.dk, d.dv, bp, (int64_t)N * H, stream)
+                                                 : dispatch_bwd<float>(d.dk, d.dv, bp, (int64_t)N * H, stream);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

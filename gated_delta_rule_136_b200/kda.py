@@ -506,7 +506,7 @@ def chunk_fwd_host(q, k, v, g, beta, cu_seqlens_host, S0=None, gate=None, scale=
 def chunk_bwd(q, k, v, g, beta, dout, cu_seqlens=None, cu_seqlens_host=None, S0=None, gate=None,
               dS_T=None, scale=None, g_floor: float = -5.0, want_dS0: bool = True):
     """``kda_chunk_bwd``: gradients of sum(o * dout) + sum(S_T * dS_T) through
-    the prefill of :func:`chunk_fwd` (same inputs and layouts; dk = dv = 128).
+    the prefill of :func:`chunk_fwd` (same inputs and layouts; dk, dv in {64, 128}).
     Returns a dict: dq, dk, dv, dg, dbeta (input dtype), dgate (if ``gate``)
     and dS0 (fp32 [N,H,dk,dv], if ``want_dS0``)."""
     _require_cuda()

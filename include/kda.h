@@ -307,7 +307,7 @@ kda_status kda_chunk_fwd_host(const kda_fwd_desc *desc, const void *q, const voi
  * head) recomputes each chunk's states from its snapshot and runs the
  * recurrence backwards.  Workspace (device, 256-byte aligned):
  * kda_chunk_bwd_workspace_size(desc, cu_seqlens_host) bytes (SIZE_MAX for a
- * bad descriptor).  dk = dv = 128, else KDA_ERR_UNSUPPORTED;
+ * bad descriptor).  dk, dv in {64, 128}, else KDA_ERR_UNSUPPORTED;
  * KDA_ERR_INVALID_ARG for null, overlapping or inconsistent arguments,
  * KDA_ERR_WORKSPACE for a short or misaligned workspace.  Asynchronous.
  */

@@ -266,7 +266,7 @@ def test_chunk_bwd_validation(lib):
         return lib.kda_chunk_bwd(ctypes.byref(desc), A, A + 4 * MB, A + 8 * MB, A + 12 * MB, A + 16 * MB,
                                  S0, cu_p, cu_h, gate, dout, None, dq, A + 34 * MB, A + 36 * MB,
                                  A + 38 * MB, A + 40 * MB, dgate, dS0, ws, ws_bytes, None)
-    assert bwd(desc=_desc(total_tokens=64, dk=64)) == 2
+    assert bwd(desc=_desc(total_tokens=64, dk=96)) == 2                 # head size outside {64, 128}
     assert bwd(cu_h=None) == 1
     assert bwd(dout=None) == 1
     assert bwd(dq=A + 4 * MB + 64) == 1                     # dq inside k

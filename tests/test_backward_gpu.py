@@ -19,13 +19,13 @@ def _cpu(x):
     return None if x is None else x.detach().to("cpu")
 
 
-def _run(lengths, H, dtype, seed, gate=True, s0=True, ds_t=True, heads=None):
-    inp = inputs.prefill_inputs(lengths, H=H, dk=128, dv=128, dtype=dtype, device="cuda", seed=seed,
+def _run(lengths, H, dtype, seed, gate=True, s0=True, ds_t=True, heads=None, dk=128, dv=128):
+    inp = inputs.prefill_inputs(lengths, H=H, dk=dk, dv=dv, dtype=dtype, device="cuda", seed=seed,
                                 s0_std=0.05 if s0 else None, gate=gate)
     gen = torch.Generator(device="cuda").manual_seed(seed + 1)
     dout = torch.randn(inp["v"].shape, generator=gen, device="cuda").to(dtype)
     N = len(lengths)
-    dS_T = (0.1 * torch.randn((N, H, 128, 128), generator=gen, device="cuda")) if ds_t else None
+    dS_T = (0.1 * torch.randn((N, H, dk, dv), generator=gen, device="cuda")) if ds_t else None
     got = chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], dout,
                     cu_seqlens=inp["cu_seqlens"], cu_seqlens_host=inp["cu_seqlens_host"], S0=inp["S0"],
                     gate=inp["gate"], dS_T=dS_T)
@@ -52,6 +52,13 @@ def _check(got, ref, dtype):
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_backward_matches_oracle(dtype):
     got, ref = _run([150, 0, 70, 64], H=2, dtype=dtype, seed=101)
+    _check(got, ref, dtype)
+
+
+@pytest.mark.parametrize("dk,dv,dtype", [(64, 64, torch.float32), (128, 64, torch.bfloat16),
+                                         (64, 128, torch.float32)])
+def test_backward_other_head_sizes(dk, dv, dtype):
+    got, ref = _run([150, 70], H=2, dtype=dtype, seed=109, dk=dk, dv=dv)
     _check(got, ref, dtype)
 
 
