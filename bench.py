@@ -66,7 +66,7 @@ PROFILED_TRAFFIC = {
                           "bytes_per_head_round": (579.116800e6 + 4.305920e6 + 555.884544e6 + 477.843968e6) / 8192,
                           "profile": "profiles/spec_kernel_verify_commit_128x64.md"},
     # backward kernel at 2 x 1024 x 16 (bf16): per token-head (the forward with snapshots not included)
-    "csrc/kda_bwd.cuh": {"sha1": "efb7c2732829", "bytes_per_token_head": (74.357504e6 + 29.543424e6) / 32768,
+    "csrc/kda_bwd.cuh": {"sha1": "674b7f1ed170", "bytes_per_token_head": (74.136576e6 + 30.980096e6) / 32768,
                          "profile": "profiles/bwd_kernel_2x1024x16.md"},
 }
 
