@@ -281,7 +281,9 @@ kda_status kda_chunk_fwd_snapshots(const kda_fwd_desc *desc, const kda_snapshots
  * with_S0, with_S_T) bytes.  When the call returns the work is enqueued;
  * synchronising `stream` waits for every copy.  Calls on one device are
  * serialised while they enqueue (they share two copy streams).  Errors as
- * kda_chunk_fwd; KDA_ERR_WORKSPACE for a short or misaligned workspace.
+ * kda_chunk_fwd; KDA_ERR_WORKSPACE for a short or misaligned workspace.  An
+ * error after the first group was enqueued can leave copies in flight:
+ * synchronise the device before reusing the buffers.
  */
 size_t kda_chunk_fwd_host_workspace_size(const kda_fwd_desc *desc, const int32_t *cu_seqlens_host,
                                          int32_t with_gate, int32_t with_S0, int32_t with_S_T);
