@@ -6,7 +6,10 @@ B=8 sequences x T=4096 tokens, H=32 heads, dk=dv=128, S0 = 0, final state
 returned -- the configuration the headline metric is quoted on.  The decode
 hot path is measured in the same run (512 sequences x 64 heads, 128x128 fp32
 state per head, bf16 inputs with a sigmoid output gate, 1000 consecutive
-steps) and reported in the ``decode`` object of the same JSON line.
+steps) and reported in the ``decode`` object of the same JSON line, and so
+are the two other prefill workloads (64 varlen sequences x 64 heads; one
+2^20-token sequence x 32 heads with decay near the floor), each with its own
+roofline object under ``other_workloads`` (``--no-extra`` skips them).
 
 Prints ONE JSON line on rank 0.  ``--impl reference`` times the fp64 CPU
 oracle (the only reference implementation there is) on a bounded sample of
@@ -39,6 +42,7 @@ CHUNK_ALG = 64
 # workload (decode)
 DEC_B, DEC_H, DEC_STEPS = 512, 64, 1000
 EXTRA_WORKLOADS = ("varlen", "long", "snapshots", "spec", "backward", "kcp")
+DEFAULT_EXTRAS = ("varlen", "long")   # the other two prefill workloads, timed in every run
 
 
 def flops_per_token_head(dk=DK, dv=DV, C=CHUNK_ALG):
@@ -251,7 +255,10 @@ def main():
     ap.add_argument("--decode-batch", type=int, default=DEC_B)
     ap.add_argument("--decode-steps", type=int, default=DEC_STEPS)
     ap.add_argument("--extra", default="",
-                    help="comma-separated extra workloads to time: " + ", ".join(EXTRA_WORKLOADS))
+                    help="comma-separated extra workloads to time: " + ", ".join(EXTRA_WORKLOADS)
+                         + " (varlen and long are timed by default)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only the headline prefill and the decode (not varlen / long)")
     ap.add_argument("--all-workloads", action="store_true",
                     help="also time the varlen (64 x [512, 32768] x 64 heads) and the "
                          "1M-token x 32-head floor-stress prefill, the headline prefill "
@@ -260,7 +267,11 @@ def main():
                          "with more than one rank, the context-parallel prefill")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
-    extras = set(EXTRA_WORKLOADS) if args.all_workloads else {x for x in args.extra.split(",") if x}
+    extras = {x for x in args.extra.split(",") if x}
+    if args.all_workloads:
+        extras = set(EXTRA_WORKLOADS)
+    elif not args.no_extra:
+        extras |= set(DEFAULT_EXTRAS)
     if extras - set(EXTRA_WORKLOADS):
         ap.error(f"--extra: unknown workload(s) {sorted(extras - set(EXTRA_WORKLOADS))}; "
                  f"choose from {', '.join(EXTRA_WORKLOADS)}")
@@ -465,9 +476,14 @@ def main():
             ttok = int(w["q"].shape[0])
             byts = ttok * c["H"] * bytes_per_token_head() + len(c["lengths"]) * c["H"] * DK * DV * 4 * (
                 2 if c["s0_std"] is not None else 1)
+            gbs = byts / (ms / 1e3) / 1e9
             others[name] = {"tokens": ttok, "ms": ms, "tokens_per_s": world * ttok / (ms / 1e3),
-                            "alg_gbs": byts / (ms / 1e3) / 1e9,
-                            "roofline_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+                            "alg_gbs": gbs, "roofline_frac": gbs / peaks["hbm_gbs"],
+                            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                                         "traffic": None, "alg_bytes_per_launch": byts,
+                                         "kernel": "kda_chunk_fwd (plan or segment split + chunk kernel)",
+                                         "peak_source": peaks["source"]}}
             del w, ow, Sw, wsw
             torch.cuda.empty_cache()
 

@@ -19,8 +19,13 @@
 // in parallel, then the state carried to the next chunk: fupanwang.com digest,
 // section 基础设施, FlashKDA).
 //
-// Precision: the products the outputs are sensitive to run in tf32 (A_qk /
-// A_kk operands, T' (K e^G) S, A_qk Vn, K^(4)^T Vn); T' V, (K e^G) S and (Q e^G) S run in bf16.
+// Precision: the products the outputs are sensitive to run in tf32 (the A_qk /
+// A_kk operands of every block, rounded to nearest, T' (K e^G) S, A_qk Vn,
+// K^(4)^T Vn); T' V, (K e^G) S and (Q e^G) S run in bf16, with S carried as a
+// leading bf16 part plus a bf16 low part (each state product issued once per
+// part into the same accumulator).  On the full-size workloads the bf16
+// off-diagonal A operands and the bf16 state were the largest terms of the
+// output error.
 //
 // Orientation: the state products are computed transposed so that the value
 // channel v is the TMEM lane (M = 128): S^T and Vn^T live in TMEM as the A
@@ -61,8 +66,7 @@ constexpr uint32_t OFF_INTRA = 65536;     // 72 KB, reused after the A MMAs
 //   during prep / A MMAs (per pass of 64 channels):
 constexpr uint32_t OFF_XT = OFF_INTRA;             // X~ [128 rows x 64 ch] tf32 K-major: 2 x 16 KB
 constexpr uint32_t OFF_KD = OFF_INTRA + 32768;     // Kbar [64 rows j x 64 ch] tf32 K-major: 2 x 8 KB
-constexpr uint32_t OFF_XB = OFF_INTRA + 49152;     // X~ rows 32-127 (blocks 1-3) bf16 K-major: 12 KB
-constexpr uint32_t OFF_KO = OFF_INTRA + 61440;     // K^(b) rows j < 16 b, b = 1..3, bf16 K-major: 12 KB
+constexpr uint32_t OFF_KO = OFF_INTRA + 49152;     // K^(b) rows j < 16 b, b = 1..3, tf32 K-major: 24 KB
 //   after the A MMAs:
 constexpr uint32_t OFF_SCR = OFF_INTRA;            // A_kk -> T, fp32 [64][68]
 constexpr uint32_t SCR_LD = 68;                    // 16-byte aligned rows
@@ -88,18 +92,21 @@ constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024; // slack for aligning the bas
 static_assert(OFF_TP % 1024 == 0 && OFF_TP + 16384 <= OFF_XS && OFF_XS + 4096 <= OFF_TPB &&
               OFF_TPB % 1024 == 0 && OFF_TPB + 8192 <= OFF_INTRA + 73728, "post-MMA tiles fit the intra region");
 static_assert((OFF_KG - OFF_QG) % 16 == 0, "Q e^G | K e^G as one MN-major operand");
-static_assert(OFF_KO + 12288 == OFF_INTRA + 73728, "intra tiles fit");
+static_assert(OFF_KO + 24576 == OFF_INTRA + 73728, "intra tiles fit");
 static_assert(SMEM_ALLOC <= 232448, "fits in 227 KB");
 
 // Off-diagonal column operands: tile b (b = 1..3) holds K^(b) rows j < 16 b
-// (tokens of the blocks before b) in bf16, one 128-byte K-block of 64 channels;
-// tiles are packed back to back.  The MMA (M = 64) reads 64 rows from a tile's
-// start; rows past the valid ones read neighbouring bytes (the next tile, or
-// for b = 3 the first 2 KB after the intra region), which only feed
-// accumulator rows that are never used.
-__host__ __device__ constexpr uint32_t ko_base(int b) { return 1024u * (uint32_t)b * (uint32_t)(b - 1); }
-static_assert(ko_base(1) == 0u && ko_base(2) == 2048u && ko_base(3) == 6144u, "packing");
-static_assert(OFF_KO + ko_base(3) + 64u * 128u <= OFF_QG + 16384u, "K^(b) reads stay in shared memory");
+// (tokens of the blocks before b) in tf32, two 128-byte K-blocks of 32
+// channels (16 b rows each, 2 KB x b); tiles are packed back to back.  The MMA
+// (M = 64) reads 64 rows from a K-block's start; rows past the valid ones read
+// neighbouring bytes (the next K-block or tile, or for b = 3 the first 2 KB
+// after the intra region), which only feed accumulator rows that are never
+// used.  The row operand is the tf32 X~ tile of the diagonal product.
+__host__ __device__ constexpr uint32_t ko_base(int b) { return 2048u * (uint32_t)b * (uint32_t)(b - 1); }
+__host__ __device__ constexpr uint32_t ko_kblk(int b) { return 2048u * (uint32_t)b; }
+static_assert(ko_base(1) == 0u && ko_base(2) == 4096u && ko_base(3) == 12288u, "packing");
+static_assert(ko_base(3) + 2u * ko_kblk(3) == 24576u, "tiles fill the region");
+static_assert(OFF_KO + ko_base(3) + ko_kblk(3) + 64u * 128u <= OFF_QG + 16384u, "K^(b) reads stay in shared memory");
 
 // ---- TMEM columns
 constexpr uint32_t T_DD = 0;      // diagonal A MMA [64 j x 128 X~ rows] (M = 64 layout)
@@ -109,7 +116,8 @@ constexpr uint32_t T_DS = 64;     // dS^T          [v x c]   } A readout and Vn
 constexpr uint32_t T_VN = 192;    // Vn^T = V^T T'^T - Y^T T'^T, then its tf32 copy (A operand)
 constexpr uint32_t T_O1 = 256;    // ((Q e^G) S)^T  [v x i]  } one MMA (N = 128)
 constexpr uint32_t T_Z = 320;     // -((K e^G) S)^T  [v x j] (read as a tf32 A operand)
-constexpr uint32_t T_S = 384;     // S^T bf16 A operand (2 per column)
+constexpr uint32_t T_S = 384;     // S^T bf16 A operand (2 per column): the leading bf16 part
+constexpr uint32_t T_LO = 448;    // S^T - bf16(S^T) in bf16: the low part of the same operand
 constexpr uint32_t TMEM_COLS = 512;
 
 // One explicit work unit (used by the long-sequence segment split): a token
@@ -328,8 +336,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t sw_lane = ((((kbyte >> 4) & 7u) ^ (uint32_t)gq) << 4) + (kbyte & 15u);
     const uint32_t xt_lane = OFF_XT + kblk * 16384u + sw_lane;
     const uint32_t kd_lane = OFF_KD + kblk * 8192u + sw_lane;
-    // the same for the bf16 tiles (one 128-byte K-block of 64 channels)
-    const uint32_t xb_lane = OFF_XB + (((((uint32_t)cA * 2u) >> 4) ^ (uint32_t)gq) << 4) + (((uint32_t)cA * 2u) & 15u);
     // constant A fragments of the prefix-sum products (bf16 1.0 = 0x3F80):
     //   a_blk: 16x16 lower triangle with diagonal;  a_ref[kb]: rows m < 4 select block kb <= m
     uint32_t a_blk[4];
@@ -394,11 +400,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int r = 0; r < 32; ++r)
         S[r] = S0p ? S0p[(cq * 32 + r) * D + vlane]
                    : ((flags & UNIT_S0_IDENTITY) && cq * 32 + r == vlane ? 1.0f : 0.0f);
-    auto store_state_bf16 = [&]() {        // S^T as the bf16 A operand (2 rows c per column)
-        uint32_t r16[16];
+    auto store_state_bf16 = [&]() {        // S^T as the bf16 A operand (2 rows c per column):
+        uint32_t r16[16];                   // the leading part, then the low part
 #pragma unroll
         for (int e = 0; e < 16; ++e) r16[e] = pack_bf16(S[2 * e], S[2 * e + 1]);
         tmem_st16(tbase + lane_base + T_S + cq * 16, r16);
+        tmem_wait_st();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float2 hi = unpack_bf16x2(r16[e]);
+            r16[e] = pack_bf16(S[2 * e] - hi.x, S[2 * e + 1] - hi.y);
+        }
+        tmem_st16(tbase + lane_base + T_LO + cq * 16, r16);
         tmem_wait_st();
     };
     store_state_bf16();
@@ -451,7 +464,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     // MMA descriptors that do not depend on the chunk (start addresses advance per K-step)
     const uint32_t id_d = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 64, 128);
-    const uint32_t id_o = instr_desc(FMT_BF16, K_MAJOR, K_MAJOR, 64, 32);
+    const uint32_t id_o = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 64, 32);
     const uint32_t id_1 = instr_desc(FMT_BF16, K_MAJOR, MN_MAJOR, 128, 128);
     const uint32_t id_vn = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 128, 64);
     const uint32_t id_u = instr_desc(FMT_BF16, MN_MAJOR, K_MAJOR, 128, 64);
@@ -467,7 +480,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     //           channels (tf32, M = 64, N = 128: every block against every
     //           block, of which the diagonal 16 x 32 tiles are used), and the
     //           off-diagonal product of block 1;
-    //   part 1: the off-diagonal products of blocks 2 and 3 (bf16, M = 64, N = 32:
+    //   part 1: the off-diagonal products of blocks 2 and 3 (tf32, M = 64, N = 32:
     //           K^(b) rows j < 16 b against X~ rows of block b); then commit, and
     //           this pass's half of [O1 | -Y]^T = S^T [Q e^G | -K e^G]^T (bf16, A =
     //           S^T from TMEM), which runs behind the A MMAs, off the critical path.
@@ -484,10 +497,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int bo = 1; bo < NB; ++bo) {
             if ((bo == 1) != (part == 0)) continue;
 #pragma unroll
-            for (int s = 0; s < 4; ++s)            // bf16 K-steps of 16 channels
-                if (leader) mma_bf16_ss(tbase + T_DO + 32u * (bo - 1), at(d_k16, OFF_KO + ko_base(bo) + 32u * s),
-                                        at(d_k16, OFF_XB + 32u * (bo - 1) * 128u + 32u * s), id_o,
+            for (int s = 0; s < 8; ++s) {          // tf32 K-steps of 8 channels
+                const uint32_t kb = (uint32_t)(s >> 2), koff = (uint32_t)(s & 3) * 32u;
+                if (leader) mma_tf32_ss(tbase + T_DO + 32u * (bo - 1),
+                                        at(d_k16, OFF_KO + ko_base(bo) + kb * ko_kblk(bo) + koff),
+                                        at(d_k16, OFF_XT + kb * 16384u + 32u * (uint32_t)bo * 128u + koff), id_o,
                                         (pass_ > 0 || s > 0) ? 1u : 0u);
+            }
         }
         if (part == 1) {
             if (leader) mma_commit(bar_mma);
@@ -495,6 +511,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int s = 0; s < 4; ++s) {
                 const uint32_t ks = (uint32_t)(4 * pass_ + s);   // K = 128 key channels in steps of 16
                 if (leader) mma_bf16_ts(tbase + T_O1, tbase + T_S + 8u * ks, at(d_qk, OFF_QG + 2048u * ks), id_1, ks > 0);
+                if (leader) mma_bf16_ts(tbase + T_O1, tbase + T_LO + 8u * ks, at(d_qk, OFF_QG + 2048u * ks), id_1, 1u);
             }
             if (pass_ == 1 && leader) mma_commit(bar_y);
         }
@@ -679,10 +696,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     ++mma_phase;
                     tc_fence_after();
                 }
-                // (4) the A-MMA operands: X~ rows (q~ at 32 b + r, k~ at 32 b + 16 + r) and Kbar
-                //     (tf32 operands of the diagonal product: the MMA reads the leading 19
-                //     bits), X~ rows of blocks 1-3 again in bf16, and the K^(b') copies,
-                //     b' > b, in bf16 for the off-diagonal products
+                // (4) the A-MMA operands, rounded to tf32: X~ rows (q~ at 32 b + r, k~ at
+                //     32 b + 16 + r) and Kbar for the diagonal product, and the K^(b') copies,
+                //     b' > b, for the off-diagonal products (whose rows are the same X~)
 #pragma unroll
                 for (int bb = 0; bb < 2; ++bb) {
                     const int b = 2 * mp + bb;
@@ -699,18 +715,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int hr = 0; hr < 2; ++hr) {
                         const uint32_t i = (uint32_t)(16 * b + 8 * hr) + (uint32_t)gq;
                         const uint32_t xrow = (uint32_t)(32 * b + 8 * hr) + (uint32_t)gq;
-                        *reinterpret_cast<float2 *>(sm + xt_lane + xrow * 128u) = qt[bb][hr];
-                        *reinterpret_cast<float2 *>(sm + xt_lane + (xrow + 16u) * 128u) = kt[bb][hr];
-                        *reinterpret_cast<float2 *>(sm + kd_lane + i * 128u) = kbar[bb][hr];
-                        if (b > 0) {
-                            *reinterpret_cast<uint32_t *>(sm + xb_lane + (xrow - 32u) * 128u) = pack_bf16(qt[bb][hr].x, qt[bb][hr].y);
-                            *reinterpret_cast<uint32_t *>(sm + xb_lane + (xrow - 16u) * 128u) = pack_bf16(kt[bb][hr].x, kt[bb][hr].y);
-                        }
+                        auto rnd2 = [](float2 x) { return make_float2(to_tf32(x.x), to_tf32(x.y)); };
+                        *reinterpret_cast<float2 *>(sm + xt_lane + xrow * 128u) = rnd2(qt[bb][hr]);
+                        *reinterpret_cast<float2 *>(sm + xt_lane + (xrow + 16u) * 128u) = rnd2(kt[bb][hr]);
+                        *reinterpret_cast<float2 *>(sm + kd_lane + i * 128u) = rnd2(kbar[bb][hr]);
 #pragma unroll
                         for (int m = 1; m < NB; ++m) {
                             if (m <= b) continue;
                             const float2 v = __fmul2_rn(kbar[bb][hr], dfac[m]);
-                            *reinterpret_cast<uint32_t *>(sm + xb_lane - OFF_XB + OFF_KO + ko_base(m) + i * 128u) = pack_bf16(v.x, v.y);
+                            *reinterpret_cast<float2 *>(sm + OFF_KO + ko_base(m) + kblk * ko_kblk(m) + sw_lane + i * 128u) =
+                                rnd2(v);
                         }
                     }
                 }

@@ -9,6 +9,7 @@
 #include <cstring>
 
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 #include <algorithm>
 #include <cstdlib>
 #include <mutex>
@@ -22,6 +23,17 @@
 #include "kda_plan.cuh"
 #include "kda_segment.cuh"
 #include "kda_bwd.cuh"
+
+namespace {
+// NVTX range over a host-side launch sequence (plan, chunk passes, scan, ...):
+// a profiler attached to the process shows which kernels each range issued.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+}  // namespace
 
 namespace {
 
@@ -366,15 +378,20 @@ cudaError_t launch_split(const kda_fwd_desc &d, const SegPlan &pl, const int32_t
     kda::tck::TcParams tp{beta, gate, nullptr, nullptr, nullptr, o, nullptr, H, d.scale, d.g_floor, d1, sn};
     if (!p1.empty()) {
         tp.units = d1;
+        NvtxRange r("kda.split.pass1");
         if ((e = launch_tc_units(d, q, k, v, g, tp, (int64_t)p1.size(), stream)) != cudaSuccess) return e;
     }
     const size_t scan_smem = 2u * DD * sizeof(float);
     if ((e = cudaFuncSetAttribute(kda::segment_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)scan_smem)) != cudaSuccess)
         return e;
-    kda::segment_scan_kernel<<<(unsigned)jobs.size(), 256, scan_smem, stream>>>(dj);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    {
+        NvtxRange r("kda.split.scan");
+        kda::segment_scan_kernel<<<(unsigned)jobs.size(), 256, scan_smem, stream>>>(dj);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     tp.units = d2;
+    NvtxRange r("kda.split.pass2");
     return launch_tc_units(d, q, k, v, g, tp, (int64_t)p2.size(), stream);
 }
 
@@ -516,9 +533,13 @@ kda_status chunk_fwd_impl(const kda_fwd_desc *desc, const kda_snapshots *snap, c
     }
 
     int32_t *seq_order = static_cast<int32_t *>(workspace);
-    cudaError_t e = kda::launch_plan_longest_first(cu_seqlens, d.num_seqs, seq_order, stream);
+    cudaError_t e;
+    {
+        NvtxRange r("kda.plan");
+        e = kda::launch_plan_longest_first(cu_seqlens, d.num_seqs, seq_order, stream);
+    }
     if (e != cudaSuccess) return KDA_ERR_CUDA;
-
+    NvtxRange r("kda.prefill");
     e = launch_prefill(d, q, k, v, g, beta, S0, cu_seqlens, seq_order, gate, o, S_T, sn, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
@@ -568,6 +589,7 @@ kda_status kda_decode_step(const kda_decode_desc *desc, const void *q, const voi
     if (overlaps(rS, ro)) return KDA_ERR_INVALID_ARG;
 
     DecodeParams p{q, k, v, g, beta, gate, S, o, d.scale, d.g_floor};
+    NvtxRange r("kda.decode");
     cudaError_t e = d.io_dtype == KDA_BF16 ? dispatch_decode<__nv_bfloat16>(d.dk, d.dv, p, units, stream)
                                            : dispatch_decode<float>(d.dk, d.dv, p, units, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
@@ -583,6 +605,7 @@ kda_status kda_spec_verify(const kda_spec_desc *desc, const void *q, const void 
     kda::SpecParams p{q, k, v, g, beta, gate, const_cast<float *>(S), o, nullptr, d.num_heads,
                       d.draft, d.scale, d.g_floor};
     const int64_t units = (int64_t)d.batch * d.num_heads;
+    NvtxRange r("kda.spec.verify");
     cudaError_t e = d.io_dtype == KDA_BF16 ? dispatch_spec<__nv_bfloat16, false>(d.dk, d.dv, p, units, stream)
                                            : dispatch_spec<float, false>(d.dk, d.dv, p, units, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
@@ -598,6 +621,7 @@ kda_status kda_spec_commit(const kda_spec_desc *desc, const void *q, const void 
     kda::SpecParams p{q, k, v, g, beta, nullptr, S, nullptr, accepted, d.num_heads, d.draft,
                       d.scale, d.g_floor};
     const int64_t units = (int64_t)d.batch * d.num_heads;
+    NvtxRange r("kda.spec.commit");
     cudaError_t e = d.io_dtype == KDA_BF16 ? dispatch_spec<__nv_bfloat16, true>(d.dk, d.dv, p, units, stream)
                                            : dispatch_spec<float, true>(d.dk, d.dv, p, units, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
@@ -724,6 +748,7 @@ kda_status kda_chunk_bwd(const kda_fwd_desc *desc, const void *q, const void *k,
     kda::bwd::BwdParams bp{q, k, v, g, beta, gate, dout, S0, dS_T, cu_seqlens, states, base_dev,
                            reinterpret_cast<float *>(ws + w.scratch), dq, dk, dv, dg, dbeta, dgate, dS0,
                            H, d.scale, d.g_floor};
+    NvtxRange r("kda.bwd");
     const cudaError_t e = d.io_dtype == KDA_BF16 ? dispatch_bwd<__nv_bfloat16>(d.dk, d.dv, bp, (int64_t)N * H, stream)
                                                  : dispatch_bwd<float>(d.dk, d.dv, bp, (int64_t)N * H, stream);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
@@ -889,7 +914,10 @@ kda_status kda_segment_summary(const kda_fwd_desc *desc, const void *q, const vo
         return KDA_ERR_CUDA;
     kda::tck::TcParams tp{beta, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, H, d.scale,
                           d.g_floor, du, kda::SnapOut{nullptr, nullptr, 0, 64}};
-    if (launch_tc_units(d, q, k, v, g, tp, (int64_t)units.size(), stream) != cudaSuccess) return KDA_ERR_CUDA;
+    {
+        NvtxRange r("kda.summary.chains");
+        if (launch_tc_units(d, q, k, v, g, tp, (int64_t)units.size(), stream) != cudaSuccess) return KDA_ERR_CUDA;
+    }
     if (jobs.empty()) return KDA_OK;
     kda::ScanJob *dj = reinterpret_cast<kda::ScanJob *>(ws + w.jobs);
     if (cudaMemcpyAsync(dj, jobs.data(), jobs.size() * sizeof(kda::ScanJob), cudaMemcpyHostToDevice,
@@ -899,6 +927,7 @@ kda_status kda_segment_summary(const kda_fwd_desc *desc, const void *q, const vo
     if (cudaFuncSetAttribute(kda::segment_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)scan_smem) != cudaSuccess)
         return KDA_ERR_CUDA;
+    NvtxRange r("kda.summary.scan");
     kda::segment_scan_kernel<<<(unsigned)jobs.size(), 256, scan_smem, stream>>>(dj);
     return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
@@ -923,6 +952,7 @@ kda_status kda_state_combine(const kda_combine_desc *desc, const float *summarie
     if (cudaFuncSetAttribute(kda::state_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return KDA_ERR_CUDA;
+    NvtxRange r("kda.combine");
     kda::state_combine_kernel<<<(unsigned)units, 256, smem, stream>>>(summaries, S_in, units,
                                                                       c.num_summaries);
     return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
@@ -995,23 +1025,50 @@ static __device__ __align__(256) int32_t g_noalloc_seq_order[KDA_NOALLOC_MAX_SEQ
 
 constexpr int kMaxDevices = 128;
 std::mutex g_noalloc_mutex;
-int32_t *g_noalloc_ptr[kMaxDevices] = {};
+struct NoallocSlot {
+    CUcontext ctx;      // the context the address belongs to
+    int32_t *ptr;
+};
+NoallocSlot g_noalloc_slot[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device, looked up once
-// per device (the host-side symbol is only a stand-in, not a device address).
+// cuCtxGetCurrent through the runtime (no link against the driver library).
+PFN_cuCtxGetCurrent_v4000 ctx_getter() {
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &ptr, 4000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(ptr);
+    });
+    return fn;
+}
+
+// Device address of the scratch array in the current context.  The address
+// is cached per device together with the context it was looked up in; a new
+// context on the device (after cudaDeviceReset, or after the primary context
+// was released and created again) looks it up afresh.
 cudaError_t noalloc_scratch(int32_t **out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    PFN_cuCtxGetCurrent_v4000 get_ctx = ctx_getter();
+    CUcontext ctx = nullptr;
+    if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS) return cudaErrorInitializationError;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
+    NoallocSlot &slot = g_noalloc_slot[dev];
+    if (!slot.ptr || !ctx || slot.ctx != ctx) {
         void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_seq_order);
+        e = cudaGetSymbolAddress(&p, g_noalloc_seq_order);   // (creates the context if none is current)
         if (e != cudaSuccess) return e;
-        g_noalloc_ptr[dev] = static_cast<int32_t *>(p);
+        if (!ctx && (get_ctx(&ctx) != CUDA_SUCCESS || !ctx)) return cudaErrorInitializationError;
+        slot.ctx = ctx;
+        slot.ptr = static_cast<int32_t *>(p);
     }
-    *out = g_noalloc_ptr[dev];
+    *out = slot.ptr;
     return cudaSuccess;
 }
 
@@ -1046,6 +1103,7 @@ extern "C" kda_status kda_chunk_fwd_noalloc(const kda_fwd_desc *desc, const void
     if (noalloc_scratch(&seq_order) != cudaSuccess) return KDA_ERR_CUDA;
     // every entry [0, num_seqs) is rewritten by the plan kernel before use,
     // so the previous call's contents never need clearing
+    NvtxRange r("kda.prefill.noalloc");
     cudaError_t e = kda::launch_plan_longest_first(cu_seqlens, d.num_seqs, seq_order, stream);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     e = launch_prefill(d, q, k, v, g, beta, S0, cu_seqlens, seq_order, gate, o, S_T, kda::SnapOut{nullptr, nullptr, 0, 64}, stream);
@@ -1210,6 +1268,7 @@ extern "C" kda_status kda_chunk_fwd_host(const kda_fwd_desc *desc, const void *q
     const int G = (int)w.groups.size();
     for (int i = 0; i < G; ++i) {
         const HostGroup &gr = w.groups[i];
+        NvtxRange r("kda.host.group");
         const int sl = i & 1;
         unsigned char *in = ws + w.in[sl], *out = ws + w.out[sl];
         const size_t nt = (size_t)(gr.t1 - gr.t0), ns = (size_t)(gr.s1 - gr.s0);

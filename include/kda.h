@@ -199,17 +199,24 @@ kda_status kda_spec_commit(const kda_spec_desc *desc, const void *q, const void 
  * input and output buffers, or a runtime that plans all device memory up
  * front and allows no allocation once it runs.
  *
- * Arguments and results are those of kda_chunk_fwd (same kernels, same
- * numbers), minus cu_seqlens_host and the workspace.  The scratch it needs
+ * Arguments are those of kda_chunk_fwd minus cu_seqlens_host and the
+ * workspace; the results agree with kda_chunk_fwd's within the parity
+ * tolerances.  Without cu_seqlens_host this entry point never splits a long
+ * sequence into segments: every (sequence, head) pair runs as one CTA, so
+ * with fewer pairs than SMs (one long sequence, few heads) it leaves SMs
+ * idle and rounds differently from kda_chunk_fwd, which splits such
+ * sequences.  The scratch it needs
  * (one int32 per sequence) is a fixed array inside the library, sized for
  * KDA_NOALLOC_MAX_SEQS sequences; every GPU that loads the library keeps
  * that array (256 KiB) until the process exits.
  *   - num_seqs > KDA_NOALLOC_MAX_SEQS returns KDA_ERR_WORKSPACE and launches
  *     nothing.
  *   - The call allocates no device or host memory.
- *   - The first call on each device looks up the array's device address
+ *   - The first call in each context looks up the array's device address
  *     (with that device current); make that first call before any stream
- *     capture begins on the device.
+ *     capture begins on the device.  The address is cached with the context
+ *     it belongs to: after cudaDeviceReset (or any new primary context) the
+ *     next call looks it up again.
  *   - All calls on a device share the one array and it keeps the last
  *     call's contents (each call rewrites the part it reads before reading
  *     it).  Calls whose kernels can overlap on the GPU -- on different

@@ -30,13 +30,15 @@ The 16-token blocks are where the per-step floor matters: within a block
 every factor is bounded by e^{-16 floor}, inside bf16/fp32 range for floor >= -5.45
 (fupanwang.com Kimi K3 report digest, KDA section, Fig. 3).
 
-``prec`` (a dict operand -> "bf16" | "tf32" | "tf32t") rounds the tensor-core
-operands the way a kernel stores them ("tf32t": fp32 stored whole, the MMA
-reading only its leading 19 bits, i.e. truncation); ``KERNEL_PREC`` with
-``KERNEL_FORM`` is the plan of the tcgen05 kernel: tf32 for the operands the
-output is sensitive to (the intra-chunk A operands, A_qk, T', Z, V_new, K^)
-and bf16 for the state and Q e^G / K e^G.  beta is folded into the columns of
-T (T' = T Diag(beta)).
+``prec`` (a dict operand -> "bf16" | "tf32" | "tf32t" | "bf16x2" | "tf32x2")
+rounds the tensor-core operands the way a kernel stores them ("tf32t": fp32
+stored whole, the MMA reading only its leading 19 bits, i.e. truncation;
+"...x2": a leading part plus a low part in that type, the product issued once
+per part); ``KERNEL_PREC`` with ``KERNEL_FORM`` is the plan of the tcgen05
+kernel: tf32 for the operands the output is sensitive to (the intra-chunk A
+operands, A_qk, T', Z, V_new, K^), the state as two bf16 parts, bf16 for
+Q e^G / K e^G and T' in T' V.  beta is folded into the columns of T
+(T' = T Diag(beta)).
 """
 from __future__ import annotations
 
@@ -69,15 +71,26 @@ def _tf32_trunc(x):
     return u.view(np.float32).astype(np.float64)
 
 
+def _split2(rnd):
+    """An operand carried as a leading part plus a low part, both in the same
+    storage type (the product is issued once per part into one accumulator)."""
+    def f(x):
+        x = np.asarray(x, np.float32).astype(np.float64)
+        hi = rnd(x)
+        return hi + rnd(x - hi)
+    return f
+
+
 _ROUND = {"bf16": _bf16, "tf32": _tf32, "tf32t": _tf32_trunc,
+          "bf16x2": _split2(_bf16), "tf32x2": _split2(_tf32),
           "fp32": lambda x: np.asarray(x, np.float32).astype(np.float64)}
 
 # operand -> storage precision in the tcgen05 kernel, and the form of its V_new
 KERNEL_PREC = {
-    "Arow": "tf32t", "Acol": "tf32t",     # q~, k~ and Kbar of the diagonal A blocks
-    "Aoff": "bf16",                       # q~, k~ and K^(b) of the off-diagonal A blocks
+    "Arow": "tf32", "Acol": "tf32",       # q~, k~ and Kbar of the diagonal A blocks (rounded)
+    "Aoff": "tf32",                       # q~, k~ and K^(b) of the off-diagonal A blocks (rounded)
     "Aqk": "tf32", "T": "tf32t", "TV": "bf16", "Y": "tf32t", "Vn": "tf32", "Khat": "tf32",
-    "KG": "bf16", "S": "bf16", "QG": "bf16",
+    "KG": "bf16", "S": "bf16x2", "QG": "bf16",
 }
 KERNEL_FORM = "split"
 

@@ -334,3 +334,16 @@ def test_summary_split_plan_sizes():
     assert whole < DD and auto >= 32 * 2 * 2 * DD                  # at least 2 sub-segments each
     mixed = _in_subprocess_env({"KDA_SEGMENTS": "3"}, _SUMMARY_WS.format(lengths=[300, 1300], H=3))
     assert mixed >= (3 * 2 + 3 * 3) * 2 * DD                        # P = 2 and 3, S_loc and M each
+
+
+def test_library_carries_nvtx_ranges():
+    """The host code marks its launch sequences with NVTX ranges (plan, the
+    split's two passes and scan, prefill, decode, speculative verify/commit,
+    backward, summary, combine, host pipeline), so a profiler attached to the
+    process can attribute kernels; the range names are compiled into the
+    library."""
+    blob = open(kda.library_path(), "rb").read()
+    for name in ("kda.plan", "kda.prefill", "kda.split.pass1", "kda.split.scan", "kda.split.pass2",
+                 "kda.decode", "kda.spec.verify", "kda.spec.commit", "kda.bwd", "kda.summary.chains",
+                 "kda.summary.scan", "kda.combine", "kda.host.group", "kda.prefill.noalloc"):
+        assert name.encode() + b"\0" in blob, name

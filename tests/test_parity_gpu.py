@@ -10,7 +10,7 @@ import torch
 
 import oracle
 from gated_delta_rule_136_b200 import chunk_fwd, decode_step, device_status, inputs
-from parity import TOL_BF16, TOL_FP32, rel_max, rel_max_beyond_bf16
+from parity import TOL_BF16, TOL_FP32, bf16_half_ulp, rel_max, rel_max_beyond_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -22,14 +22,17 @@ def _cpu(x):
 
 
 def _oracle_prefill(inp, heads=None, seqs=None, g_floor=-5.0):
-    """Oracle on a subset of heads / sequences (units are independent)."""
-    q, k, v, g, beta = (_cpu(inp[n]) for n in ("q", "k", "v", "g", "beta"))
-    gate, S0 = _cpu(inp["gate"]), _cpu(inp["S0"])
+    """Oracle on a subset of heads / sequences (units are independent).  The
+    heads are selected on the device, so only their slices reach the host."""
+    def pick(name):
+        t = inp[name]
+        if t is None:
+            return None
+        if heads is not None:   # dim 1 is the head for every input, S0 included
+            t = t.index_select(1, torch.tensor(heads, device=t.device))
+        return _cpu(t)
+    q, k, v, g, beta, gate, S0 = (pick(n) for n in ("q", "k", "v", "g", "beta", "gate", "S0"))
     cu = list(inp["cu_seqlens_host"])
-    if heads is not None:
-        sel = lambda t: None if t is None else t[:, heads].contiguous()
-        q, k, v, g, beta, gate = (sel(t) for t in (q, k, v, g, beta, gate))
-        S0 = None if S0 is None else S0[:, heads].contiguous()
     if seqs is not None:
         rows = torch.cat([torch.arange(cu[n], cu[n + 1]) for n in seqs])
         newcu = [0]
@@ -200,52 +203,91 @@ def test_linearity_in_v_and_S0_fp32():
     assert rel_max(o3, o1 + o2) <= TOL_FP32 and rel_max(S3, S1 + S2) <= TOL_FP32
 
 
-def test_config1_full_size_sampled_units():
-    """B=8, H=32, T=4096, dk=dv=128, bf16 in the bench's launch; two
-    (sequence, head) units checked in full against the oracle, every output
-    checked finite."""
+def _unit_errors(o, S, o_ref, S_ref, cu, heads):
+    """Parity of a full-size output, and its per-(sequence, head) breakdown.
+
+    The stated metric is taken over the whole compared output: o (bf16) --
+    max over all compared elements of |d| beyond half a bf16 ulp, divided by
+    the RMS of all compared reference values; S_T (fp32) likewise, plain.
+    The per-unit figures (each unit's max over that unit's own RMS) are
+    returned for the report.  ``o``/``S`` hold the CUDA results for ``heads``
+    (in that order), ``o_ref``/``S_ref`` the oracle's."""
+    o = o.detach().to("cpu", torch.float64).numpy()
+    S = S.detach().to("cpu", torch.float64).numpy()
+    units = {}
+    dmax_o = dmax_s = 0.0
+    ss_o = ss_s = 0.0
+    cnt_o = cnt_s = 0
+    for n in range(len(cu) - 1):
+        a, b = cu[n], cu[n + 1]
+        for j, h in enumerate(heads):
+            r, x = o_ref[a:b, j], o[a:b, j]
+            rs, xs = S_ref[n, j], S[n, j]
+            do = float(np.max(np.maximum(np.abs(x - r) - bf16_half_ulp(r), 0.0))) if r.size else 0.0
+            ds = float(np.max(np.abs(xs - rs)))
+            so, sst = float(np.sum(r * r)), float(np.sum(rs * rs))
+            dmax_o, dmax_s = max(dmax_o, do), max(dmax_s, ds)
+            ss_o, ss_s, cnt_o, cnt_s = ss_o + so, ss_s + sst, cnt_o + r.size, cnt_s + rs.size
+            units[(n, h)] = (do / np.sqrt(so / r.size) if r.size and so > 0 else do,
+                             ds / np.sqrt(sst / rs.size) if sst > 0 else ds)
+    whole = (dmax_o / np.sqrt(ss_o / cnt_o), dmax_s / np.sqrt(ss_s / cnt_s))
+    return whole, units
+
+
+def _check_units(res, what):
+    (eo, es), units = res
+    worst_o = max(units.items(), key=lambda kv: kv[1][0])
+    worst_s = max(units.items(), key=lambda kv: kv[1][1])
+    print(f"{what}: {len(units)} units; whole output o {eo:.3e}, S_T {es:.3e}; per unit: "
+          f"worst o {worst_o[1][0]:.3e} at {worst_o[0]}, worst S_T {worst_s[1][1]:.3e} at {worst_s[0]}")
+    assert eo <= TOL_BF16 and es <= TOL_BF16, f"{what}: o {eo:.3e}, S_T {es:.3e}"
+
+
+def test_config1_full_size_all_units():
+    """B=8, H=32, T=4096, dk=dv=128, bf16 in the bench's launch: all 256
+    (sequence, head) units against the oracle, each unit's error on its own."""
     inp = inputs.prefill_inputs([4096] * 8, H=32, dk=128, dv=128, device=DEV, seed=0)
     o, S = chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
                      cu_seqlens=inp["cu_seqlens"], cu_seqlens_host=inp["cu_seqlens_host"])
-    assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
-    for n, h in ((0, 0), (7, 31)):
-        o_ref, S_ref = _oracle_prefill(inp, heads=[h], seqs=[n])
-        a, b = n * 4096, (n + 1) * 4096
-        _assert_close(o[a:b, h:h + 1], S[n:n + 1, h:h + 1], o_ref, S_ref, torch.bfloat16,
-                      f"config 1 unit ({n},{h})")
     assert device_status() == 0
+    o_ref, S_ref = _oracle_prefill(inp)
+    _check_units(_unit_errors(o, S, o_ref, S_ref, list(inp["cu_seqlens_host"]), list(range(32))),
+                 "config 1")
 
 
-def test_config2_varlen_full_size_sampled_units():
+def test_config2_varlen_full_size_all_sequences_four_heads():
     """64 packed sequences with lengths uniform in [512, 32768], H=64,
-    dk=dv=128, bf16, S0 ~ N(0, 0.02): the shortest and the longest sequence
-    checked in full on two heads; every output checked finite."""
+    dk=dv=128, bf16, S0 ~ N(0, 0.02): all 64 sequences on 4 seeded heads
+    against the oracle, each (sequence, head) error on its own; every output
+    checked finite."""
     lengths = inputs.varlen_lengths(64, 512, 32768, seed=0)
     inp = inputs.prefill_inputs(lengths, H=64, dk=128, dv=128, device=DEV, seed=0, s0_std=0.02)
     o, S = chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S0=inp["S0"],
                      cu_seqlens=inp["cu_seqlens"], cu_seqlens_host=inp["cu_seqlens_host"])
     assert _all_finite(o) and _all_finite(S)
-    cu = inp["cu_seqlens_host"]
-    seqs = [int(np.argmin(lengths)), int(np.argmax(lengths))]
-    heads = [0, 63]
-    o_ref, S_ref = _oracle_prefill(inp, heads=heads, seqs=seqs)
-    rows = torch.cat([torch.arange(cu[n], cu[n + 1]) for n in seqs]).to(o.device)
-    _assert_close(o[rows][:, heads], S[seqs][:, heads], o_ref, S_ref, torch.bfloat16, "config 2")
     assert device_status() == 0
+    heads = sorted(int(h) for h in np.random.default_rng(2).choice(64, size=4, replace=False))
+    o_ref, S_ref = _oracle_prefill(inp, heads=heads)
+    hsel = torch.tensor(heads, device=o.device)
+    _check_units(_unit_errors(o.index_select(1, hsel), S.index_select(1, hsel), o_ref, S_ref,
+                              list(inp["cu_seqlens_host"]), heads), "config 2")
 
 
-def test_config3_long_context_full_size_sampled_head():
+def test_config3_long_context_full_size_four_heads():
     """B=1, H=32, T=2^20, dk=dv=128, bf16, decay near the floor
-    (g ~ -5 U(0.8, 1)): head 0 checked in full (1M tokens); every output
-    checked finite."""
+    (g ~ -5 U(0.8, 1)): 4 seeded heads checked in full (1M tokens each);
+    every output checked finite."""
     inp = inputs.prefill_inputs([1 << 20], H=32, dk=128, dv=128, device=DEV, seed=0,
                                 g_mode="floor_stress")
     o, S = chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
                      cu_seqlens=inp["cu_seqlens"], cu_seqlens_host=inp["cu_seqlens_host"])
     assert _all_finite(o) and _all_finite(S)
-    o_ref, S_ref = _oracle_prefill(inp, heads=[0])
-    _assert_close(o[:, :1], S[:, :1], o_ref, S_ref, torch.bfloat16, "config 3 head 0")
     assert device_status() == 0
+    heads = sorted(int(h) for h in np.random.default_rng(3).choice(32, size=4, replace=False))
+    o_ref, S_ref = _oracle_prefill(inp, heads=heads)
+    hsel = torch.tensor(heads, device=o.device)
+    _check_units(_unit_errors(o.index_select(1, hsel), S.index_select(1, hsel), o_ref, S_ref,
+                              list(inp["cu_seqlens_host"]), heads), "config 3")
 
 
 def test_config4_decode_full_batch_all_units():

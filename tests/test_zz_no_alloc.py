@@ -1,23 +1,34 @@
-"""kda_chunk_fwd_noalloc, called through the C ABI, against kda_chunk_fwd.
+"""kda_chunk_fwd_noalloc, called through the C ABI, against the fp64 oracle
+and against kda_chunk_fwd.
 
 This entry point serves callers that cannot give the library any device
 memory (a plugin interface that passes only inputs and outputs, a runtime
 that plans all device memory in advance and forbids allocating once it
 runs): its scratch is a fixed array compiled into the library.  The test
 makes two calls in a row with different shapes, so the second one runs on
-scratch the first one left behind, and compares each result with the
-workspace-taking entry point within the parity tolerances.  It is meant to
+scratch the first one left behind, and compares each result with the oracle
+and with the workspace-taking entry point within the parity tolerances; a
+third call goes through the Python wrapper with caller-provided outputs.  It is meant to
 pass on its own in a fresh process (where its first call also performs the
 per-device set-up) and after every other test.  This file is named so that
 pytest collects it last.
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
+import oracle
 from gated_delta_rule_136_b200 import chunk_fwd, device_status, inputs, kda
 from parity import TOL_BF16, rel_max, rel_max_beyond_bf16
+
+
+def _oracle(inp):
+    cpu = lambda t: None if t is None else t.detach().cpu()
+    return oracle.kda_fwd_ref(*(cpu(inp[n]) for n in ("q", "k", "v", "g", "beta")),
+                              cu_seqlens=np.array(inp["cu_seqlens_host"], dtype=np.int64),
+                              S0=cpu(inp["S0"]), scale=inp["scale"], gate=cpu(inp["gate"]))
 
 
 def _call_noalloc(lib, inp, o, S_T):
@@ -53,12 +64,35 @@ def test_noalloc_matches_workspace_entry_point_twice():
         o = torch.empty((T, H, 128), dtype=torch.bfloat16, device="cuda")
         S_T = torch.empty((N, H, 128, 128), dtype=torch.float32, device="cuda")
         assert _call_noalloc(lib, inp, o, S_T) == 0
-        o_ref, S_ref = chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
-                                 S0=inp["S0"], cu_seqlens=inp["cu_seqlens"],
-                                 cu_seqlens_host=inp["cu_seqlens_host"], gate=inp["gate"])
+        o_ws, S_ws = chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                               S0=inp["S0"], cu_seqlens=inp["cu_seqlens"],
+                               cu_seqlens_host=inp["cu_seqlens_host"], gate=inp["gate"])
         torch.cuda.synchronize()
+        o_ref, S_ref = _oracle(inp)
         assert rel_max_beyond_bf16(o, o_ref) <= TOL_BF16
         assert rel_max(S_T, S_ref) <= TOL_BF16
+        assert rel_max_beyond_bf16(o, o_ws) <= TOL_BF16
+        assert rel_max(S_T, S_ws) <= TOL_BF16
+    assert device_status() == 0
+
+
+@pytest.mark.gpu
+def test_noalloc_python_wrapper_with_caller_outputs():
+    """kda.chunk_fwd_noalloc with out= and final_state_out=: the results land in
+    the caller's tensors and match the oracle."""
+    inp = inputs.prefill_inputs([200, 64, 7, 333], H=3, dk=128, dv=128, device="cuda", seed=41,
+                                s0_std=0.02, gate=True)
+    T, H = inp["q"].shape[:2]
+    o = torch.full((T, H, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    S_T = torch.full((4, H, 128, 128), float("nan"), dtype=torch.float32, device="cuda")
+    o2, S2 = kda.chunk_fwd_noalloc(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                                   inp["cu_seqlens"], S0=inp["S0"], gate=inp["gate"],
+                                   out=o, final_state_out=S_T)
+    assert o2 is o and S2 is S_T
+    torch.cuda.synchronize()
+    o_ref, S_ref = _oracle(inp)
+    assert rel_max_beyond_bf16(o, o_ref) <= TOL_BF16
+    assert rel_max(S_T, S_ref) <= TOL_BF16
     assert device_status() == 0
 
 
