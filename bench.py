@@ -553,11 +553,27 @@ def main():
             if device_status(dev) != 0:
                 raise RuntimeError("device error word after speculative decode")
             ms = max_over_ranks(a.elapsed_time(b)) / rounds
+
+            def time_one(fn):   # one call type alone, on the same (cached-out) state
+                a.record(stream)
+                for _ in range(rounds):
+                    fn()
+                b.record(stream)
+                barrier()
+                return max_over_ranks(a.elapsed_time(b)) / rounds
+            ms_v = time_one(lambda: spec_verify(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], Ssp,
+                                                gate=xs["gate"], out=osp))
+            ms_c = time_one(lambda: spec_commit(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], Ssp, accd))
             heads = DEC_B * DEC_H
             byts = heads * (3 * DK * DV * 4 + Dd * (2 * (3 * DK + DV + 1) + 2 * DV + 2 * DV)
                             + 3 * 2 * (3 * DK + DV + 1))
+            byts_v = heads * (DK * DV * 4 + Dd * (2 * (3 * DK + DV + 1) + 2 * DV + 2 * DV))
             others[f"speculative decode batch={DEC_B} H={DEC_H}: verify {Dd} draft tokens, commit 3"] = {
                 "rounds_per_s": world * 1e3 / ms, "ms_per_round": ms,
+                "ms_verify": ms_v, "ms_commit": ms_c,
+                "verify_roofline": {"bound": "hbm", "achieved": byts_v / (ms_v / 1e3) / 1e9,
+                                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                    "frac": byts_v / (ms_v / 1e3) / 1e9 / peaks["hbm_gbs"], "traffic": None},
                 "verified_tokens_per_s": world * DEC_B * Dd / (ms / 1e3),
                 "alg_gbs": byts / (ms / 1e3) / 1e9, "roofline_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
                 "alg_bytes_per_round": byts,

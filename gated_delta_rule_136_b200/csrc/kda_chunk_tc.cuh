@@ -19,9 +19,11 @@
 // in parallel, then the state carried to the next chunk: fupanwang.com digest,
 // section 基础设施, FlashKDA).
 //
-// Precision: the products the outputs are sensitive to run in tf32 (the A_qk /
-// A_kk operands of every block, rounded to nearest, T' (K e^G) S, A_qk Vn,
-// K^(4)^T Vn); T' V, (K e^G) S and (Q e^G) S run in bf16, with S carried as a
+// Precision: the products the outputs are sensitive to run in tf32 or fp16 (the
+// A_qk / A_kk operands: tf32 rounded to nearest on the diagonal 16 x 16 blocks,
+// fp16 -- the same 11-bit significand -- on the off-diagonal ones, whose
+// operands are all at most 1; T' (K e^G) S, A_qk Vn, K^(4)^T Vn in tf32);
+// T' V, (K e^G) S and (Q e^G) S run in bf16, with S carried as a
 // leading bf16 part plus a bf16 low part (each state product issued once per
 // part into the same accumulator).  On the full-size workloads the bf16
 // off-diagonal A operands and the bf16 state were the largest terms of the
@@ -43,6 +45,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include "kda_common.cuh"
 #include "kda_tc.cuh"
@@ -66,7 +69,8 @@ constexpr uint32_t OFF_INTRA = 65536;     // 72 KB, reused after the A MMAs
 //   during prep / A MMAs (per pass of 64 channels):
 constexpr uint32_t OFF_XT = OFF_INTRA;             // X~ [128 rows x 64 ch] tf32 K-major: 2 x 16 KB
 constexpr uint32_t OFF_KD = OFF_INTRA + 32768;     // Kbar [64 rows j x 64 ch] tf32 K-major: 2 x 8 KB
-constexpr uint32_t OFF_KO = OFF_INTRA + 49152;     // K^(b) rows j < 16 b, b = 1..3, tf32 K-major: 24 KB
+constexpr uint32_t OFF_XB = OFF_INTRA + 49152;     // X~ rows 32-127 (blocks 1-3) fp16 K-major: 12 KB
+constexpr uint32_t OFF_KO = OFF_INTRA + 61440;     // K^(b) rows j < 16 b, b = 1..3, fp16 K-major: 12 KB
 //   after the A MMAs:
 constexpr uint32_t OFF_SCR = OFF_INTRA;            // A_kk -> T, fp32 [64][68]
 constexpr uint32_t SCR_LD = 68;                    // 16-byte aligned rows
@@ -92,21 +96,21 @@ constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024; // slack for aligning the bas
 static_assert(OFF_TP % 1024 == 0 && OFF_TP + 16384 <= OFF_XS && OFF_XS + 4096 <= OFF_TPB &&
               OFF_TPB % 1024 == 0 && OFF_TPB + 8192 <= OFF_INTRA + 73728, "post-MMA tiles fit the intra region");
 static_assert((OFF_KG - OFF_QG) % 16 == 0, "Q e^G | K e^G as one MN-major operand");
-static_assert(OFF_KO + 24576 == OFF_INTRA + 73728, "intra tiles fit");
+static_assert(OFF_KO + 12288 == OFF_INTRA + 73728, "intra tiles fit");
 static_assert(SMEM_ALLOC <= 232448, "fits in 227 KB");
 
-// Off-diagonal column operands: tile b (b = 1..3) holds K^(b) rows j < 16 b
-// (tokens of the blocks before b) in tf32, two 128-byte K-blocks of 32
-// channels (16 b rows each, 2 KB x b); tiles are packed back to back.  The MMA
-// (M = 64) reads 64 rows from a K-block's start; rows past the valid ones read
-// neighbouring bytes (the next K-block or tile, or for b = 3 the first 2 KB
-// after the intra region), which only feed accumulator rows that are never
-// used.  The row operand is the tf32 X~ tile of the diagonal product.
-__host__ __device__ constexpr uint32_t ko_base(int b) { return 2048u * (uint32_t)b * (uint32_t)(b - 1); }
-__host__ __device__ constexpr uint32_t ko_kblk(int b) { return 2048u * (uint32_t)b; }
-static_assert(ko_base(1) == 0u && ko_base(2) == 4096u && ko_base(3) == 12288u, "packing");
-static_assert(ko_base(3) + 2u * ko_kblk(3) == 24576u, "tiles fill the region");
-static_assert(OFF_KO + ko_base(3) + ko_kblk(3) + 64u * 128u <= OFF_QG + 16384u, "K^(b) reads stay in shared memory");
+// Off-diagonal operands, fp16: tile b (b = 1..3) holds K^(b) rows j < 16 b
+// (tokens of the blocks before b), one 128-byte K-block of 64 channels; tiles
+// are packed back to back.  The row operand is an fp16 copy of X~ rows of
+// blocks 1-3.  Every value is at most |q| or |k| (<= 1: the decays only shrink
+// it), so fp16 holds it without overflow, with tf32's 11-bit significand; a
+// value below fp16's range is below 6e-8 and so is its every product.  The
+// MMA (M = 64) reads 64 rows from a tile's start; rows past the valid ones
+// read neighbouring bytes (the next tile, or for b = 3 the first 2 KB after
+// the intra region), which only feed accumulator rows that are never used.
+__host__ __device__ constexpr uint32_t ko_base(int b) { return 1024u * (uint32_t)b * (uint32_t)(b - 1); }
+static_assert(ko_base(1) == 0u && ko_base(2) == 2048u && ko_base(3) == 6144u, "packing");
+static_assert(OFF_KO + ko_base(3) + 64u * 128u <= OFF_QG + 16384u, "K^(b) reads stay in shared memory");
 
 // ---- TMEM columns
 constexpr uint32_t T_DD = 0;      // diagonal A MMA [64 j x 128 X~ rows] (M = 64 layout)
@@ -158,6 +162,12 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t kbyte) {
 // pipe: adding half a tf32 ulp to the magnitude bits and truncating the low
 // 13 bits gives that rounding for every finite value (a carry into the
 // exponent is the correct round-up).
+// two fp32 -> one 32-bit word of fp16 (round to nearest even), lo in the low half
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    const __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
 __device__ __forceinline__ float to_tf32(float x) {
     return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 }
@@ -336,6 +346,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t sw_lane = ((((kbyte >> 4) & 7u) ^ (uint32_t)gq) << 4) + (kbyte & 15u);
     const uint32_t xt_lane = OFF_XT + kblk * 16384u + sw_lane;
     const uint32_t kd_lane = OFF_KD + kblk * 8192u + sw_lane;
+    // the same for the fp16 tiles (one 128-byte K-block of 64 channels)
+    const uint32_t xb_lane = OFF_XB + (((((uint32_t)cA * 2u) >> 4) ^ (uint32_t)gq) << 4) + (((uint32_t)cA * 2u) & 15u);
     // constant A fragments of the prefix-sum products (bf16 1.0 = 0x3F80):
     //   a_blk: 16x16 lower triangle with diagonal;  a_ref[kb]: rows m < 4 select block kb <= m
     uint32_t a_blk[4];
@@ -464,7 +476,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     // MMA descriptors that do not depend on the chunk (start addresses advance per K-step)
     const uint32_t id_d = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 64, 128);
-    const uint32_t id_o = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 64, 32);
+    const uint32_t id_o = instr_desc(FMT_F16, K_MAJOR, K_MAJOR, 64, 32);
     const uint32_t id_1 = instr_desc(FMT_BF16, K_MAJOR, MN_MAJOR, 128, 128);
     const uint32_t id_vn = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 128, 64);
     const uint32_t id_u = instr_desc(FMT_BF16, MN_MAJOR, K_MAJOR, 128, 64);
@@ -480,13 +492,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     //           channels (tf32, M = 64, N = 128: every block against every
     //           block, of which the diagonal 16 x 32 tiles are used), and the
     //           off-diagonal product of block 1;
-    //   part 1: the off-diagonal products of blocks 2 and 3 (tf32, M = 64, N = 32:
+    //   part 1: the off-diagonal products of blocks 2 and 3 (fp16, M = 64, N = 32:
     //           K^(b) rows j < 16 b against X~ rows of block b); then commit, and
     //           this pass's half of [O1 | -Y]^T = S^T [Q e^G | -K e^G]^T (bf16, A =
     //           S^T from TMEM), which runs behind the A MMAs, off the critical path.
     auto issue_a = [&](int pass_, int part) {
         if (part == 0) {
-#pragma unroll
+#pragma unroll 1
             for (int s = 0; s < 8; ++s) {          // tf32 K-steps of 8 channels
                 const uint32_t kb = (uint32_t)(s >> 2), koff = (uint32_t)(s & 3) * 32u;
                 if (leader) mma_tf32_ss(tbase + T_DD, at(d_k16, OFF_KD + kb * 8192u + koff),
@@ -497,17 +509,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int bo = 1; bo < NB; ++bo) {
             if ((bo == 1) != (part == 0)) continue;
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {          // tf32 K-steps of 8 channels
-                const uint32_t kb = (uint32_t)(s >> 2), koff = (uint32_t)(s & 3) * 32u;
-                if (leader) mma_tf32_ss(tbase + T_DO + 32u * (bo - 1),
-                                        at(d_k16, OFF_KO + ko_base(bo) + kb * ko_kblk(bo) + koff),
-                                        at(d_k16, OFF_XT + kb * 16384u + 32u * (uint32_t)bo * 128u + koff), id_o,
+            for (int s = 0; s < 4; ++s)            // fp16 K-steps of 16 channels
+                if (leader) mma_bf16_ss(tbase + T_DO + 32u * (bo - 1), at(d_k16, OFF_KO + ko_base(bo) + 32u * s),
+                                        at(d_k16, OFF_XB + 32u * (bo - 1) * 128u + 32u * s), id_o,
                                         (pass_ > 0 || s > 0) ? 1u : 0u);
-            }
         }
         if (part == 1) {
             if (leader) mma_commit(bar_mma);
-#pragma unroll
+#pragma unroll 1
             for (int s = 0; s < 4; ++s) {
                 const uint32_t ks = (uint32_t)(4 * pass_ + s);   // K = 128 key channels in steps of 16
                 if (leader) mma_bf16_ts(tbase + T_O1, tbase + T_S + 8u * ks, at(d_qk, OFF_QG + 2048u * ks), id_1, ks > 0);
@@ -696,9 +705,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     ++mma_phase;
                     tc_fence_after();
                 }
-                // (4) the A-MMA operands, rounded to tf32: X~ rows (q~ at 32 b + r, k~ at
-                //     32 b + 16 + r) and Kbar for the diagonal product, and the K^(b') copies,
-                //     b' > b, for the off-diagonal products (whose rows are the same X~)
+                // (4) the A-MMA operands: X~ rows (q~ at 32 b + r, k~ at 32 b + 16 + r) and
+                //     Kbar for the diagonal product (tf32, rounded), X~ rows of blocks 1-3
+                //     again in fp16 and the K^(b') copies, b' > b, in fp16 for the
+                //     off-diagonal products
 #pragma unroll
                 for (int bb = 0; bb < 2; ++bb) {
                     const int b = 2 * mp + bb;
@@ -719,12 +729,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         *reinterpret_cast<float2 *>(sm + xt_lane + xrow * 128u) = rnd2(qt[bb][hr]);
                         *reinterpret_cast<float2 *>(sm + xt_lane + (xrow + 16u) * 128u) = rnd2(kt[bb][hr]);
                         *reinterpret_cast<float2 *>(sm + kd_lane + i * 128u) = rnd2(kbar[bb][hr]);
+                        if (b > 0) {
+                            *reinterpret_cast<uint32_t *>(sm + xb_lane + (xrow - 32u) * 128u) = pack_f16(qt[bb][hr].x, qt[bb][hr].y);
+                            *reinterpret_cast<uint32_t *>(sm + xb_lane + (xrow - 16u) * 128u) = pack_f16(kt[bb][hr].x, kt[bb][hr].y);
+                        }
 #pragma unroll
                         for (int m = 1; m < NB; ++m) {
                             if (m <= b) continue;
                             const float2 v = __fmul2_rn(kbar[bb][hr], dfac[m]);
-                            *reinterpret_cast<float2 *>(sm + OFF_KO + ko_base(m) + kblk * ko_kblk(m) + sw_lane + i * 128u) =
-                                rnd2(v);
+                            *reinterpret_cast<uint32_t *>(sm + xb_lane - OFF_XB + OFF_KO + ko_base(m) + i * 128u) = pack_f16(v.x, v.y);
                         }
                     }
                 }
