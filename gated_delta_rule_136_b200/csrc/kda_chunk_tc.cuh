@@ -493,9 +493,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     //           block, of which the diagonal 16 x 32 tiles are used), and the
     //           off-diagonal product of block 1;
     //   part 1: the off-diagonal products of blocks 2 and 3 (fp16, M = 64, N = 32:
-    //           K^(b) rows j < 16 b against X~ rows of block b); then commit, and
-    //           this pass's half of [O1 | -Y]^T = S^T [Q e^G | -K e^G]^T (bf16, A =
-    //           S^T from TMEM), which runs behind the A MMAs, off the critical path.
+    //           K^(b) rows j < 16 b against X~ rows of block b); then commit.
     auto issue_a = [&](int pass_, int part) {
         if (part == 0) {
 #pragma unroll 1
@@ -514,16 +512,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                         at(d_k16, OFF_XB + 32u * (bo - 1) * 128u + 32u * s), id_o,
                                         (pass_ > 0 || s > 0) ? 1u : 0u);
         }
-        if (part == 1) {
-            if (leader) mma_commit(bar_mma);
-#pragma unroll 1
-            for (int s = 0; s < 4; ++s) {
-                const uint32_t ks = (uint32_t)(4 * pass_ + s);   // K = 128 key channels in steps of 16
-                if (leader) mma_bf16_ts(tbase + T_O1, tbase + T_S + 8u * ks, at(d_qk, OFF_QG + 2048u * ks), id_1, ks > 0);
-                if (leader) mma_bf16_ts(tbase + T_O1, tbase + T_LO + 8u * ks, at(d_qk, OFF_QG + 2048u * ks), id_1, 1u);
-            }
-            if (pass_ == 1 && leader) mma_commit(bar_y);
-        }
+        if (part == 1 && leader) mma_commit(bar_mma);
     };
 
     const float L2E = 1.4426950408889634f;
@@ -862,6 +851,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
         bool z_ok = true;
         ++y_issued;
+        // [O1 | -Y]^T = S^T [Q e^G | -K e^G]^T (bf16, A = S^T from TMEM as its leading and
+        // low parts), issued by warp 8 while warps 0-3 run the inverse: the tensor pipe
+        // is idle then, and no prep warp waits on the issue
+        if (warp == 8) {
+#pragma unroll 1
+            for (int ks = 0; ks < 8; ++ks) {       // K = 128 key channels in steps of 16
+                if (leader) mma_bf16_ts(tbase + T_O1, tbase + T_S + 8u * (uint32_t)ks,
+                                        at(d_qk, OFF_QG + 2048u * (uint32_t)ks), id_1, ks > 0);
+                if (leader) mma_bf16_ts(tbase + T_O1, tbase + T_LO + 8u * (uint32_t)ks,
+                                        at(d_qk, OFF_QG + 2048u * (uint32_t)ks), id_1, 1u);
+            }
+            if (leader) mma_commit(bar_y);
+            __syncwarp();
+        }
         // ================================================= T = (I + A_kk)^-1, then T' = T Diag(beta) (warps 0-3)
         // Blocked inverse of the unit lower-triangular 64x64 matrix: 16x16
         // diagonal blocks by forward substitution, then the block merges
