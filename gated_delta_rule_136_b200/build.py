@@ -20,6 +20,11 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(PKG, "_build")
 LIB_NAME = "libkda_b200.so"
 LIB_PATH = os.path.join(BUILD_DIR, LIB_NAME)
+# The debug variant: the same sources with -DKDA_DEBUG, whose kernels check
+# each unit's token range, sequence and head on the device and record
+# KDA_ERR_DEVICE_BOUNDS instead of touching memory outside them.  The binding
+# loads it when the environment sets KDA_DEBUG_LIBRARY=1.
+DEBUG_LIB_PATH = os.path.join(BUILD_DIR, "libkda_b200_debug.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -46,23 +51,27 @@ def is_stale(path: str = LIB_PATH) -> bool:
     return any(os.path.getmtime(d) > t for d in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    """Compile every ``csrc/*.cu`` into one shared library; returns its path."""
-    if not force and not is_stale():
-        return LIB_PATH
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
+          debug: bool = False) -> str:
+    """Compile every ``csrc/*.cu`` into one shared library; returns its path
+    (``debug``: the variant with device-side argument checks)."""
+    path = DEBUG_LIB_PATH if debug else LIB_PATH
+    if not force and not is_stale(path):
+        return path
     os.makedirs(BUILD_DIR, exist_ok=True)
-    tmp = LIB_PATH + f".tmp{os.getpid()}"
+    tmp = path + f".tmp{os.getpid()}"
     cmd = [_nvcc(), *ARCH, "-O3", "-std=c++17", "-lineinfo", "-shared",
-           "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
+           "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr", *(["-DKDA_DEBUG"] if debug else []),
            "-I", INCLUDE, "-I", CSRC, *sources(), "-o", tmp]
     if ptxas_info:
         cmd[1:1] = ["-Xptxas", "-v"]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, path)
+    return path
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True, ptxas_info="--ptxas-info" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose=True, ptxas_info="--ptxas-info" in sys.argv,
+                debug="--debug" in sys.argv))

@@ -63,6 +63,8 @@ struct SimtParams {
     int32_t num_heads;
     float scale, g_floor;
     SnapOut snap;
+    int64_t total_tokens;       // extents, for the debug build's unit checks
+    int32_t num_seqs;
 };
 
 template <int DK, int DV, typename TIO>
@@ -88,8 +90,16 @@ __global__ void __launch_bounds__(2 * DV, 1) chunk_simt_kernel(SimtParams p)
     const int n_slot = blockIdx.x / H;
     const int h = blockIdx.x % H;
     const int n = p.seq_order ? p.seq_order[n_slot] : n_slot;
+    if (kDebugChecks && (n < 0 || n >= p.num_seqs)) {   // (uniform over the CTA)
+        if (tid == 0) raise_error(ERR_BOUNDS);
+        return;
+    }
     const int64_t t_begin = p.cu_seqlens[n];
     const int64_t t_end = p.cu_seqlens[n + 1];
+    if (kDebugChecks && (t_begin < 0 || t_end < t_begin || t_end > p.total_tokens)) {
+        if (tid == 0) raise_error(ERR_BOUNDS);
+        return;
+    }
     const int64_t unit = (int64_t)n * H + h;
 
     float S[RH];

@@ -151,6 +151,8 @@ struct TcParams {
     float scale, g_floor;
     const TcUnit *units;   // when set, block b runs units[b] instead of a (sequence, head)
     SnapOut snap;          // state snapshots (units with UNIT_STORE_O only)
+    int64_t total_tokens;  // extents, for the debug build's unit checks
+    int32_t num_seqs;
 };
 
 // byte offset of (row, byte kb within a 128-byte K-block row) in a swizzled block
@@ -313,12 +315,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int n_slot = blockIdx.x / H;
         hh = blockIdx.x % H;
         const int n = p.seq_order ? p.seq_order[n_slot] : n_slot;
+        if (kDebugChecks && (n < 0 || n >= p.num_seqs)) {
+            if (tid == 0) raise_error(ERR_BOUNDS);
+            return;
+        }
         t_begin = p.cu_seqlens[n]; t_end = p.cu_seqlens[n + 1];
         const int64_t unit = (int64_t)n * H + hh;
         S0p = p.S0 ? p.S0 + unit * D * D : nullptr;
         S_outp = p.S_T ? p.S_T + unit * D * D : nullptr;
         flags = UNIT_STORE_O;
         snap_n = n; seq_start = t_begin;
+    }
+    if (kDebugChecks) {   // the unit must lie inside the launch's extents
+        const bool bad = t_begin < 0 || t_end < t_begin || t_end > p.total_tokens || hh < 0 || hh >= H ||
+                         snap_n < 0 || snap_n >= p.num_seqs;
+        if (bad) {
+            if (tid == 0) raise_error(ERR_BOUNDS);
+            return;                      // (uniform over the CTA, before any shared or TMEM state)
+        }
     }
     const bool store_o = (flags & UNIT_STORE_O) != 0;
     const bool zero_v = (flags & UNIT_ZERO_V) != 0;

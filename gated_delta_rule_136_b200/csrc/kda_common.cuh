@@ -15,6 +15,17 @@ enum : unsigned int { ERR_TIMEOUT = 1u, ERR_BOUNDS = 2u };
 
 __device__ __forceinline__ void raise_error(unsigned int bit) { atomicOr(&g_err_word, bit); }
 
+// Device-side argument checks of the debug build (-DKDA_DEBUG, built as
+// libkda_b200_debug.so): a kernel checks the token range, sequence and head
+// of its unit before touching memory; a bad one records ERR_BOUNDS and the
+// unit is skipped (never a trap: the error word is read by
+// kda_get_device_status).  In the release build the checks compile away.
+#ifdef KDA_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+
 // Element loads/stores for the two I/O dtypes.
 __device__ __forceinline__ float ld(const float *p, int64_t i) { return p[i]; }
 __device__ __forceinline__ float ld(const __nv_bfloat16 *p, int64_t i) { return __bfloat162float(p[i]); }

@@ -305,11 +305,11 @@ cudaError_t launch_prefill(const kda_fwd_desc &d, const void *q, const void *k, 
                            void *o, float *S_T, const kda::SnapOut &sn, cudaStream_t stream) {
     if (tc_path_applies(d, q, k, v, g, o)) {
         kda::tck::TcParams tp{beta, gate, S0, cu_seqlens, seq_order, o, S_T, d.num_heads, d.scale,
-                              d.g_floor, nullptr, sn};
+                              d.g_floor, nullptr, sn, d.total_tokens, d.num_seqs};
         return launch_tc(d, q, k, v, g, tp, stream);
     }
     SimtParams p{q, k, v, g, beta, gate, S0, cu_seqlens, seq_order, o, S_T,
-                 d.num_heads, d.scale, d.g_floor, sn};
+                 d.num_heads, d.scale, d.g_floor, sn, d.total_tokens, d.num_seqs};
     return d.io_dtype == KDA_BF16 ? dispatch_simt<__nv_bfloat16>(d.dk, d.dv, p, d.num_seqs, stream)
                                   : dispatch_simt<float>(d.dk, d.dv, p, d.num_seqs, stream);
 }
@@ -375,7 +375,8 @@ cudaError_t launch_split(const kda_fwd_desc &d, const SegPlan &pl, const int32_t
     if ((e = cudaMemcpyAsync(dj, jobs.data(), jobs.size() * sizeof(kda::ScanJob), cudaMemcpyHostToDevice,
                              stream)) != cudaSuccess)
         return e;
-    kda::tck::TcParams tp{beta, gate, nullptr, nullptr, nullptr, o, nullptr, H, d.scale, d.g_floor, d1, sn};
+    kda::tck::TcParams tp{beta, gate, nullptr, nullptr, nullptr, o, nullptr, H, d.scale, d.g_floor, d1, sn,
+                          d.total_tokens, d.num_seqs};
     if (!p1.empty()) {
         tp.units = d1;
         NvtxRange r("kda.split.pass1");
@@ -913,7 +914,7 @@ kda_status kda_segment_summary(const kda_fwd_desc *desc, const void *q, const vo
                         stream) != cudaSuccess)
         return KDA_ERR_CUDA;
     kda::tck::TcParams tp{beta, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, H, d.scale,
-                          d.g_floor, du, kda::SnapOut{nullptr, nullptr, 0, 64}};
+                          d.g_floor, du, kda::SnapOut{nullptr, nullptr, 0, 64}, d.total_tokens, d.num_seqs};
     {
         NvtxRange r("kda.summary.chains");
         if (launch_tc_units(d, q, k, v, g, tp, (int64_t)units.size(), stream) != cudaSuccess) return KDA_ERR_CUDA;

@@ -9,6 +9,7 @@ fallback, and a missing library or GPU raises.
 from __future__ import annotations
 
 import ctypes
+import os
 import itertools
 import math
 import threading
@@ -79,17 +80,24 @@ _lib = None
 _lock = threading.Lock()
 
 
+def _debug_library() -> bool:
+    return os.environ.get("KDA_DEBUG_LIBRARY", "") not in ("", "0")
+
+
 def library_path() -> str:
-    return _build.LIB_PATH
+    return _build.DEBUG_LIB_PATH if _debug_library() else _build.LIB_PATH
 
 
 def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
-    """Load (building first if missing or stale) the KDA shared library."""
+    """Load (building first if missing or stale) the KDA shared library; with
+    KDA_DEBUG_LIBRARY=1 in the environment, its debug variant (device-side
+    argument checks)."""
     global _lib
     with _lock:
         if _lib is not None:
             return _lib
-        path = _build.build() if build_if_missing else _build.LIB_PATH
+        debug = _debug_library()
+        path = _build.build(debug=debug) if build_if_missing else library_path()
         lib = ctypes.CDLL(path)
         vp, sz, i32p = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(ctypes.c_int32)
         lib.kda_chunk_fwd_workspace_size.argtypes = [ctypes.POINTER(FwdDesc), i32p]
