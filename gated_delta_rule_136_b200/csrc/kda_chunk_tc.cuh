@@ -80,17 +80,17 @@ constexpr uint32_t XS_LD = 8;
 constexpr uint32_t OFF_TPB = OFF_INTRA + 37888;    // T' bf16 K-major [64 i x 64 j]: 8 KB
 constexpr uint32_t OFF_QG = OFF_INTRA + 73728;     // Q e^G bf16 MN-major [128 c x 64 i]: 16 KB
 constexpr uint32_t OFF_KG = OFF_QG + 16384;        // K e^G bf16 K-major [128 c x 64 j]: 16 KB
-// B operand of the second state MMA: rows 0-63 = A_qk [i x j], rows 64-191 =
-// K^(4)^T [c x j]; tf32 K-major with two 128-byte K-blocks of 192 rows each
+// B operand of the second state MMA: rows 0-63 = 2^8 A_qk [i x j], rows 64-191
+// = 2^8 K^(4)^T [c x j]; fp16 K-major, one 128-byte K-block of 64 tokens (its A
+// operand is 2^-8 Vn^T in fp16: the scales cancel exactly, and fp16 keeps
+// tf32's 11-bit significand for these values, |A_qk| and |K^| being at most 1)
 constexpr uint32_t OFF_AK = OFF_KG + 16384;
-constexpr uint32_t AK_KBLK = 192u * 128u;          // 24 KB per K-block
-constexpr uint32_t OFF_AQK = OFF_AK;               // + kb * AK_KBLK + row * 128
-// Between the second state MMA and the next A readout the A_qk rows are free:
-// the output tile waits there for its TMA store, bf16 [64 tokens x 64 v] per
-// K-block (v in [0, 64) at OFF_AK, [64, 128) at OFF_AK + AK_KBLK).
-constexpr uint32_t OFF_OST = OFF_AK;
-constexpr uint32_t OFF_KHT = OFF_AK + 64u * 128u;  // + kb * AK_KBLK + row * 128
-constexpr uint32_t OFF_SMALL = OFF_AK + 2u * AK_KBLK;  // beta[64], gamma[2][128], barriers, tmem base
+constexpr uint32_t OFF_AQK = OFF_AK;               // + row * 128
+constexpr uint32_t OFF_KHT = OFF_AK + 64u * 128u;  // + row * 128
+// The output tile waits here for its TMA store, bf16 [64 tokens x 64 v] per
+// half (v in [0, 64), then [64, 128)).
+constexpr uint32_t OFF_OST = OFF_AK + 192u * 128u;
+constexpr uint32_t OFF_SMALL = OFF_OST + 2u * 8192u;   // beta[64], gamma[2][128], barriers, tmem base
 constexpr uint32_t SMEM_BYTES = OFF_SMALL + 2048;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024; // slack for aligning the base
 static_assert(OFF_TP % 1024 == 0 && OFF_TP + 16384 <= OFF_XS && OFF_XS + 4096 <= OFF_TPB &&
@@ -117,11 +117,12 @@ constexpr uint32_t T_DD = 0;      // diagonal A MMA [64 j x 128 X~ rows] (M = 64
 constexpr uint32_t T_DO = 128;    // off-diagonal A MMAs: 3 x 32 columns (blocks 1-3)
 constexpr uint32_t T_O2 = 0;      // (A_qk Vn)^T   [v x i]   } one MMA (N = 192), after the
 constexpr uint32_t T_DS = 64;     // dS^T          [v x c]   } A readout and Vn
-constexpr uint32_t T_VN = 192;    // Vn^T = V^T T'^T - Y^T T'^T, then its tf32 copy (A operand)
+constexpr uint32_t T_VN = 192;    // Vn^T = V^T T'^T - Y^T T'^T (fp32; its fp16 copy goes to T_LO)
 constexpr uint32_t T_O1 = 256;    // ((Q e^G) S)^T  [v x i]  } one MMA (N = 128)
 constexpr uint32_t T_Z = 320;     // -((K e^G) S)^T  [v x j] (read as a tf32 A operand)
 constexpr uint32_t T_S = 384;     // S^T bf16 A operand (2 per column): the leading bf16 part
-constexpr uint32_t T_LO = 448;    // S^T - bf16(S^T) in bf16: the low part of the same operand
+constexpr uint32_t T_LO = 448;    // S^T - bf16(S^T) in bf16, the low part of the same operand; then,
+                                  // its MMAs done, 2^-8 Vn^T in fp16 (32 columns: two tokens each)
 constexpr uint32_t TMEM_COLS = 512;
 
 // One explicit work unit (used by the long-sequence segment split): a token
@@ -168,6 +169,13 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t kbyte) {
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
     const __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+          "r"(r[7]) : "memory");
 }
 
 __device__ __forceinline__ float to_tf32(float x) {
@@ -463,7 +471,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     auto store_o_tile = [&]() {            // tid 0; the staging tile is complete and fenced
         const int x = hh * D;
         tma_store_2d(&tm_o, smb + OFF_OST, x, (int)o_row);
-        tma_store_2d(&tm_o, smb + OFF_OST + AK_KBLK, x + 64, (int)o_row);
+        tma_store_2d(&tm_o, smb + OFF_OST + 8192u, x + 64, (int)o_row);
         bulk_commit();
     };
     // beta of the next chunk, loaded one chunk ahead (64 strided values)
@@ -494,7 +502,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t id_1 = instr_desc(FMT_BF16, K_MAJOR, MN_MAJOR, 128, 128);
     const uint32_t id_vn = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 128, 64);
     const uint32_t id_u = instr_desc(FMT_BF16, MN_MAJOR, K_MAJOR, 128, 64);
-    const uint32_t id_2 = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 128, 192);
+    const uint32_t id_2 = instr_desc(FMT_F16, K_MAJOR, K_MAJOR, 128, 192);
     const uint64_t d_k16 = smem_desc_sw128(smb, 16, 1024);          // K-major template
     const uint64_t d_qk = smem_desc_sw128(smb, OFF_KG - OFF_QG, 1024);  // [Q e^G | -K e^G] MN-major
     const uint64_t d_mnv = smem_desc_sw128(smb, 8192, 1024);             // v: MN blocks 8 KB apart
@@ -543,9 +551,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int b = 2 * mp + bb;
         const uint32_t i = (uint32_t)(16 * b + 8 * hr + gq);
         const uint32_t cg = (uint32_t)(pass_ * 64 + cA);
-        const uint32_t kho = OFF_KHT + (i >> 5) * AK_KBLK;
-        *reinterpret_cast<float *>(sm + kho + sw128(cg, (i & 31u) * 4u)) = khv[bb][hr].x;
-        *reinterpret_cast<float *>(sm + kho + sw128(cg + 1u, (i & 31u) * 4u)) = khv[bb][hr].y;
+        *reinterpret_cast<__half *>(sm + OFF_KHT + sw128(cg, i * 2u)) = __float2half_rn(khv[bb][hr].x);
+        *reinterpret_cast<__half *>(sm + OFF_KHT + sw128(cg + 1u, i * 2u)) = __float2half_rn(khv[bb][hr].y);
     };
 #pragma unroll 1
     for (int st = 0; st <= 2 * nchunks && !failed; ++st) {
@@ -692,7 +699,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         // K^(4)^T [c x j] tf32: two channels of token i; on the first pass the
                         // previous chunk's last MMA may still read these rows: stored later
                         const float2 kh = __fmul2_rn(kbar[bb][hr], eK);
-                        khv[bb][hr] = make_float2(to_tf32(kh.x), to_tf32(kh.y));
+                        khv[bb][hr] = make_float2(kh.x * 256.0f, kh.y * 256.0f);   // 2^8 K^, as fp16
                         if (pass == 1) store_khat(1, bb, hr);
                     }
                     // Q e^G and -K e^G (bf16 [c x i], tokens contiguous): transposing matrix stores
@@ -790,7 +797,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         }
                         if (Lp == C) {
                             // full chunk: into the staging tile, stored by TMA after the next block barrier
-                            unsigned char *ost = sm + OFF_OST + (uint32_t)(vlane >> 6) * AK_KBLK;
+                            unsigned char *ost = sm + OFF_OST + (uint32_t)(vlane >> 6) * 8192u;
                             const uint32_t vb = (uint32_t)(vlane & 63) * 2u;
 #pragma unroll
                             for (int e = 0; e < 16; ++e)
@@ -847,14 +854,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tmem_wait_ld();
             if (lane < 16) {
                 const int j = lq * 16 + lane;
-                const uint32_t kbj = (uint32_t)j * 4u;
-                unsigned char *aqk = sm + OFF_AQK + (kbj >> 7) * AK_KBLK;
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int i = 16 * cq + e;
                     const float aq = j <= i ? __uint_as_float(ra[e]) : 0.0f;
                     const float ak = j < i ? s_beta[i] * __uint_as_float(rk[e]) : 0.0f;
-                    *reinterpret_cast<float *>(aqk + sw128(i, kbj & 127u)) = to_tf32(aq);
+                    *reinterpret_cast<__half *>(sm + OFF_AQK + sw128(i, (uint32_t)j * 2u)) = __float2half_rn(aq * 256.0f);
                     scr[i * SCR_LD + j] = ak;
                 }
             }
@@ -1019,7 +1024,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!__syncthreads_and(z_ok)) { failed = true; break; }
         tc_fence_after();
 
-        // ================================================= Vn^T = V^T T'^T + (-Y)^T T'^T, then rounded to tf32
+        // ================================================= Vn^T = V^T T'^T + (-Y)^T T'^T, then 2^-8 Vn^T in fp16
         // (bf16 with v as the MN-major A operand from its TMA tile, then tf32 with
         // -Y^T from TMEM, into one accumulator)
         ++mma_issued;
@@ -1042,27 +1047,27 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (tid == 0) issue_loads(ci + 1, 4);
             note_loads(4);
         }
-        {
-            uint32_t rv[16];
+        {   // 2^-8 Vn^T in fp16, two tokens per column, over the state's low part (whose
+            // MMAs completed before the V_new MMAs)
+            uint32_t rv[16], ph[8];
             tmem_ld16(tbase + lane_base + T_VN + cq * 16, rv);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) rv[e] = __float_as_uint(to_tf32(__uint_as_float(rv[e])));
-            tmem_st16(tbase + lane_base + T_VN + cq * 16, rv);
+            for (int e = 0; e < 8; ++e)
+                ph[e] = pack_f16(__uint_as_float(rv[2 * e]) * 0.00390625f, __uint_as_float(rv[2 * e + 1]) * 0.00390625f);
+            tmem_st8(tbase + lane_base + T_LO + cq * 8, ph);
             tmem_wait_st();
         }
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
 
-        // ================================================= O2^T = Vn^T A_qk^T, dS^T = Vn^T K^(4) (tf32)
+        // ================================================= O2^T = Vn^T A_qk^T, dS^T = Vn^T K^(4) (fp16, scales 2^-8 x 2^8)
         ++mma_issued;
         if (warp == 0) {
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {          // K = 64 tokens in steps of 8
-                const uint32_t kb = (uint32_t)(s >> 2), koff = (uint32_t)(s & 3) * 32u;
-                if (leader) mma_tf32_ts(tbase + T_O2, tbase + T_VN + 8u * s, at(d_k16, OFF_AK + kb * AK_KBLK + koff), id_2, s > 0);
-            }
+            for (int s = 0; s < 4; ++s)            // K = 64 tokens in steps of 16
+                if (leader) mma_bf16_ts(tbase + T_O2, tbase + T_LO + 8u * s, at(d_k16, OFF_AK + 32u * s), id_2, s > 0);
             if (leader) mma_commit(bar_mma);
         }
     }

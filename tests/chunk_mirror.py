@@ -30,15 +30,16 @@ The 16-token blocks are where the per-step floor matters: within a block
 every factor is bounded by e^{-16 floor}, inside bf16/fp32 range for floor >= -5.45
 (fupanwang.com Kimi K3 report digest, KDA section, Fig. 3).
 
-``prec`` (a dict operand -> "bf16" | "tf32" | "tf32t" | "fp16" | "bf16x2" | "tf32x2")
+``prec`` (a dict operand -> "bf16" | "tf32" | "tf32t" | "fp16" | "fp16x256" |
+"fp16d256" | "bf16x2" | "tf32x2")
 rounds the tensor-core operands the way a kernel stores them ("tf32t": fp32
 stored whole, the MMA reading only its leading 19 bits, i.e. truncation;
 "...x2": a leading part plus a low part in that type, the product issued once
 per part); ``KERNEL_PREC`` with ``KERNEL_FORM`` is the plan of the tcgen05
 kernel: tf32 for the operands the output is sensitive to (the diagonal A
-operands, A_qk, T', Z, V_new, K^), fp16 (the same 11-bit significand) for the
-off-diagonal A operands, the state as two bf16 parts, bf16 for
-Q e^G / K e^G and T' in T' V.  beta is folded into the columns of T
+operands, T', Z), fp16 (the same 11-bit significand) for the off-diagonal A
+operands and for the last product (2^8 A_qk, 2^8 K^ and 2^-8 V_new), the state
+as two bf16 parts, bf16 for Q e^G / K e^G and T' in T' V.  beta is folded into the columns of T
 (T' = T Diag(beta)).
 """
 from __future__ import annotations
@@ -87,7 +88,14 @@ def _fp16(x):
     return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
 
 
+def _fp16_scaled(scale):
+    """fp16 storage of scale * x (a power of two), read back as x: the scale moves
+    the values away from fp16's subnormal and overflow ranges."""
+    return lambda x: _fp16(np.asarray(x, np.float64) * scale) / scale
+
+
 _ROUND = {"bf16": _bf16, "tf32": _tf32, "tf32t": _tf32_trunc, "fp16": _fp16,
+          "fp16x256": _fp16_scaled(256.0), "fp16d256": _fp16_scaled(1.0 / 256.0),
           "bf16x2": _split2(_bf16), "tf32x2": _split2(_tf32),
           "fp32": lambda x: np.asarray(x, np.float32).astype(np.float64)}
 
@@ -95,7 +103,8 @@ _ROUND = {"bf16": _bf16, "tf32": _tf32, "tf32t": _tf32_trunc, "fp16": _fp16,
 KERNEL_PREC = {
     "Arow": "tf32", "Acol": "tf32",       # q~, k~ and Kbar of the diagonal A blocks (rounded)
     "Aoff": "fp16",                       # q~, k~ and K^(b) of the off-diagonal A blocks (all <= 1)
-    "Aqk": "tf32", "T": "tf32t", "TV": "bf16", "Y": "tf32t", "Vn": "tf32", "Khat": "tf32",
+    "T": "tf32t", "TV": "bf16", "Y": "tf32t",
+    "Aqk": "fp16x256", "Khat": "fp16x256", "Vn": "fp16d256",   # the last MMA: fp16, scales 2^8 / 2^-8
     "KG": "bf16", "S": "bf16x2", "QG": "bf16",
 }
 KERNEL_FORM = "split"
