@@ -1,0 +1,687 @@
+// kda_bwd_chunk.cuh -- KDA backward in the chunked form (dk = dv = 128).
+//
+// The forward of one 64-token chunk with start state S0, in the chunk's frame
+// (Kimi K3 report digest, section "KDA": per-channel decay with a floor,
+// delta-rule write, sigmoid output gate):
+//   lG_t = sum_{s<=t} max(g_s, floor),  lgam = lG_63
+//   Qbar = q e^{lG}, Kbar = k e^{lG}, Khat = k e^{lgam - lG}
+//   A_qk[i][j] = sum_c q_ic k_jc e^{lG_ic - lG_jc} (j <= i),  At the same with k_i (j < i)
+//   T = (I + Diag(beta) At)^-1,  Z = V - Kbar S0,  nu = T Diag(beta) Z
+//   Oraw = scale (Qbar S0 + A_qk nu),  o = Oraw sigmoid(z),  S_C = e^{lgam} S0 + Khat^T nu
+// Every pair factor e^{lG_i - lG_j} (i >= j) is a_i m[b(i)][b(j)] bf_j over
+// 16-token blocks (a = e^{lG - r_b}, bf = 1 / a, m = e^{r_bi - r_bj}, r_b the
+// sum up to block b), so no factor leaves fp32's range for |floor| <= 5.45.
+//
+// Reverse mode in three kernels (dS_C: gradient of the chunk's end state):
+//   chain_prep  (a CTA per chunk x head): the chain's per-chunk constants
+//       Et = Diag(beta) T^T (scale A_qk^T go),  Wt = Diag(beta) T^T Khat,
+//       F = scale Qbar^T go,  Kbar,  e^{lgam},  with go = do sigmoid(z);
+//       and Z, nu, T, At, A_qk for the last kernel, dz of the output gate.
+//   chain       (a CTA per sequence x head, chunks last first):
+//       dZ = Et + Wt dS_C,  dS0 = F + e^{lgam} dS_C - Kbar^T dZ  (dS_C of every chunk kept).
+//   chain_grad  (a CTA per chunk x head): with dS_C,
+//       dnu = scale A_qk^T go + Khat dS_C,  dY = T^T dnu,  dv = Diag(beta) dY,
+//       dT = dnu (Diag(beta) Z)^T,  dA_kk = -T^T dT T^T (j < i),  dA_qk = scale go nu^T (j <= i),
+//       dq  = a (e^{r} scale go S0^T + sum_j dA_qk m bf k_j),
+//       dk1 = a (-e^{r} Diag(beta) dY S0^T + sum_j Diag(beta) dA_kk m bf k_j),
+//       dk2 = bf (sum_i dA_qk m a q_i + sum_i Diag(beta) dA_kk m a k_i + e^{lgam - r} nu dS_C^T),
+//       dk = dk1 + dk2,  dg_s = [g_s >= floor] (sum_{t>=s} (q dq + k (dk1 - dk2))_t + dlgam),
+//       dlgam = e^{lgam} rowsum(dS_C o S0) + sum_t k_t dkh_t, dkh the Khat part of dk2
+//       (the same rounded terms as in dk2, so the two sides of the cancellation
+//       inside sum_t match; S_C from a forward's snapshot would not),
+//       dbeta = rowsum(dY o Z) + rowsum(dA_kk o At).
+// Every product runs on the warp-level tensor cores in tf32 with fp32
+// accumulation, 3xTF32 (leading and low parts) for fp32 I/O and, for every
+// I/O dtype, for the four products (dq, dk1, dk2 and its Khat part) whose
+// outputs hold the two sides of the pair terms that cancel inside dg's sum
+// over the chunk: rounded alike, they cancel to fp32 accuracy.
+#pragma once
+
+#include "kda_common.cuh"
+
+namespace kda {
+namespace bwdc {
+
+constexpr int C = 64;           // chunk
+constexpr int D = 128;          // dk = dv
+constexpr int NB = 4;           // 16-token blocks per chunk
+constexpr int NT = 512, NW = NT / 32;
+constexpr int CD = C * D, CC = C * C, DD = D * D;
+
+// per (chunk, head) scratch, floats
+struct Scratch {
+    static constexpr int64_t ET = 0, WT = ET + CD, KBAR = WT + CD, Z = KBAR + CD, NU = Z + CD,
+                             DY = NU + CD, F = DY + CD, DSC = F + DD, T = DSC + DD, AT = T + CC,
+                             AQK = AT + CC, GAM = AQK + CC, FLOATS = GAM + D;
+};
+
+struct ChunkBwdParams {
+    const void *q, *k, *v, *g, *beta, *gate, *dout;   // I/O dtype
+    const float *S0, *dS_T;                           // [N][H][D][D] or null
+    const int32_t *cu_seqlens;                        // [N + 1]
+    const float *ckpt;                                // state after 64 m tokens: slot ckpt_base[n] + m - 1
+    const int64_t *ckpt_base;                         // [N + 1]
+    const int32_t *chunk_seq, *chunk_idx;             // [chunks]: sequence, index in it
+    const int64_t *chunk_base;                        // [N + 1]: first chunk of sequence n
+    float *scratch;                                   // [chunks * H][Scratch::FLOATS]
+    void *dq, *dk, *dv, *dg, *dbeta, *dgate;
+    float *dS0;
+    int32_t num_heads;
+    float scale, g_floor;
+};
+
+// XOR-swizzled element offsets of row-major fp32 tiles (128 or 64 columns):
+// groups of 4 columns move with the row's low 3 bits, so the fragment loads
+// below (8 rows x 4 columns, or 4 rows x 8 columns) touch distinct banks, or
+// two-way at most, without padding.
+__device__ __forceinline__ int xd(int r, int c) { return r * D + (c ^ ((r & 7) << 2)); }
+__device__ __forceinline__ int xc(int r, int c) { return r * C + (c ^ ((r & 7) << 2)); }
+
+__device__ __forceinline__ uint32_t tf32_rna(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// D[16x8] += A[16x8] B[8x8], tf32 inputs, fp32 accumulation; g = lane / 4, t = lane % 4:
+//   a = {A[g][t], A[g+8][t], A[g][t+4], A[g+8][t+4]},  b = {B[t][g], B[t+4][g]},
+//   d = {D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1]}.
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+                 "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// out[M x N] = sum_k A(i, k) B(k, j): warp tiles of 16 rows x 8 NT8 columns,
+// dealt round-robin to warps w0 .. w0 + nw - 1.  krange(i0, j0, lo, hi) gives
+// the tile's contraction range (multiples of 8); fa(i, k) and fb(i0, k, j) the
+// operands (fb sees the tile's first row, for factors that depend on the output
+// row block); epi(i, j, x) receives every result.  SPLIT: 3xTF32.
+template <int M, int N, int NT8, bool SPLIT, class FK, class FA, class FB, class FE>
+__device__ __forceinline__ void gemm(int warp, int w0, int nw, int lane, FK krange, FA fa, FB fb, FE epi) {
+    static_assert(M % 16 == 0 && N % (8 * NT8) == 0, "tile shape");
+    constexpr int TN = N / (8 * NT8), TILES = (M / 16) * TN;
+    if (warp < w0 || warp >= w0 + nw) return;
+    const int g = lane >> 2, t = lane & 3;
+    for (int tile = warp - w0; tile < TILES; tile += nw) {
+        const int i0 = (tile / TN) * 16, j0 = (tile % TN) * (8 * NT8);
+        float acc[NT8][4];
+#pragma unroll
+        for (int n = 0; n < NT8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
+        int lo, hi;
+        krange(i0, j0, lo, hi);
+#pragma unroll 2
+        for (int k0 = lo; k0 < hi; k0 += 8) {
+            const float av[4] = {fa(i0 + g, k0 + t), fa(i0 + g + 8, k0 + t), fa(i0 + g, k0 + t + 4),
+                                 fa(i0 + g + 8, k0 + t + 4)};
+            uint32_t ah[4], al[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                ah[e] = tf32_rna(av[e]);
+                if constexpr (SPLIT) al[e] = tf32_rna(av[e] - __uint_as_float(ah[e]));
+            }
+#pragma unroll
+            for (int n = 0; n < NT8; ++n) {
+                const int j = j0 + 8 * n + g;
+                const float b0 = fb(i0, k0 + t, j), b1 = fb(i0, k0 + t + 4, j);
+                const uint32_t h0 = tf32_rna(b0), h1 = tf32_rna(b1);
+                mma_tf32(acc[n], ah, h0, h1);
+                if constexpr (SPLIT) {
+                    mma_tf32(acc[n], ah, tf32_rna(b0 - __uint_as_float(h0)), tf32_rna(b1 - __uint_as_float(h1)));
+                    mma_tf32(acc[n], al, h0, h1);
+                }
+            }
+        }
+#pragma unroll
+        for (int n = 0; n < NT8; ++n) {
+            const int j = j0 + 8 * n + 2 * t;
+            epi(i0 + g, j, acc[n][0]);
+            epi(i0 + g, j + 1, acc[n][1]);
+            epi(i0 + g + 8, j, acc[n][2]);
+            epi(i0 + g + 8, j + 1, acc[n][3]);
+        }
+    }
+}
+
+// The chunk a CTA works on, and where its tokens are.
+struct ChunkRef {
+    int64_t u;          // chunk * H + head: scratch index
+    int64_t n, h, ci;   // sequence, head, chunk index in the sequence
+    int64_t tok0;       // first token (packed row) of the chunk
+    int Lc;             // tokens in the chunk
+    int64_t L;          // tokens in the sequence
+};
+
+__device__ __forceinline__ ChunkRef chunk_ref(const ChunkBwdParams &p) {
+    ChunkRef r;
+    const int64_t H = p.num_heads;
+    const int64_t c = blockIdx.x / H;
+    r.h = blockIdx.x % H;
+    r.u = blockIdx.x;
+    r.n = p.chunk_seq[c];
+    r.ci = p.chunk_idx[c];
+    const int64_t tb = p.cu_seqlens[r.n];
+    r.L = (int64_t)p.cu_seqlens[r.n + 1] - tb;
+    r.tok0 = tb + r.ci * C;
+    const int64_t left = r.L - r.ci * C;
+    r.Lc = (int)(left < C ? left : C);
+    return r;
+}
+
+// the chunk's start state (null: zero)
+__device__ __forceinline__ const float *start_state(const ChunkBwdParams &p, const ChunkRef &r) {
+    const int64_t H = p.num_heads;
+    if (r.ci == 0) return p.S0 ? p.S0 + (r.n * H + r.h) * DD : nullptr;
+    return p.ckpt + ((p.ckpt_base[r.n] + r.ci - 1) * H + r.h) * DD;
+}
+
+// Decay tables of a chunk from gc = max(g, floor) (zero past the chunk's end,
+// swizzled [C][D] at gc): a = e^{lG - r_b} into `a_out` (may alias gc), and
+// m[bi][bj] = e^{r_bi - r_bj} (bi >= bj, else 0), eR[b] = e^{r_b},
+// eG[b] = e^{lgam - r_b}, gam = e^{lgam}.  Every exponent is a sum of at most
+// 16 terms or of block totals, never a difference of long running sums.
+// Threads 0 .. D-1, one channel each.
+__device__ __forceinline__ void decay_tables(int tid, float *gc, float *a_out, float *m, float *eR,
+                                             float *eG, float *gam) {
+    if (tid >= D) return;
+    const int c = tid;
+    float tot[NB];                       // block totals of gc
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        float x = 0.0f;
+#pragma unroll 4
+        for (int t = 16 * b; t < 16 * b + 16; ++t) {
+            x += gc[xd(t, c)];
+            a_out[xd(t, c)] = expf(x);
+        }
+        tot[b] = x;
+    }
+#pragma unroll
+    for (int bi = 0; bi < NB; ++bi) {
+        float r = 0.0f, rest = 0.0f;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            if (b < bi) r += tot[b];
+            else rest += tot[b];
+        }
+        eR[bi * D + c] = expf(r);
+        eG[bi * D + c] = expf(rest);
+#pragma unroll
+        for (int bj = 0; bj < NB; ++bj) {
+            float x = 0.0f;
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+                if (b >= bj && b < bi) x += tot[b];
+            m[(bi * NB + bj) * D + c] = bj <= bi ? expf(x) : 0.0f;
+        }
+    }
+    gam[c] = expf((tot[0] + tot[1]) + (tot[2] + tot[3]));
+}
+
+// T = (I + Diag(beta) At)^-1 (unit lower triangular, 64 x 64, swizzled [C][C]
+// at Tm) from At (swizzled, at At) and beta: 16 x 16 diagonal blocks by forward
+// substitution, then the merges [[T11, 0], [T21, T22]], T21 = -T22 (A21 T11),
+// for 16 -> 32 and 32 -> 64.  xs: 2 x 16 x 16 + 32 x 32 floats of scratch.
+// Every thread of the CTA calls it (it holds block barriers).
+template <bool SPLIT>
+__device__ void invert_T(int tid, int warp, int lane, const float *At, const float *beta, float *Tm, float *xs) {
+    for (int i = tid; i < CC; i += NT) Tm[i] = 0.0f;
+    __syncthreads();
+    if (warp < 2) {
+        const int d0 = 32 * warp + 16 * (lane >> 4), jj = lane & 15;
+        float t[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) t[i] = i == jj ? 1.0f : 0.0f;
+#pragma unroll
+        for (int i = 1; i < 16; ++i) {
+            const float b = beta[d0 + i];
+            float acc = 0.0f;
+#pragma unroll
+            for (int m = 0; m < 15; ++m)
+                if (m < i) acc = fmaf(b * At[xc(d0 + i, d0 + m)], t[m], acc);
+            if (i > jj) t[i] = -acc;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Tm[xc(d0 + i, d0 + jj)] = t[i];
+    }
+    __syncthreads();
+    // 16 -> 32, pair p on warp p: X = A21 T11, T21 = -T22 X
+    if (warp < 2) {
+        const int p = warp, o = 32 * p;
+        float *X = xs + p * 256;           // [16][16]
+        auto kr = [](int, int, int &lo, int &hi) { lo = 0; hi = 16; };
+        gemm<16, 16, 2, SPLIT>(warp, p, 1, lane, kr,
+            [&](int i, int m) { return beta[o + 16 + i] * At[xc(o + 16 + i, o + m)]; },
+            [&](int, int m, int j) { return Tm[xc(o + m, o + j)]; },
+            [&](int i, int j, float x) { X[i * 16 + j] = x; });
+        __syncwarp();
+        gemm<16, 16, 2, SPLIT>(warp, p, 1, lane, kr,
+            [&](int i, int m) { return Tm[xc(o + 16 + i, o + 16 + m)]; },
+            [&](int, int m, int j) { return X[m * 16 + j]; },
+            [&](int i, int j, float x) { Tm[xc(o + 16 + i, o + j)] = -x; });
+    }
+    __syncthreads();
+    // 32 -> 64: X = A[32:64, 0:32] T[0:32, 0:32], T[32:64, 0:32] = -T[32:64, 32:64] X
+    {
+        float *X = xs + 512;               // [32][32]
+        auto kr = [](int, int, int &lo, int &hi) { lo = 0; hi = 32; };
+        gemm<32, 32, 4, SPLIT>(warp, 0, NW, lane, kr,
+            [&](int i, int m) { return beta[32 + i] * At[xc(32 + i, m)]; },
+            [&](int, int m, int j) { return Tm[xc(m, j)]; },
+            [&](int i, int j, float x) { X[i * 32 + j] = x; });
+        __syncthreads();
+        gemm<32, 32, 4, SPLIT>(warp, 0, NW, lane, kr,
+            [&](int i, int m) { return Tm[xc(32 + i, 32 + m)]; },
+            [&](int, int m, int j) { return X[m * 32 + j]; },
+            [&](int i, int j, float x) { Tm[xc(32 + i, j)] = -x; });
+    }
+    __syncthreads();
+}
+
+// shared memory of chain_prep: 4 [C][D] tiles, 3 [C][C] tiles, tables
+struct PrepSmem {
+    static constexpr int B0 = 0, B1 = B0 + CD, B2 = B1 + CD, B3 = B2 + CD;
+    static constexpr int AQ = B3 + CD, AT = AQ + CC, TT = AT + CC;
+    static constexpr int M = TT + CC, ER = M + NB * NB * D, EG = ER + NB * D, GM = EG + NB * D;
+    static constexpr int BT = GM + D, FLOATS = BT + C;
+    static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
+};
+
+// Stage the chunk's q, k (I/O dtype -> fp32) and gc = max(g, floor), zero past its end.
+template <typename TIO>
+__device__ __forceinline__ void stage_qkg(const ChunkBwdParams &p, const ChunkRef &r, int tid, float *sq,
+                                          float *sk, float *sg, float *sb) {
+    const TIO *q = static_cast<const TIO *>(p.q);
+    const TIO *k = static_cast<const TIO *>(p.k);
+    const TIO *g = static_cast<const TIO *>(p.g);
+    const int64_t H = p.num_heads;
+    for (int i = tid; i < CD; i += NT) {
+        const int t = i / D, c = i % D;
+        float qv = 0.0f, kv = 0.0f, gv = 0.0f;
+        if (t < r.Lc) {
+            const int64_t e = ((r.tok0 + t) * H + r.h) * D + c;
+            qv = ld(q, e);
+            kv = ld(k, e);
+            gv = fmaxf(ld(g, e), p.g_floor);
+        }
+        sq[xd(t, c)] = qv;
+        sk[xd(t, c)] = kv;
+        sg[xd(t, c)] = gv;
+    }
+    if (tid < C) sb[tid] = tid < r.Lc ? ld(static_cast<const TIO *>(p.beta), (r.tok0 + tid) * H + r.h) : 0.0f;
+}
+
+template <typename TIO, bool SPLIT>
+__global__ void __launch_bounds__(NT, 1) chain_prep_kernel(ChunkBwdParams p) {
+    using S = PrepSmem;
+    extern __shared__ float4 bwdc_smem4[];
+    float *sm = reinterpret_cast<float *>(bwdc_smem4);
+    float *qa = sm + S::B0, *ka = sm + S::B1, *kb = sm + S::B2, *b3 = sm + S::B3;
+    float *Aq = sm + S::AQ, *At = sm + S::AT, *Tm = sm + S::TT;
+    float *m = sm + S::M, *eR = sm + S::ER, *eG = sm + S::EG, *gam = sm + S::GM, *sb = sm + S::BT;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const ChunkRef r = chunk_ref(p);
+    const int64_t H = p.num_heads;
+    float *scr = p.scratch + r.u * Scratch::FLOATS;
+    const float *S0p = start_state(p, r);
+    const TIO *vin = static_cast<const TIO *>(p.v);
+    const TIO *dout = static_cast<const TIO *>(p.dout);
+    const TIO *gate = static_cast<const TIO *>(p.gate);
+    const float scale = p.scale;
+
+    // q -> qa, k -> ka (and kb), gc -> a (in b3)
+    stage_qkg<TIO>(p, r, tid, qa, ka, b3, sb);
+    __syncthreads();
+    decay_tables(tid, b3, b3, m, eR, eG, gam);
+    __syncthreads();
+    for (int i = tid; i < CD; i += NT) {
+        const int t = i / D, c = i % D, x = xd(t, c);
+        const float a = b3[x], kv = ka[x];
+        qa[x] *= a;
+        ka[x] = kv * a;
+        kb[x] = kv / a;
+    }
+    __syncthreads();
+
+    // A_qk (warps 0-7) and At (warps 8-15): the pair factor's middle term rides on kb
+    auto kr_tri = [](int i0, int j0, int &lo, int &hi) { lo = 0; hi = j0 > i0 + 15 ? 0 : D; };
+    auto fb_mkb = [&](int i0, int c, int j) { return kb[xd(j, c)] * m[((i0 >> 4) * NB + (j >> 4)) * D + c]; };
+    gemm<C, C, 4, SPLIT>(warp, 0, 8, lane, kr_tri, [&](int i, int c) { return qa[xd(i, c)]; }, fb_mkb,
+                         [&](int i, int j, float x) { Aq[xc(i, j)] = j <= i ? x : 0.0f; });
+    gemm<C, C, 4, SPLIT>(warp, 8, 8, lane, kr_tri, [&](int i, int c) { return ka[xd(i, c)]; }, fb_mkb,
+                         [&](int i, int j, float x) { At[xc(i, j)] = j < i ? x : 0.0f; });
+    __syncthreads();
+    invert_T<SPLIT>(tid, warp, lane, At, sb, Tm, b3);   // b3 (a) is not needed any more
+
+    // Z = V - Kbar S0 (into b3), Kbar and the small tiles to scratch
+    gemm<C, D, 4, SPLIT>(warp, 0, NW, lane,
+        [&](int, int, int &lo, int &hi) { lo = 0; hi = S0p ? D : 0; },
+        [&](int i, int c) { return ka[xd(i, c)] * eR[(i >> 4) * D + c]; },
+        [&](int, int c, int v) { return S0p[c * D + v]; },
+        [&](int i, int v, float x) {
+            const float vi = i < r.Lc ? ld(vin, ((r.tok0 + i) * H + r.h) * D + v) : 0.0f;
+            const float z = vi - x;
+            b3[xd(i, v)] = z;
+            scr[Scratch::Z + i * D + v] = z;
+        });
+    for (int i = tid; i < CD; i += NT) {
+        const int t = i / D, c = i % D;
+        scr[Scratch::KBAR + i] = ka[xd(t, c)] * eR[(t >> 4) * D + c];
+    }
+    for (int i = tid; i < CC; i += NT) {
+        const int a = i / C, b = i % C;
+        scr[Scratch::T + i] = Tm[xc(a, b)];
+        scr[Scratch::AT + i] = At[xc(a, b)];
+        scr[Scratch::AQK + i] = Aq[xc(a, b)];
+    }
+    if (tid < D) scr[Scratch::GAM + tid] = gam[tid];
+    __syncthreads();
+    // nu = T Diag(beta) Z (into ka)
+    gemm<C, D, 4, SPLIT>(warp, 0, NW, lane,
+        [&](int i0, int, int &lo, int &hi) { lo = 0; hi = i0 + 16; },
+        [&](int i, int l) { return Tm[xc(i, l)]; },
+        [&](int, int l, int v) { return sb[l] * b3[xd(l, v)]; },
+        [&](int i, int v, float x) {
+            ka[xd(i, v)] = x;
+            scr[Scratch::NU + i * D + v] = x;
+        });
+    __syncthreads();
+    // Oraw = scale (Qbar S0 + A_qk nu): dz of the gate, and go = do sigmoid(z) (into b3)
+    float *nu = ka;
+    gemm<C, D, 4, SPLIT>(warp, 0, NW, lane,
+        [&](int i0, int, int &lo, int &hi) { lo = S0p ? 0 : D; hi = D + i0 + 16; },
+        [&](int i, int k) { return k < D ? qa[xd(i, k)] * eR[(i >> 4) * D + k] : Aq[xc(i, k - D)]; },
+        [&](int, int k, int v) { return k < D ? S0p[k * D + v] : nu[xd(k - D, v)]; },
+        [&](int i, int v, float x) {
+            float go = 0.0f;
+            if (i < r.Lc) {
+                const int64_t e = ((r.tok0 + i) * H + r.h) * D + v;
+                const float dov = ld(dout, e);
+                if (gate) {
+                    const float sg = sigmoidf(ld(gate, e));
+                    st(static_cast<TIO *>(p.dgate), e, dov * scale * x * sg * (1.0f - sg));
+                    go = dov * sg;
+                } else {
+                    go = dov;
+                }
+            }
+            b3[xd(i, v)] = go;
+        });
+    __syncthreads();
+    // F = scale Qbar^T go (to scratch), E = scale A_qk^T go (into nu's tile)
+    gemm<D, D, 4, SPLIT>(warp, 0, NW, lane, [](int, int, int &lo, int &hi) { lo = 0; hi = C; },
+        [&](int c, int i) { return qa[xd(i, c)] * eR[(i >> 4) * D + c]; },
+        [&](int, int i, int v) { return b3[xd(i, v)]; },
+        [&](int c, int v, float x) { scr[Scratch::F + c * D + v] = scale * x; });
+    float *E = ka;
+    gemm<C, D, 4, SPLIT>(warp, 0, NW, lane, [](int i0, int, int &lo, int &hi) { lo = i0; hi = C; },
+        [&](int j, int i) { return Aq[xc(i, j)]; },
+        [&](int, int i, int v) { return b3[xd(i, v)]; },
+        [&](int j, int v, float x) { E[xd(j, v)] = scale * x; });
+    __syncthreads();
+    // Et = Diag(beta) T^T E, Wt = Diag(beta) T^T Khat (to scratch)
+    gemm<C, D, 4, SPLIT>(warp, 0, NW, lane, [](int i0, int, int &lo, int &hi) { lo = i0; hi = C; },
+        [&](int i, int l) { return Tm[xc(l, i)]; },
+        [&](int, int l, int v) { return E[xd(l, v)]; },
+        [&](int i, int v, float x) { scr[Scratch::ET + i * D + v] = sb[i] * x; });
+    gemm<C, D, 4, SPLIT>(warp, 0, NW, lane, [](int i0, int, int &lo, int &hi) { lo = i0; hi = C; },
+        [&](int i, int l) { return Tm[xc(l, i)]; },
+        [&](int, int l, int c) { return kb[xd(l, c)] * eG[(l >> 4) * D + c]; },
+        [&](int i, int c, float x) { scr[Scratch::WT + i * D + c] = sb[i] * x; });
+}
+
+// shared memory of chain: dS [D][D], dZ, Wt, Kbar [C][D], e^{lgam}
+struct ChainSmem {
+    static constexpr int DS = 0, DZ = DS + DD, WT = DZ + CD, KB = WT + CD, GM = KB + CD;
+    static constexpr int FLOATS = GM + D;
+    static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
+};
+
+template <bool SPLIT>
+__global__ void __launch_bounds__(NT, 1) chain_kernel(ChunkBwdParams p) {
+    using S = ChainSmem;
+    extern __shared__ float4 bwdc_smem4[];
+    float *sm = reinterpret_cast<float *>(bwdc_smem4);
+    float *dS = sm + S::DS, *dZ = sm + S::DZ, *Wt = sm + S::WT, *Kb = sm + S::KB, *gam = sm + S::GM;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t H = p.num_heads, n = blockIdx.x / H, h = blockIdx.x % H;
+    const int64_t L = (int64_t)p.cu_seqlens[n + 1] - p.cu_seqlens[n];
+    const int64_t nch = (L + C - 1) / C;
+    const float *dST = p.dS_T ? p.dS_T + (n * H + h) * DD : nullptr;
+    for (int i = tid; i < DD; i += NT) {
+        const int c = i / D, v = i % D;
+        dS[xd(c, v)] = dST ? dST[i] : 0.0f;
+    }
+    for (int64_t ci = nch - 1; ci >= 0; --ci) {
+        float *scr = p.scratch + ((p.chunk_base[n] + ci) * H + h) * Scratch::FLOATS;
+        float *dsc = scr + Scratch::DSC;
+        __syncthreads();
+        for (int i = tid; i < DD; i += NT) {
+            const int c = i / D, v = i % D;
+            dsc[i] = dS[xd(c, v)];
+        }
+        for (int i = tid; i < CD; i += NT) {
+            const int j = i / D, c = i % D;
+            Wt[xd(j, c)] = scr[Scratch::WT + i];
+            Kb[xd(j, c)] = scr[Scratch::KBAR + i];
+        }
+        if (tid < D) gam[tid] = scr[Scratch::GAM + tid];
+        __syncthreads();
+        // dZ = Et + Wt dS
+        gemm<C, D, 4, SPLIT>(warp, 0, NW, lane, [](int, int, int &lo, int &hi) { lo = 0; hi = D; },
+            [&](int j, int c) { return Wt[xd(j, c)]; },
+            [&](int, int c, int v) { return dS[xd(c, v)]; },
+            [&](int j, int v, float x) { dZ[xd(j, v)] = scr[Scratch::ET + j * D + v] + x; });
+        __syncthreads();
+        // dS <- F + e^{lgam} dS - Kbar^T dZ (each element read and written by its own thread)
+        gemm<D, D, 4, SPLIT>(warp, 0, NW, lane, [](int, int, int &lo, int &hi) { lo = 0; hi = C; },
+            [&](int c, int j) { return Kb[xd(j, c)]; },
+            [&](int, int j, int v) { return dZ[xd(j, v)]; },
+            [&](int c, int v, float x) {
+                const int e = xd(c, v);
+                dS[e] = scr[Scratch::F + c * D + v] + gam[c] * dS[e] - x;
+            });
+    }
+    __syncthreads();
+    if (p.dS0) {
+        float *out = p.dS0 + (n * H + h) * DD;
+        for (int i = tid; i < DD; i += NT) {
+            const int c = i / D, v = i % D;
+            out[i] = dS[xd(c, v)];
+        }
+    }
+}
+
+// shared memory of chain_grad: 5 [C][D] tiles, 3 [C][C] tiles, tables
+struct GradSmem {
+    static constexpr int B0 = 0, B1 = B0 + CD, B2 = B1 + CD, B3 = B2 + CD, B4 = B3 + CD;
+    static constexpr int TT = B4 + CD, S1 = TT + CC, S2 = S1 + CC;
+    static constexpr int M = S2 + CC, ER = M + NB * NB * D, EG = ER + NB * D, GM = EG + NB * D;
+    static constexpr int BT = GM + D, DL = BT + C, FLOATS = DL + D;
+    static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
+};
+
+template <typename TIO, bool SPLIT>
+__global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
+    using S = GradSmem;
+    extern __shared__ float4 bwdc_smem4[];
+    float *sm = reinterpret_cast<float *>(bwdc_smem4);
+    float *qa = sm + S::B0, *kb = sm + S::B1, *aa = sm + S::B2, *b3 = sm + S::B3, *b4 = sm + S::B4;
+    float *Tm = sm + S::TT, *s1 = sm + S::S1, *s2 = sm + S::S2;
+    float *m = sm + S::M, *eR = sm + S::ER, *eG = sm + S::EG, *gam = sm + S::GM, *sb = sm + S::BT;
+    float *sdl = sm + S::DL;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const ChunkRef r = chunk_ref(p);
+    const int64_t H = p.num_heads;
+    float *scr = p.scratch + r.u * Scratch::FLOATS;
+    const float *S0p = start_state(p, r);
+    const float *dSC = scr + Scratch::DSC;
+    const TIO *qin = static_cast<const TIO *>(p.q);
+    const TIO *kin = static_cast<const TIO *>(p.k);
+    const TIO *gin = static_cast<const TIO *>(p.g);
+    const TIO *dout = static_cast<const TIO *>(p.dout);
+    const TIO *gate = static_cast<const TIO *>(p.gate);
+    const float scale = p.scale;
+    auto row = [&](int i) { return ((r.tok0 + i) * H + r.h) * D; };
+
+    // q -> qa, k -> kb, gc -> lG tables (a into aa)
+    stage_qkg<TIO>(p, r, tid, qa, kb, b4, sb);
+    for (int i = tid; i < CC; i += NT) Tm[xc(i / C, i % C)] = scr[Scratch::T + i];
+    __syncthreads();
+    decay_tables(tid, b4, aa, m, eR, eG, gam);
+    __syncthreads();
+    for (int i = tid; i < CD; i += NT) {
+        const int t = i / D, c = i % D, x = xd(t, c);
+        const float a = aa[x];
+        qa[x] *= a;
+        kb[x] /= a;
+        float go = 0.0f;
+        if (t < r.Lc) {
+            const int64_t e = row(t) + c;
+            go = ld(dout, e);
+            if (gate) go *= sigmoidf(ld(gate, e));
+        }
+        b3[x] = go;
+    }
+    __syncthreads();
+    // dnu = scale A_qk^T go + Khat dS_C (into b4)
+    const float *Aqk = scr + Scratch::AQK;
+    gemm<C, D, 4, SPLIT>(warp, 0, NW, lane, [](int i0, int, int &lo, int &hi) { lo = i0; hi = C + D; },
+        [&](int j, int k) { return k < C ? scale * Aqk[k * C + j] : kb[xd(j, k - C)] * eG[(j >> 4) * D + k - C]; },
+        [&](int, int k, int v) { return k < C ? b3[xd(k, v)] : dSC[(k - C) * D + v]; },
+        [&](int j, int v, float x) { b4[xd(j, v)] = x; });
+    __syncthreads();
+    // dY = T^T dnu: dv = Diag(beta) dY, dY to scratch;  dT = dnu (Diag(beta) Z)^T (into s1)
+    const float *Zg = scr + Scratch::Z;
+    gemm<C, D, 4, SPLIT>(warp, 0, NW, lane, [](int i0, int, int &lo, int &hi) { lo = i0; hi = C; },
+        [&](int i, int l) { return Tm[xc(l, i)]; },
+        [&](int, int l, int v) { return b4[xd(l, v)]; },
+        [&](int i, int v, float x) {
+            scr[Scratch::DY + i * D + v] = x;
+            if (i < r.Lc) st(static_cast<TIO *>(p.dv), row(i) + v, sb[i] * x);
+        });
+    gemm<C, C, 4, SPLIT>(warp, 0, NW, lane, [](int i0, int j0, int &lo, int &hi) { lo = 0; hi = j0 > i0 + 15 ? 0 : D; },
+        [&](int i, int v) { return b4[xd(i, v)]; },
+        [&](int, int v, int j) { return sb[j] * Zg[j * D + v]; },
+        [&](int i, int j, float x) { s1[xc(i, j)] = x; });
+    __syncthreads();
+    // X = dT T^T (into s2), then dA_kk = -T^T X, j < i (into s1)
+    gemm<C, C, 4, SPLIT>(warp, 0, NW, lane, [](int, int, int &lo, int &hi) { lo = 0; hi = C; },
+        [&](int i, int b) { return s1[xc(i, b)]; },
+        [&](int, int b, int j) { return Tm[xc(j, b)]; },
+        [&](int i, int j, float x) { s2[xc(i, j)] = x; });
+    __syncthreads();
+    gemm<C, C, 4, SPLIT>(warp, 0, NW, lane, [](int i0, int j0, int &lo, int &hi) { lo = i0; hi = j0 > i0 + 15 ? i0 : C; },
+        [&](int i, int a) { return Tm[xc(a, i)]; },
+        [&](int, int a, int j) { return s2[xc(a, j)]; },
+        [&](int i, int j, float x) { s1[xc(i, j)] = j < i ? -x : 0.0f; });
+    __syncthreads();
+    // dA_qk = scale go nu^T, j <= i (into s2)
+    const float *nug = scr + Scratch::NU;
+    gemm<C, C, 4, SPLIT>(warp, 0, NW, lane, [](int i0, int j0, int &lo, int &hi) { lo = 0; hi = j0 > i0 + 15 ? 0 : D; },
+        [&](int i, int v) { return b3[xd(i, v)]; },
+        [&](int, int v, int j) { return nug[j * D + v]; },
+        [&](int i, int j, float x) { s2[xc(i, j)] = j <= i ? scale * x : 0.0f; });
+    __syncthreads();
+    // dbeta = rowsum(dY o Z) + rowsum(dA_kk o At): a warp per row
+    {
+        const float *dYg = scr + Scratch::DY, *Atg = scr + Scratch::AT;
+        for (int i = warp; i < r.Lc; i += NW) {
+            float s = 0.0f;
+#pragma unroll
+            for (int e = 0; e < D / 32; ++e) s = fmaf(dYg[i * D + lane + 32 * e], Zg[i * D + lane + 32 * e], s);
+#pragma unroll
+            for (int e = 0; e < C / 32; ++e) s = fmaf(s1[xc(i, lane + 32 * e)], Atg[i * C + lane + 32 * e], s);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+            if (lane == 0) st(static_cast<TIO *>(p.dbeta), (r.tok0 + i) * H + r.h, s);
+        }
+    }
+    // dq = a (e^r scale go S0^T + dA_qk m kb); q dq into b4 (dlG)
+    auto kr_pair = [&](int i0, int, int &lo, int &hi) { lo = S0p ? 0 : D; hi = D + i0 + 16; };
+    auto fb_pair = [&](int i0, int k, int c) {
+        return k < D ? S0p[c * D + k] * eR[(i0 >> 4) * D + c]
+                     : m[((i0 >> 4) * NB + ((k - D) >> 4)) * D + c] * kb[xd(k - D, c)];
+    };
+    gemm<C, D, 4, true>(warp, 0, NW, lane, kr_pair,
+        [&](int i, int k) { return k < D ? scale * b3[xd(i, k)] : s2[xc(i, k - D)]; }, fb_pair,
+        [&](int i, int c, float x) {
+            const float dq = aa[xd(i, c)] * x;
+            float ql = 0.0f;
+            if (i < r.Lc) {
+                st(static_cast<TIO *>(p.dq), row(i) + c, dq);
+                ql = ld(qin, row(i) + c);
+            }
+            b4[xd(i, c)] = ql * dq;
+        });
+    __syncthreads();
+    // dk1 = a (-e^r Diag(beta) dY S0^T + Diag(beta) dA_kk m kb) (into b3); dlG += k dk1
+    const float *dYg = scr + Scratch::DY;
+    gemm<C, D, 4, true>(warp, 0, NW, lane, kr_pair,
+        [&](int i, int k) { return k < D ? -sb[i] * dYg[i * D + k] : sb[i] * s1[xc(i, k - D)]; }, fb_pair,
+        [&](int i, int c, float x) {
+            const int e = xd(i, c);
+            const float d1 = aa[e] * x;
+            b3[e] = d1;
+            if (i < r.Lc) b4[e] += ld(kin, row(i) + c) * d1;
+        });
+    __syncthreads();
+    // dk2 through Kbrev: bf (dA_qk^T m qa + (Diag(beta) dA_kk)^T m ka); b3 <- dk1 + that
+    gemm<C, D, 4, true>(warp, 0, NW, lane, [](int, int, int &lo, int &hi) { lo = 0; hi = 2 * C; },
+        [&](int j, int k) { return k < C ? s2[xc(k, j)] : sb[k - C] * s1[xc(k - C, j)]; },
+        [&](int j0, int k, int c) {
+            if (k < C) return m[((k >> 4) * NB + (j0 >> 4)) * D + c] * qa[xd(k, c)];
+            const int i = k - C, e = xd(i, c);
+            return m[((i >> 4) * NB + (j0 >> 4)) * D + c] * ((kb[e] * aa[e]) * aa[e]);   // k a
+        },
+        [&](int j, int c, float x) {
+            const int e = xd(j, c);
+            const float d2 = x / aa[e];
+            b3[e] += d2;
+            if (j < r.Lc) b4[e] -= ld(kin, row(j) + c) * d2;
+        });
+    // dkh = bf e^{lgam - r} nu dS_C^T (through Khat): dk = b3 + dkh; k dkh into b3 for dlgam
+    gemm<C, D, 4, true>(warp, 0, NW, lane, [](int, int, int &lo, int &hi) { lo = 0; hi = D; },
+        [&](int j, int v) { return nug[j * D + v]; },
+        [&](int j0, int v, int c) { return dSC[c * D + v] * eG[(j0 >> 4) * D + c]; },
+        [&](int j, int c, float x) {
+            const int e = xd(j, c);
+            const float dh = x / aa[e];
+            float kdh = 0.0f;
+            if (j < r.Lc) {
+                st(static_cast<TIO *>(p.dk), row(j) + c, b3[e] + dh);
+                kdh = ld(kin, row(j) + c) * dh;
+                b4[e] -= kdh;
+            }
+            b3[e] = kdh;
+        });
+    // e^{lgam} rowsum(dS_C o S0): a warp per 8 channels
+    for (int c = warp; c < D; c += NW) {
+        float s = 0.0f;
+        if (S0p) {
+#pragma unroll
+            for (int e = 0; e < D / 32; ++e) s = fmaf(dSC[c * D + lane + 32 * e], S0p[c * D + lane + 32 * e], s);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        }
+        if (lane == 0) sdl[c] = gam[c] * s;
+    }
+    __syncthreads();
+    // dg_s = [g_s >= floor] (sum_{t >= s} dlG_t + dlgam), one channel per thread
+    if (tid < D) {
+        const int c = tid;
+        float run = sdl[c];
+        for (int t = 0; t < C; ++t) run += b3[xd(t, c)];      // + sum_t k_t dkh_t
+        for (int t = C - 1; t >= 0; --t) {
+            run += b4[xd(t, c)];
+            if (t < r.Lc) {
+                const int64_t e = row(t) + c;
+                st(static_cast<TIO *>(p.dg), e, ld(gin, e) >= p.g_floor ? run : 0.0f);
+            }
+        }
+    }
+}
+
+}  // namespace bwdc
+}  // namespace kda

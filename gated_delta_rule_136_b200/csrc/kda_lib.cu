@@ -13,6 +13,7 @@
 #include <algorithm>
 #include <cstdlib>
 #include <mutex>
+#include <type_traits>
 #include <vector>
 
 #include "kda_common.cuh"
@@ -23,6 +24,7 @@
 #include "kda_plan.cuh"
 #include "kda_segment.cuh"
 #include "kda_bwd.cuh"
+#include "kda_bwd_chunk.cuh"
 
 namespace {
 // NVTX range over a host-side launch sequence (plan, chunk passes, scan, ...):
@@ -630,24 +632,39 @@ kda_status kda_spec_commit(const kda_spec_desc *desc, const void *q, const void 
 
 // ---------------------------------------------------------------- backward
 namespace {
+// dk = dv = 128: the chunked backward (kda_bwd_chunk.cuh); other head sizes:
+// the per-token backward (kda_bwd.cuh)
+bool chunked_bwd(const kda_fwd_desc &d) { return d.dk == 128 && d.dv == 128; }
+
 struct BwdLayout {
     size_t base = 0, states = 0, o = 0, fws = 0, scratch = 0, total = 0;
-    int64_t slots = 0;
+    size_t ctab = 0;               // chunked: chunk tables
+    int64_t slots = 0, chunks = 0;
     size_t fws_bytes = 0;
 };
 
 BwdLayout bwd_layout(const kda_fwd_desc &d, const int32_t *cu) {
     BwdLayout w;
-    for (int32_t n = 0; n < d.num_seqs; ++n) w.slots += ((int64_t)cu[n + 1] - cu[n]) / kda::bwd::CH;
+    for (int32_t n = 0; n < d.num_seqs; ++n) {
+        const int64_t L = (int64_t)cu[n + 1] - cu[n];
+        w.slots += L / kda::bwd::CH;
+        w.chunks += (L + kda::bwdc::C - 1) / kda::bwdc::C;
+    }
     const size_t esz = d.io_dtype == KDA_BF16 ? 2 : 4;
     const size_t DD = (size_t)d.dk * d.dv;
+    const size_t NH = (size_t)d.num_seqs * d.num_heads;
     size_t off = 0;
     w.base = off;    off += align256(sizeof(int64_t) * (size_t)(d.num_seqs + 1));
     w.states = off;  off += align256((size_t)w.slots * d.num_heads * DD * sizeof(float));
     w.o = off;       off += align256((size_t)d.total_tokens * d.num_heads * d.dv * esz);
     w.fws_bytes = fwd_workspace_bytes(&d, cu);
     w.fws = off;     off += align256(w.fws_bytes);
-    w.scratch = off; off += align256((size_t)d.num_seqs * d.num_heads * kda::bwd::scratch_floats(d.dk, d.dv) * sizeof(float));
+    if (chunked_bwd(d)) {
+        w.ctab = off;    off += align256(sizeof(int64_t) * (size_t)(d.num_seqs + 1) + 2 * sizeof(int32_t) * (size_t)w.chunks);
+        w.scratch = off; off += align256((size_t)w.chunks * d.num_heads * kda::bwdc::Scratch::FLOATS * sizeof(float));
+    } else {
+        w.scratch = off; off += align256(NH * kda::bwd::scratch_floats(d.dk, d.dv) * sizeof(float));
+    }
     w.total = off;
     return w;
 }
@@ -660,6 +677,37 @@ cudaError_t launch_bwd(const kda::bwd::BwdParams &bp, int64_t units, cudaStream_
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)units, kda::bwd::NT, SM::BYTES, stream>>>(bp);
     return cudaGetLastError();
+}
+
+template <typename TIO>
+cudaError_t launch_bwd_chunked(const kda::bwdc::ChunkBwdParams &bp, int64_t chunk_heads, int64_t units,
+                               cudaStream_t stream) {
+    using namespace kda::bwdc;
+    constexpr bool SPLIT = std::is_same<TIO, float>::value;   // 3xTF32 products for fp32 I/O
+    auto prep = chain_prep_kernel<TIO, SPLIT>;
+    auto chain = chain_kernel<SPLIT>;
+    auto grad = chain_grad_kernel<TIO, SPLIT>;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PrepSmem::BYTES)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(chain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ChainSmem::BYTES)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(grad, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GradSmem::BYTES)) != cudaSuccess)
+        return e;
+    if (chunk_heads > 0) {
+        NvtxRange r("kda.bwd.chain_prep");
+        prep<<<(unsigned)chunk_heads, NT, PrepSmem::BYTES, stream>>>(bp);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+        NvtxRange r("kda.bwd.chain");
+        chain<<<(unsigned)units, NT, ChainSmem::BYTES, stream>>>(bp);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (chunk_heads > 0) {
+        NvtxRange r("kda.bwd.chain_grad");
+        grad<<<(unsigned)chunk_heads, NT, GradSmem::BYTES, stream>>>(bp);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 template <typename TIO>
@@ -742,9 +790,41 @@ kda_status kda_chunk_bwd(const kda_fwd_desc *desc, const void *q, const void *k,
         return KDA_ERR_CUDA;
     float *states = reinterpret_cast<float *>(ws + w.states);
     const kda_snapshots sn{kda::bwd::CH, w.slots, base_dev, states};
+    const bool chunked = chunked_bwd(d);
     st = chunk_fwd_impl(desc, &sn, q, k, v, g, beta, S0, cu_seqlens, cu_seqlens_host, nullptr,
                         ws + w.o, nullptr, w.fws_bytes ? ws + w.fws : nullptr, w.fws_bytes, stream);
     if (st != KDA_OK) return st;
+
+    if (chunked) {
+        // chunk c of sequence n is chunk_base[n] + (its index in the sequence)
+        std::vector<int64_t> cbase((size_t)N + 1, 0);
+        std::vector<int32_t> cmap(2 * (size_t)w.chunks);
+        for (int32_t n = 0; n < N; ++n) {
+            const int64_t L = (int64_t)cu_seqlens_host[n + 1] - cu_seqlens_host[n];
+            const int64_t nc = (L + kda::bwdc::C - 1) / kda::bwdc::C;
+            for (int64_t ci = 0; ci < nc; ++ci) {
+                cmap[(size_t)(cbase[n] + ci)] = n;
+                cmap[(size_t)(w.chunks + cbase[n] + ci)] = (int32_t)ci;
+            }
+            cbase[n + 1] = cbase[n] + nc;
+        }
+        int64_t *cbase_dev = reinterpret_cast<int64_t *>(ws + w.ctab);
+        int32_t *cmap_dev = reinterpret_cast<int32_t *>(cbase_dev + N + 1);
+        if (cudaMemcpyAsync(cbase_dev, cbase.data(), cbase.size() * sizeof(int64_t), cudaMemcpyHostToDevice,
+                            stream) != cudaSuccess ||
+            (w.chunks > 0 && cudaMemcpyAsync(cmap_dev, cmap.data(), cmap.size() * sizeof(int32_t),
+                                             cudaMemcpyHostToDevice, stream) != cudaSuccess))
+            return KDA_ERR_CUDA;
+        kda::bwdc::ChunkBwdParams cp{q, k, v, g, beta, gate, dout, S0, dS_T, cu_seqlens, states, base_dev,
+                                     cmap_dev, cmap_dev + w.chunks, cbase_dev,
+                                     reinterpret_cast<float *>(ws + w.scratch), dq, dk, dv, dg, dbeta, dgate, dS0,
+                                     H, d.scale, d.g_floor};
+        NvtxRange r("kda.bwd");
+        const int64_t ch = w.chunks * H, units = (int64_t)N * H;
+        const cudaError_t e = d.io_dtype == KDA_BF16 ? launch_bwd_chunked<__nv_bfloat16>(cp, ch, units, stream)
+                                                     : launch_bwd_chunked<float>(cp, ch, units, stream);
+        return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
 
     kda::bwd::BwdParams bp{q, k, v, g, beta, gate, dout, S0, dS_T, cu_seqlens, states, base_dev,
                            reinterpret_cast<float *>(ws + w.scratch), dq, dk, dv, dg, dbeta, dgate, dS0,

@@ -25,13 +25,16 @@ The chain over chunks needs only dS0 from dS_C, which is affine:
     dZ = Et + Wt dS_C,   dS0 = F + e^{lgam} dS_C - Kbar^T dZ,
     Et = Diag(beta) T^T (scale A_qk^T go),  Wt = Diag(beta) T^T Khat,  F = scale Qbar^T go
 (stage 1 forms Et, Wt, F, Kbar per chunk; stage 2 runs the chain; stage 3
-forms every gradient of a chunk from its S0, S_C and dS_C).  The key-side
+forms every gradient of a chunk from its S0 and dS_C).  The key-side
 gradients in the bounded form:
     dq  = a (eR scale go S0^T + sum_j dA_qk m bf k_j)
     dk1 = a (-eR dZ S0^T + sum_j dAt m bf k_j)                      (through Kbar)
     dk2 = bf (sum_i dA_qk m a q_i + sum_i dAt m a k_i + eG nu dS_C^T)  (through Kbrev, Khat)
     dk = dk1 + dk2,   dlG_t = q dq + k (dk1 - dk2)
-    dlgam = rowsum(dS_C o S_C),   dg_s = [g_s >= floor] (sum_{t >= s} dlG_t + dlgam)
+    dlgam = e^{lgam} rowsum(dS_C o S0) + sum_t k_t dkh_t  (dkh = bf eG nu dS_C^T: the Khat part of dk2,
+            i.e. rowsum(dS_C o S_C) written with the terms dlG holds, so that their
+            cancellation inside sum_t is exact in the kernel's rounding as well)
+    dg_s = [g_s >= floor] (sum_{t >= s} dlG_t + dlgam)
     dbeta = rowsum(dY o Z) + rowsum(dA_kk o At)
 with eR[b] = e^{r_b} and eG[b] = e^{lgam - r_b}.
 """
@@ -173,12 +176,13 @@ def head_backward(q, k, v, g, beta, do, gate, S0, dS_T, scale, floor):
         dAqk = np.tril(scale * go @ ch["nu"].T)
         acc_q = eR[blk] * (scale * go @ S0c.T) + _pair(dAqk, ch["kb"], tb, "i")
         acc_k1 = -eR[blk] * (dZ @ S0c.T) + _pair(dAt, ch["kb"], tb, "i")
-        acc_k2 = (_pair(dAqk, ch["qa"], tb, "j") + _pair(dAt, ch["ka"], tb, "j")
-                  + eG[blk] * (ch["nu"] @ dSC.T))
+        dkh = bf * (eG[blk] * (ch["nu"] @ dSC.T))
+        dk2 = bf * (_pair(dAqk, ch["qa"], tb, "j") + _pair(dAt, ch["ka"], tb, "j")) + dkh
         dq = a * acc_q
-        dk1, dk2 = a * acc_k1, bf * acc_k2
+        dk1 = a * acc_k1
         dlG = ch["q"] * dq + ch["k"] * (dk1 - dk2)
-        dlgam = np.sum(dSC * ch["S_C"], axis=1)
+        # d/dlgam of S_C = e^{lgam} S0 + Khat^T nu, with the Khat part taken from dkh itself
+        dlgam = np.exp(tb["lgam"]) * np.sum(dSC * S0c, axis=1) + np.sum(ch["k"] * dkh, axis=0)
         dgc = np.cumsum(dlG[::-1], axis=0)[::-1] + dlgam[None, :]
         dg = np.where(ch["g"] >= floor, dgc, 0.0)
         dbeta = np.sum(dY * ch["Z"], axis=1) + np.sum(dAkk * ch["At"], axis=1)
