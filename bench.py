@@ -61,7 +61,7 @@ def bytes_per_token_head(dk=DK, dv=DV, esz=2):
 # DRAM traffic per unit from the ncu captures under profiles/ (bytes), valid only
 # for the kernel source they were taken from (sha1 prefix); otherwise null.
 PROFILED_TRAFFIC = {
-    "csrc/kda_chunk_tc.cuh": {"sha1": "4d8760d81e00", "bytes_per_token_head": (269.354496e6 + 53.167104e6) / 262144,
+    "csrc/kda_chunk_tc.cuh": {"sha1": "ebf32283505e", "bytes_per_token_head": (269.184768e6 + 52.762368e6) / 262144,
                               "profile": "profiles/chunk_tc_kernel_prefill_4x4096x16.md"},
     "csrc/kda_decode.cuh": {"sha1": "8e75484b34f3", "bytes_per_head_step": (273.707520e6 + 212.401408e6) / 4096,
                             "profile": "profiles/decode_kernel_64x64.md"},
@@ -69,9 +69,9 @@ PROFILED_TRAFFIC = {
     "csrc/kda_spec.cuh": {"sha1": "5f78f5eaf7b5",
                           "bytes_per_head_round": (579.116800e6 + 4.305920e6 + 555.884544e6 + 477.843968e6) / 8192,
                           "profile": "profiles/spec_kernel_verify_commit_128x64.md"},
-    # backward kernel at 2 x 1024 x 16 (bf16): per token-head (the forward with snapshots not included)
-    "csrc/kda_bwd.cuh": {"sha1": "674b7f1ed170", "bytes_per_token_head": (74.136576e6 + 30.980096e6) / 32768,
-                         "profile": "profiles/bwd_kernel_2x1024x16.md"},
+    # chunked backward's gradient kernel (chain_grad) at 1 x 4096 x 32 (bf16): per token-head
+    "csrc/kda_bwd_chunk.cuh": {"sha1": "858596339c55", "bytes_per_token_head": (630.093568e6 + 184.078336e6) / 131072,
+                               "profile": "profiles/bwd_chunk_kernels_1x4096x32.md"},
 }
 
 
@@ -614,9 +614,12 @@ def main():
                 "tokens": B * T, "ms": ms, "tokens_per_s": world * B * T / (ms / 1e3),
                 "alg_gbs": byts / (ms / 1e3) / 1e9, "roofline_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
                 "alg_bytes": byts,
-                "traffic_bwd_kernel": profiled_traffic("csrc/kda_bwd.cuh", "bytes_per_token_head", B * T * H),
-                "note": "forward with 64-token state snapshots, then per (sequence, head) a CUDA-core "
-                        "replay of each chunk and the reverse recurrence"}
+                "traffic_chain_grad_kernel": profiled_traffic("csrc/kda_bwd_chunk.cuh", "bytes_per_token_head",
+                                                              B * T * H),
+                "note": "forward with 64-token state snapshots, then the chunked backward: the gradient "
+                        "chain's per-chunk constants (a CTA per chunk x head), the chain over chunks (a CTA "
+                        "per sequence x head), every gradient of a chunk (a CTA per chunk x head); tf32 "
+                        "mma.sync products, 3xTF32 where dg's terms cancel"}
             del xb, dout
             torch.cuda.empty_cache()
 
