@@ -1,4 +1,4 @@
-// kda_bwd_chunk.cuh -- KDA backward in the chunked form (dk = dv = 128).
+// kda_bwd_chunk.cuh -- KDA backward in the chunked form (dk = dv = 128, bf16 I/O).
 //
 // The forward of one 64-token chunk with start state S0, in the chunk's frame
 // (Kimi K3 report digest, section "KDA": per-channel decay with a floor,
@@ -31,10 +31,10 @@
 //       inside sum_t match; S_C from a forward's snapshot would not),
 //       dbeta = rowsum(dY o Z) + rowsum(dA_kk o At).
 // Every product runs on the warp-level tensor cores in tf32 with fp32
-// accumulation, 3xTF32 (leading and low parts) for fp32 I/O and, for every
-// I/O dtype, for the four products (dq, dk1, dk2 and its Khat part) whose
+// accumulation; the four products (dq, dk1, dk2 and its Khat part) whose
 // outputs hold the two sides of the pair terms that cancel inside dg's sum
-// over the chunk: rounded alike, they cancel to fp32 accuracy.
+// over the chunk run in 3xTF32 (leading and low parts), so that they cancel
+// to fp32 accuracy.  SPLIT puts every other product in 3xTF32 as well.
 #pragma once
 
 #include "kda_common.cuh"

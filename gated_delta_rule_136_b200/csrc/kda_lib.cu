@@ -13,7 +13,6 @@
 #include <algorithm>
 #include <cstdlib>
 #include <mutex>
-#include <type_traits>
 #include <vector>
 
 #include "kda_common.cuh"
@@ -632,9 +631,12 @@ kda_status kda_spec_commit(const kda_spec_desc *desc, const void *q, const void 
 
 // ---------------------------------------------------------------- backward
 namespace {
-// dk = dv = 128: the chunked backward (kda_bwd_chunk.cuh); other head sizes:
-// the per-token backward (kda_bwd.cuh)
-bool chunked_bwd(const kda_fwd_desc &d) { return d.dk == 128 && d.dv == 128; }
+// bf16 I/O at dk = dv = 128: the chunked backward (kda_bwd_chunk.cuh).  Other
+// head sizes, and fp32 I/O: the per-token backward (kda_bwd.cuh), whose dg is
+// formed per token; the chunked form's dg sums the chunk's pair terms, which
+// cancel, and under strong decay (g near the floor) keeps about 3e-4 of
+// relative accuracy in fp32 arithmetic, short of fp32 I/O's 1e-4.
+bool chunked_bwd(const kda_fwd_desc &d) { return d.dk == 128 && d.dv == 128 && d.io_dtype == KDA_BF16; }
 
 struct BwdLayout {
     size_t base = 0, states = 0, o = 0, fws = 0, scratch = 0, total = 0;
@@ -679,14 +681,12 @@ cudaError_t launch_bwd(const kda::bwd::BwdParams &bp, int64_t units, cudaStream_
     return cudaGetLastError();
 }
 
-template <typename TIO>
 cudaError_t launch_bwd_chunked(const kda::bwdc::ChunkBwdParams &bp, int64_t chunk_heads, int64_t units,
                                cudaStream_t stream) {
     using namespace kda::bwdc;
-    constexpr bool SPLIT = std::is_same<TIO, float>::value;   // 3xTF32 products for fp32 I/O
-    auto prep = chain_prep_kernel<TIO, SPLIT>;
-    auto chain = chain_kernel<SPLIT>;
-    auto grad = chain_grad_kernel<TIO, SPLIT>;
+    auto prep = chain_prep_kernel<__nv_bfloat16, false>;
+    auto chain = chain_kernel<false>;
+    auto grad = chain_grad_kernel<__nv_bfloat16, false>;
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PrepSmem::BYTES)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(chain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ChainSmem::BYTES)) != cudaSuccess ||
@@ -821,8 +821,7 @@ kda_status kda_chunk_bwd(const kda_fwd_desc *desc, const void *q, const void *k,
                                      H, d.scale, d.g_floor};
         NvtxRange r("kda.bwd");
         const int64_t ch = w.chunks * H, units = (int64_t)N * H;
-        const cudaError_t e = d.io_dtype == KDA_BF16 ? launch_bwd_chunked<__nv_bfloat16>(cp, ch, units, stream)
-                                                     : launch_bwd_chunked<float>(cp, ch, units, stream);
+        const cudaError_t e = launch_bwd_chunked(cp, ch, units, stream);
         return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     }
 

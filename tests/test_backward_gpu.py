@@ -2,7 +2,8 @@
 (autograd through the token recurrence, itself pinned by finite differences):
 dq, dk, dv, dg, dbeta, dgate and dS0 for L = sum(o * dout) + sum(S_T * dS_T).
 Ragged sequences cover partial chunks and sub-blocks and an empty sequence;
-fp32 I/O runs the CUDA-core forward for the checkpoints, bf16 I/O the
+fp32 I/O runs the CUDA-core forward for the checkpoints and the per-token
+backward, bf16 I/O the
 tensor-core one."""
 import numpy as np
 import pytest
@@ -19,9 +20,9 @@ def _cpu(x):
     return None if x is None else x.detach().to("cpu")
 
 
-def _run(lengths, H, dtype, seed, gate=True, s0=True, ds_t=True, heads=None, dk=128, dv=128):
+def _run(lengths, H, dtype, seed, gate=True, s0=True, ds_t=True, heads=None, dk=128, dv=128, g_mode="softplus"):
     inp = inputs.prefill_inputs(lengths, H=H, dk=dk, dv=dv, dtype=dtype, device="cuda", seed=seed,
-                                s0_std=0.05 if s0 else None, gate=gate)
+                                s0_std=0.05 if s0 else None, gate=gate, g_mode=g_mode)
     gen = torch.Generator(device="cuda").manual_seed(seed + 1)
     dout = torch.randn(inp["v"].shape, generator=gen, device="cuda").to(dtype)
     N = len(lengths)
@@ -73,3 +74,11 @@ def test_backward_full_length_sampled_head():
     checked against the oracle over the whole sequence."""
     got, ref = _run([4096], H=32, dtype=torch.bfloat16, seed=107, heads=[5])
     _check(got, ref, torch.bfloat16)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_backward_floor_stress(dtype):
+    """g spread down to and below the floor: the 16-token block factors of the
+    chunked form reach e^{16 |floor|}, and clamped entries must pass no gradient."""
+    got, ref = _run([200, 64, 33], H=2, dtype=dtype, seed=113, g_mode="floor_stress")
+    _check(got, ref, dtype)

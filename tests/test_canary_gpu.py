@@ -2,13 +2,15 @@
 whose bytes before and after it hold a known pattern; after each call the
 pattern must be intact, so no kernel writes outside the buffers it was given.
 Covers the tensor-core prefill (ragged, gated, with S0; the long-sequence
-segment split), the CUDA-core prefill (fp32), decode and speculative
-verify/commit."""
+segment split), the CUDA-core prefill (fp32), decode, speculative
+verify/commit and the backward (chunked and per-token)."""
+import ctypes
+
 import pytest
 import torch
 
-from gated_delta_rule_136_b200 import (chunk_fwd, chunk_fwd_snapshots, decode_step, device_status,
-                                       inputs, spec_commit, spec_verify)
+from gated_delta_rule_136_b200 import (chunk_bwd, chunk_fwd, chunk_fwd_snapshots, decode_step, device_status,
+                                       inputs, kda, spec_commit, spec_verify)
 
 pytestmark = pytest.mark.gpu
 
@@ -81,4 +83,43 @@ def test_decode_and_speculative_writes_stay_in_bounds():
     acc = torch.tensor([0, 1, 2, 3, 4] * 3 + [2], dtype=torch.int32, device="cuda")
     spec_commit(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], Ss, acc)
     assert intact(rSs) and intact(rov)
+    assert device_status() == 0
+
+
+@pytest.mark.parametrize("dk,dtype", [(128, torch.bfloat16), (128, torch.float32), (64, torch.float32)])
+def test_backward_writes_stay_in_bounds(dk, dtype):
+    """kda_chunk_bwd through the C ABI with every gradient inside canaries (dk = dv = 128:
+    the chunked kernels; 64: the per-token kernel); the gradients equal the wrapper's."""
+    lengths, H = [150, 0, 70, 64], 2
+    inp = inputs.prefill_inputs(lengths, H=H, dk=dk, dv=dk, dtype=dtype, device="cuda", seed=71,
+                                s0_std=0.05, gate=True)
+    gen = torch.Generator(device="cuda").manual_seed(72)
+    dout = torch.randn(inp["v"].shape, generator=gen, device="cuda").to(dtype)
+    N, T = len(lengths), inp["q"].shape[0]
+    dS_T = 0.1 * torch.randn((N, H, dk, dk), generator=gen, device="cuda")
+    ref = chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], dout, cu_seqlens=inp["cu_seqlens"],
+                    cu_seqlens_host=inp["cu_seqlens_host"], S0=inp["S0"], gate=inp["gate"], dS_T=dS_T)
+    shapes = {"dq": (T, H, dk), "dk": (T, H, dk), "dv": (T, H, dk), "dg": (T, H, dk), "dbeta": (T, H),
+              "dgate": (T, H, dk)}
+    raws, outs = {}, {}
+    for name, shape in shapes.items():
+        raws[name], outs[name] = padded(shape, dtype)
+    raws["dS0"], outs["dS0"] = padded((N, H, dk, dk), torch.float32)
+    lib = kda.load_library()
+    desc = kda.FwdDesc(T, N, H, dk, dk, kda.KDA_BF16 if dtype == torch.bfloat16 else kda.KDA_FP32,
+                       float(inp["scale"]), -5.0, 0, 0)
+    cu_h = (ctypes.c_int32 * (N + 1))(*inp["cu_seqlens_host"])
+    ws_bytes = lib.kda_chunk_bwd_workspace_size(ctypes.byref(desc), cu_h)
+    ws = torch.empty(int(ws_bytes), dtype=torch.uint8, device="cuda")
+    vp = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    st = lib.kda_chunk_bwd(ctypes.byref(desc), vp(inp["q"]), vp(inp["k"]), vp(inp["v"]), vp(inp["g"]),
+                           vp(inp["beta"]), vp(inp["S0"]),
+                           ctypes.cast(vp(inp["cu_seqlens"]), ctypes.POINTER(ctypes.c_int32)), cu_h,
+                           vp(inp["gate"]), vp(dout), vp(dS_T), vp(outs["dq"]), vp(outs["dk"]), vp(outs["dv"]),
+                           vp(outs["dg"]), vp(outs["dbeta"]), vp(outs["dgate"]), vp(outs["dS0"]), vp(ws),
+                           ctypes.c_size_t(ws.numel()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    for name in outs:
+        assert intact(raws[name]), name
+        assert torch.equal(outs[name], ref[name]), name
     assert device_status() == 0
