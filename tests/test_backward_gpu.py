@@ -3,8 +3,8 @@
 dq, dk, dv, dg, dbeta, dgate and dS0 for L = sum(o * dout) + sum(S_T * dS_T).
 Ragged sequences cover partial chunks and sub-blocks and an empty sequence;
 fp32 I/O runs the CUDA-core forward for the checkpoints and the per-token
-backward, bf16 I/O the
-tensor-core one."""
+backward, bf16 I/O the tensor-core forward and (dk = dv = 128) the chunked
+backward."""
 import numpy as np
 import pytest
 import torch
