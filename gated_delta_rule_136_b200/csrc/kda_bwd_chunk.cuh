@@ -111,25 +111,40 @@ __device__ __forceinline__ void gemm(int warp, int w0, int nw, int lane, FK kran
         for (int n = 0; n < NT8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
         int lo, hi;
         krange(i0, j0, lo, hi);
-#pragma unroll 2
+        // fragments of the next k-step are read while the current one's MMAs issue
+        float av[4], bv[NT8][2];
+        auto fetch = [&](int k0) {
+            av[0] = fa(i0 + g, k0 + t); av[1] = fa(i0 + g + 8, k0 + t);
+            av[2] = fa(i0 + g, k0 + t + 4); av[3] = fa(i0 + g + 8, k0 + t + 4);
+#pragma unroll
+            for (int n = 0; n < NT8; ++n) {
+                bv[n][0] = fb(i0, k0 + t, j0 + 8 * n + g);
+                bv[n][1] = fb(i0, k0 + t + 4, j0 + 8 * n + g);
+            }
+        };
+        if (lo < hi) fetch(lo);
+#pragma unroll 1
         for (int k0 = lo; k0 < hi; k0 += 8) {
-            const float av[4] = {fa(i0 + g, k0 + t), fa(i0 + g + 8, k0 + t), fa(i0 + g, k0 + t + 4),
-                                 fa(i0 + g + 8, k0 + t + 4)};
-            uint32_t ah[4], al[4];
+            uint32_t ah[4], al[4], bh[NT8][2], bl[NT8][2];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 ah[e] = tf32_rna(av[e]);
                 if constexpr (SPLIT) al[e] = tf32_rna(av[e] - __uint_as_float(ah[e]));
             }
 #pragma unroll
+            for (int n = 0; n < NT8; ++n)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    bh[n][e] = tf32_rna(bv[n][e]);
+                    if constexpr (SPLIT) bl[n][e] = tf32_rna(bv[n][e] - __uint_as_float(bh[n][e]));
+                }
+            if (k0 + 8 < hi) fetch(k0 + 8);
+#pragma unroll
             for (int n = 0; n < NT8; ++n) {
-                const int j = j0 + 8 * n + g;
-                const float b0 = fb(i0, k0 + t, j), b1 = fb(i0, k0 + t + 4, j);
-                const uint32_t h0 = tf32_rna(b0), h1 = tf32_rna(b1);
-                mma_tf32(acc[n], ah, h0, h1);
+                mma_tf32(acc[n], ah, bh[n][0], bh[n][1]);
                 if constexpr (SPLIT) {
-                    mma_tf32(acc[n], ah, tf32_rna(b0 - __uint_as_float(h0)), tf32_rna(b1 - __uint_as_float(h1)));
-                    mma_tf32(acc[n], al, h0, h1);
+                    mma_tf32(acc[n], ah, bl[n][0], bl[n][1]);
+                    mma_tf32(acc[n], al, bh[n][0], bh[n][1]);
                 }
             }
         }
