@@ -37,6 +37,8 @@
 // to fp32 accuracy.  SPLIT puts every other product in 3xTF32 as well.
 #pragma once
 
+#include <type_traits>
+
 #include "kda_common.cuh"
 
 namespace kda {
@@ -303,32 +305,79 @@ struct PrepSmem {
     static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
 };
 
-// Stage the chunk's q, k (I/O dtype -> fp32) and gc = max(g, floor), zero past its end.
-template <typename TIO>
-__device__ __forceinline__ void stage_qkg(const ChunkBwdParams &p, const ChunkRef &r, int tid, float *sq,
-                                          float *sk, float *sg, float *sb) {
-    const TIO *q = static_cast<const TIO *>(p.q);
-    const TIO *k = static_cast<const TIO *>(p.k);
-    const TIO *g = static_cast<const TIO *>(p.g);
-    const int64_t H = p.num_heads;
-    for (int i = tid; i < CD; i += NT) {
-        const int t = i / D, c = i % D;
-        float qv = 0.0f, kv = 0.0f, gv = 0.0f;
-        if (t < r.Lc) {
-            const int64_t e = ((r.tok0 + t) * H + r.h) * D + c;
-            qv = ld(q, e);
-            kv = ld(k, e);
-            gv = fmaxf(ld(g, e), p.g_floor);
-        }
-        sq[xd(t, c)] = qv;
-        sk[xd(t, c)] = kv;
-        sg[xd(t, c)] = gv;
+// Loads of data that no thread writes during the launch (inputs, and what
+// earlier launches left in the scratch): the read-only path, which also lets
+// the compiler issue them ahead of the stores that follow.
+__device__ __forceinline__ float ldn(const float *p) { return __ldg(p); }
+__device__ __forceinline__ float ldn(const __nv_bfloat16 *p) { return __bfloat162float(__ldg(p)); }
+__device__ __forceinline__ float4 ldn4(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
+
+// A [C][D] bf16 tile of the chunk (rows past its end zero) as 16-byte pieces:
+// thread tid holds pieces tid and tid + NT (row = piece / 16, 8 channels from
+// (piece % 16) * 8).  The rows of a token are D = 128 bf16 = 256 bytes apart
+// within a head, and the host sends only 16-byte aligned tensors here.
+struct Tile8 {
+    uint4 v[2];
+};
+__device__ __forceinline__ Tile8 load_tile8(const __nv_bfloat16 *base, const ChunkRef &r, int64_t H, int tid) {
+    Tile8 x;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int piece = tid + u * NT, t = piece >> 4, c8 = (piece & 15) * 8;
+        x.v[u] = t < r.Lc ? __ldg(reinterpret_cast<const uint4 *>(base + ((r.tok0 + t) * H + r.h) * D + c8))
+                          : make_uint4(0u, 0u, 0u, 0u);
     }
-    if (tid < C) sb[tid] = tid < r.Lc ? ld(static_cast<const TIO *>(p.beta), (r.tok0 + tid) * H + r.h) : 0.0f;
+    return x;
+}
+__device__ __forceinline__ void unpack8(uint4 w, float (&f)[8]) {
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        f[2 * e] = __uint_as_float(u[e] << 16);
+        f[2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+    }
+}
+// 8 floats at (t, c8) of a swizzled [C][D] tile: two 4-float groups
+__device__ __forceinline__ void put8(float *tile, int t, int c8, const float (&f)[8]) {
+    *reinterpret_cast<float4 *>(tile + xd(t, c8)) = make_float4(f[0], f[1], f[2], f[3]);
+    *reinterpret_cast<float4 *>(tile + xd(t, c8 + 4)) = make_float4(f[4], f[5], f[6], f[7]);
+}
+
+// Stage the chunk's q, k (bf16 -> fp32) and gc = max(g, floor), zero past its end;
+// with `mask`, bit c % 32 of mask[t * 4 + c / 32] = [g_tc >= floor].
+__device__ __forceinline__ void stage_qkg(const ChunkBwdParams &p, const ChunkRef &r, int tid, float *sq,
+                                          float *sk, float *sg, float *sb, uint32_t *mask) {
+    const int64_t H = p.num_heads;
+    const Tile8 tq = load_tile8(static_cast<const __nv_bfloat16 *>(p.q), r, H, tid);
+    const Tile8 tk = load_tile8(static_cast<const __nv_bfloat16 *>(p.k), r, H, tid);
+    const Tile8 tg = load_tile8(static_cast<const __nv_bfloat16 *>(p.g), r, H, tid);
+    const float bt = tid < r.Lc ? ldn(static_cast<const __nv_bfloat16 *>(p.beta) + (r.tok0 + tid) * H + r.h) : 0.0f;
+    if (mask && tid < C * D / 32) mask[tid] = 0u;
+    if (mask) __syncthreads();
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int piece = tid + u * NT, t = piece >> 4, c8 = (piece & 15) * 8;
+        float f[8];
+        unpack8(tq.v[u], f);
+        put8(sq, t, c8, f);
+        unpack8(tk.v[u], f);
+        put8(sk, t, c8, f);
+        unpack8(tg.v[u], f);
+        uint32_t bits = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            if (t < r.Lc && f[e] >= p.g_floor) bits |= 1u << e;
+            f[e] = t < r.Lc ? fmaxf(f[e], p.g_floor) : 0.0f;
+        }
+        put8(sg, t, c8, f);
+        if (mask) atomicOr(mask + t * (D / 32) + (c8 >> 5), bits << (c8 & 31));
+    }
+    if (tid < C) sb[tid] = bt;
 }
 
 template <typename TIO, bool SPLIT>
 __global__ void __launch_bounds__(NT, 1) chain_prep_kernel(ChunkBwdParams p) {
+    static_assert(std::is_same<TIO, __nv_bfloat16>::value, "the chunked backward reads bf16 in 16-byte pieces");
     using S = PrepSmem;
     extern __shared__ float4 bwdc_smem4[];
     float *sm = reinterpret_cast<float *>(bwdc_smem4);
@@ -346,7 +395,7 @@ __global__ void __launch_bounds__(NT, 1) chain_prep_kernel(ChunkBwdParams p) {
     const float scale = p.scale;
 
     // q -> qa, k -> ka (and kb), gc -> a (in b3)
-    stage_qkg<TIO>(p, r, tid, qa, ka, b3, sb);
+    stage_qkg(p, r, tid, qa, ka, b3, sb, nullptr);
     __syncthreads();
     decay_tables(tid, b3, b3, m, eR, eG, gam);
     __syncthreads();
@@ -373,9 +422,9 @@ __global__ void __launch_bounds__(NT, 1) chain_prep_kernel(ChunkBwdParams p) {
     gemm<C, D, 4, SPLIT>(warp, 0, NW, lane,
         [&](int, int, int &lo, int &hi) { lo = 0; hi = S0p ? D : 0; },
         [&](int i, int c) { return ka[xd(i, c)] * eR[(i >> 4) * D + c]; },
-        [&](int, int c, int v) { return S0p[c * D + v]; },
+        [&](int, int c, int v) { return ldn(S0p + c * D + v); },
         [&](int i, int v, float x) {
-            const float vi = i < r.Lc ? ld(vin, ((r.tok0 + i) * H + r.h) * D + v) : 0.0f;
+            const float vi = i < r.Lc ? ldn(vin + ((r.tok0 + i) * H + r.h) * D + v) : 0.0f;
             const float z = vi - x;
             b3[xd(i, v)] = z;
             scr[Scratch::Z + i * D + v] = z;
@@ -407,14 +456,14 @@ __global__ void __launch_bounds__(NT, 1) chain_prep_kernel(ChunkBwdParams p) {
     gemm<C, D, 4, SPLIT>(warp, 0, NW, lane,
         [&](int i0, int, int &lo, int &hi) { lo = S0p ? 0 : D; hi = D + i0 + 16; },
         [&](int i, int k) { return k < D ? qa[xd(i, k)] * eR[(i >> 4) * D + k] : Aq[xc(i, k - D)]; },
-        [&](int, int k, int v) { return k < D ? S0p[k * D + v] : nu[xd(k - D, v)]; },
+        [&](int, int k, int v) { return k < D ? ldn(S0p + k * D + v) : nu[xd(k - D, v)]; },
         [&](int i, int v, float x) {
             float go = 0.0f;
             if (i < r.Lc) {
                 const int64_t e = ((r.tok0 + i) * H + r.h) * D + v;
-                const float dov = ld(dout, e);
+                const float dov = ldn(dout + e);
                 if (gate) {
-                    const float sg = sigmoidf(ld(gate, e));
+                    const float sg = sigmoidf(ldn(gate + e));
                     st(static_cast<TIO *>(p.dgate), e, dov * scale * x * sg * (1.0f - sg));
                     go = dov * sg;
                 } else {
@@ -513,12 +562,13 @@ struct GradSmem {
     static constexpr int B0 = 0, B1 = B0 + CD, B2 = B1 + CD, B3 = B2 + CD, B4 = B3 + CD;
     static constexpr int TT = B4 + CD, S1 = TT + CC, S2 = S1 + CC;
     static constexpr int M = S2 + CC, ER = M + NB * NB * D, EG = ER + NB * D, GM = EG + NB * D;
-    static constexpr int BT = GM + D, DL = BT + C, FLOATS = DL + D;
+    static constexpr int BT = GM + D, DL = BT + C, MK = DL + D, FLOATS = MK + C * D / 32;
     static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
 };
 
 template <typename TIO, bool SPLIT>
 __global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
+    static_assert(std::is_same<TIO, __nv_bfloat16>::value, "the chunked backward reads bf16 in 16-byte pieces");
     using S = GradSmem;
     extern __shared__ float4 bwdc_smem4[];
     float *sm = reinterpret_cast<float *>(bwdc_smem4);
@@ -526,6 +576,7 @@ __global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
     float *Tm = sm + S::TT, *s1 = sm + S::S1, *s2 = sm + S::S2;
     float *m = sm + S::M, *eR = sm + S::ER, *eG = sm + S::EG, *gam = sm + S::GM, *sb = sm + S::BT;
     float *sdl = sm + S::DL;
+    uint32_t *gmask = reinterpret_cast<uint32_t *>(sm + S::MK);   // [g >= floor] bits, [C][D / 32]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const ChunkRef r = chunk_ref(p);
     const int64_t H = p.num_heads;
@@ -534,37 +585,57 @@ __global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
     const float *dSC = scr + Scratch::DSC;
     const TIO *qin = static_cast<const TIO *>(p.q);
     const TIO *kin = static_cast<const TIO *>(p.k);
-    const TIO *gin = static_cast<const TIO *>(p.g);
-    const TIO *dout = static_cast<const TIO *>(p.dout);
     const TIO *gate = static_cast<const TIO *>(p.gate);
     const float scale = p.scale;
     auto row = [&](int i) { return ((r.tok0 + i) * H + r.h) * D; };
 
-    // q -> qa, k -> kb, gc -> lG tables (a into aa)
-    stage_qkg<TIO>(p, r, tid, qa, kb, b4, sb);
-    for (int i = tid; i < CC; i += NT) Tm[xc(i / C, i % C)] = scr[Scratch::T + i];
+    // every load first: dout and the gate, T and A_qk, then q, k, g (staged); the
+    // decay tables (a into aa); qa, kb, and go = dout sigmoid(z) into b3
+    const Tile8 tdo = load_tile8(static_cast<const __nv_bfloat16 *>(p.dout), r, H, tid);
+    Tile8 tz;
+    if (gate) tz = load_tile8(static_cast<const __nv_bfloat16 *>(p.gate), r, H, tid);
+    {
+        float4 tt[2], ta[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            tt[u] = ldn4(scr + Scratch::T + 4 * (tid + u * NT));
+            ta[u] = ldn4(scr + Scratch::AQK + 4 * (tid + u * NT));
+        }
+        stage_qkg(p, r, tid, qa, kb, b4, sb, gmask);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int i = 4 * (tid + u * NT), a = i / C, b = i % C;
+            *reinterpret_cast<float4 *>(Tm + xc(a, b)) = tt[u];
+            *reinterpret_cast<float4 *>(s2 + xc(a, b)) = ta[u];      // A_qk, for dnu
+        }
+    }
     __syncthreads();
     decay_tables(tid, b4, aa, m, eR, eG, gam);
     __syncthreads();
     for (int i = tid; i < CD; i += NT) {
-        const int t = i / D, c = i % D, x = xd(t, c);
+        const int x = xd(i / D, i % D);
         const float a = aa[x];
         qa[x] *= a;
         kb[x] /= a;
-        float go = 0.0f;
-        if (t < r.Lc) {
-            const int64_t e = row(t) + c;
-            go = ld(dout, e);
-            if (gate) go *= sigmoidf(ld(gate, e));
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int piece = tid + u * NT, t = piece >> 4, c8 = (piece & 15) * 8;
+        float f[8];
+        unpack8(tdo.v[u], f);
+        if (gate) {
+            float z[8];
+            unpack8(tz.v[u], z);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] *= sigmoidf(z[e]);
         }
-        b3[x] = go;
+        put8(b3, t, c8, f);
     }
     __syncthreads();
-    // dnu = scale A_qk^T go + Khat dS_C (into b4)
-    const float *Aqk = scr + Scratch::AQK;
+    // dnu = scale A_qk^T go + Khat dS_C (into b4; A_qk staged in s2)
     gemm<C, D, 4, SPLIT>(warp, 0, NW, lane, [](int i0, int, int &lo, int &hi) { lo = i0; hi = C + D; },
-        [&](int j, int k) { return k < C ? scale * Aqk[k * C + j] : kb[xd(j, k - C)] * eG[(j >> 4) * D + k - C]; },
-        [&](int, int k, int v) { return k < C ? b3[xd(k, v)] : dSC[(k - C) * D + v]; },
+        [&](int j, int k) { return k < C ? scale * s2[xc(k, j)] : kb[xd(j, k - C)] * eG[(j >> 4) * D + k - C]; },
+        [&](int, int k, int v) { return k < C ? b3[xd(k, v)] : ldn(dSC + (k - C) * D + v); },
         [&](int j, int v, float x) { b4[xd(j, v)] = x; });
     __syncthreads();
     // dY = T^T dnu: dv = Diag(beta) dY, dY to scratch;  dT = dnu (Diag(beta) Z)^T (into s1)
@@ -578,7 +649,7 @@ __global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
         });
     gemm<C, C, 4, SPLIT>(warp, 0, NW, lane, [](int i0, int j0, int &lo, int &hi) { lo = 0; hi = j0 > i0 + 15 ? 0 : D; },
         [&](int i, int v) { return b4[xd(i, v)]; },
-        [&](int, int v, int j) { return sb[j] * Zg[j * D + v]; },
+        [&](int, int v, int j) { return sb[j] * ldn(Zg + j * D + v); },
         [&](int i, int j, float x) { s1[xc(i, j)] = x; });
     __syncthreads();
     // X = dT T^T (into s2), then dA_kk = -T^T X, j < i (into s1)
@@ -596,7 +667,7 @@ __global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
     const float *nug = scr + Scratch::NU;
     gemm<C, C, 4, SPLIT>(warp, 0, NW, lane, [](int i0, int j0, int &lo, int &hi) { lo = 0; hi = j0 > i0 + 15 ? 0 : D; },
         [&](int i, int v) { return b3[xd(i, v)]; },
-        [&](int, int v, int j) { return nug[j * D + v]; },
+        [&](int, int v, int j) { return ldn(nug + j * D + v); },
         [&](int i, int j, float x) { s2[xc(i, j)] = j <= i ? scale * x : 0.0f; });
     __syncthreads();
     // dbeta = rowsum(dY o Z) + rowsum(dA_kk o At): a warp per row
@@ -605,9 +676,9 @@ __global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
         for (int i = warp; i < r.Lc; i += NW) {
             float s = 0.0f;
 #pragma unroll
-            for (int e = 0; e < D / 32; ++e) s = fmaf(dYg[i * D + lane + 32 * e], Zg[i * D + lane + 32 * e], s);
+            for (int e = 0; e < D / 32; ++e) s = fmaf(dYg[i * D + lane + 32 * e], ldn(Zg + i * D + lane + 32 * e), s);
 #pragma unroll
-            for (int e = 0; e < C / 32; ++e) s = fmaf(s1[xc(i, lane + 32 * e)], Atg[i * C + lane + 32 * e], s);
+            for (int e = 0; e < C / 32; ++e) s = fmaf(s1[xc(i, lane + 32 * e)], ldn(Atg + i * C + lane + 32 * e), s);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
             if (lane == 0) st(static_cast<TIO *>(p.dbeta), (r.tok0 + i) * H + r.h, s);
@@ -616,7 +687,7 @@ __global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
     // dq = a (e^r scale go S0^T + dA_qk m kb); q dq into b4 (dlG)
     auto kr_pair = [&](int i0, int, int &lo, int &hi) { lo = S0p ? 0 : D; hi = D + i0 + 16; };
     auto fb_pair = [&](int i0, int k, int c) {
-        return k < D ? S0p[c * D + k] * eR[(i0 >> 4) * D + c]
+        return k < D ? ldn(S0p + c * D + k) * eR[(i0 >> 4) * D + c]
                      : m[((i0 >> 4) * NB + ((k - D) >> 4)) * D + c] * kb[xd(k - D, c)];
     };
     gemm<C, D, 4, true>(warp, 0, NW, lane, kr_pair,
@@ -626,7 +697,7 @@ __global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
             float ql = 0.0f;
             if (i < r.Lc) {
                 st(static_cast<TIO *>(p.dq), row(i) + c, dq);
-                ql = ld(qin, row(i) + c);
+                ql = ldn(qin + row(i) + c);
             }
             b4[xd(i, c)] = ql * dq;
         });
@@ -639,7 +710,7 @@ __global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
             const int e = xd(i, c);
             const float d1 = aa[e] * x;
             b3[e] = d1;
-            if (i < r.Lc) b4[e] += ld(kin, row(i) + c) * d1;
+            if (i < r.Lc) b4[e] += ldn(kin + row(i) + c) * d1;
         });
     __syncthreads();
     // dk2 through Kbrev: bf (dA_qk^T m qa + (Diag(beta) dA_kk)^T m ka); b3 <- dk1 + that
@@ -654,33 +725,45 @@ __global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
             const int e = xd(j, c);
             const float d2 = x / aa[e];
             b3[e] += d2;
-            if (j < r.Lc) b4[e] -= ld(kin, row(j) + c) * d2;
+            if (j < r.Lc) b4[e] -= ldn(kin + row(j) + c) * d2;
         });
     // dkh = bf e^{lgam - r} nu dS_C^T (through Khat): dk = b3 + dkh; k dkh into b3 for dlgam
     gemm<C, D, 4, true>(warp, 0, NW, lane, [](int, int, int &lo, int &hi) { lo = 0; hi = D; },
-        [&](int j, int v) { return nug[j * D + v]; },
-        [&](int j0, int v, int c) { return dSC[c * D + v] * eG[(j0 >> 4) * D + c]; },
+        [&](int j, int v) { return ldn(nug + j * D + v); },
+        [&](int j0, int v, int c) { return ldn(dSC + c * D + v) * eG[(j0 >> 4) * D + c]; },
         [&](int j, int c, float x) {
             const int e = xd(j, c);
             const float dh = x / aa[e];
             float kdh = 0.0f;
             if (j < r.Lc) {
                 st(static_cast<TIO *>(p.dk), row(j) + c, b3[e] + dh);
-                kdh = ld(kin, row(j) + c) * dh;
+                kdh = ldn(kin + row(j) + c) * dh;
                 b4[e] -= kdh;
             }
             b3[e] = kdh;
         });
-    // e^{lgam} rowsum(dS_C o S0): a warp per 8 channels
-    for (int c = warp; c < D; c += NW) {
-        float s = 0.0f;
+    // e^{lgam} rowsum(dS_C o S0): warp w the channels w + 16 n, a float4 of each row per lane
+    {
+        float rs[D / NW];
         if (S0p) {
+            float4 xa[D / NW], xb[D / NW];
 #pragma unroll
-            for (int e = 0; e < D / 32; ++e) s = fmaf(dSC[c * D + lane + 32 * e], S0p[c * D + lane + 32 * e], s);
+            for (int n = 0; n < D / NW; ++n) {
+                xa[n] = ldn4(dSC + (warp + NW * n) * D + 4 * lane);
+                xb[n] = ldn4(S0p + (warp + NW * n) * D + 4 * lane);
+            }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+            for (int n = 0; n < D / NW; ++n) {
+                float s = xa[n].x * xb[n].x + xa[n].y * xb[n].y + xa[n].z * xb[n].z + xa[n].w * xb[n].w;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                rs[n] = s;
+            }
         }
-        if (lane == 0) sdl[c] = gam[c] * s;
+        if (lane == 0) {
+#pragma unroll
+            for (int n = 0; n < D / NW; ++n) sdl[warp + NW * n] = S0p ? gam[warp + NW * n] * rs[n] : 0.0f;
+        }
     }
     __syncthreads();
     // dg_s = [g_s >= floor] (sum_{t >= s} dlG_t + dlgam), one channel per thread
@@ -692,7 +775,8 @@ __global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
             run += b4[xd(t, c)];
             if (t < r.Lc) {
                 const int64_t e = row(t) + c;
-                st(static_cast<TIO *>(p.dg), e, ld(gin, e) >= p.g_floor ? run : 0.0f);
+                const bool pass = (gmask[t * (D / 32) + (c >> 5)] >> (c & 31)) & 1u;
+                st(static_cast<TIO *>(p.dg), e, pass ? run : 0.0f);
             }
         }
     }

@@ -13,6 +13,7 @@
 #include <algorithm>
 #include <cstdlib>
 #include <mutex>
+#include <initializer_list>
 #include <vector>
 
 #include "kda_common.cuh"
@@ -636,7 +637,14 @@ namespace {
 // formed per token; the chunked form's dg sums the chunk's pair terms, which
 // cancel, and under strong decay (g near the floor) keeps about 3e-4 of
 // relative accuracy in fp32 arithmetic, short of fp32 I/O's 1e-4.
+// The chunked kernels also read q, k, g, dout and the gate in 16-byte pieces.
 bool chunked_bwd(const kda_fwd_desc &d) { return d.dk == 128 && d.dv == 128 && d.io_dtype == KDA_BF16; }
+bool chunked_bwd_applies(const kda_fwd_desc &d, std::initializer_list<const void *> ptrs) {
+    if (!chunked_bwd(d)) return false;
+    for (const void *ptr : ptrs)
+        if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return false;
+    return true;
+}
 
 struct BwdLayout {
     size_t base = 0, states = 0, o = 0, fws = 0, scratch = 0, total = 0;
@@ -661,12 +669,15 @@ BwdLayout bwd_layout(const kda_fwd_desc &d, const int32_t *cu) {
     w.o = off;       off += align256((size_t)d.total_tokens * d.num_heads * d.dv * esz);
     w.fws_bytes = fwd_workspace_bytes(&d, cu);
     w.fws = off;     off += align256(w.fws_bytes);
+    // the per-token kernel's scratch, or (chunked shape) the larger of it and the
+    // chunked kernels' (the per-token kernel also runs the chunked shape when a
+    // tensor is not 16-byte aligned)
+    size_t scratch = NH * kda::bwd::scratch_floats(d.dk, d.dv) * sizeof(float);
     if (chunked_bwd(d)) {
         w.ctab = off;    off += align256(sizeof(int64_t) * (size_t)(d.num_seqs + 1) + 2 * sizeof(int32_t) * (size_t)w.chunks);
-        w.scratch = off; off += align256((size_t)w.chunks * d.num_heads * kda::bwdc::Scratch::FLOATS * sizeof(float));
-    } else {
-        w.scratch = off; off += align256(NH * kda::bwd::scratch_floats(d.dk, d.dv) * sizeof(float));
+        scratch = std::max(scratch, (size_t)w.chunks * d.num_heads * kda::bwdc::Scratch::FLOATS * sizeof(float));
     }
+    w.scratch = off; off += align256(scratch);
     w.total = off;
     return w;
 }
@@ -790,7 +801,7 @@ kda_status kda_chunk_bwd(const kda_fwd_desc *desc, const void *q, const void *k,
         return KDA_ERR_CUDA;
     float *states = reinterpret_cast<float *>(ws + w.states);
     const kda_snapshots sn{kda::bwd::CH, w.slots, base_dev, states};
-    const bool chunked = chunked_bwd(d);
+    const bool chunked = chunked_bwd_applies(d, {q, k, g, dout, gate});
     st = chunk_fwd_impl(desc, &sn, q, k, v, g, beta, S0, cu_seqlens, cu_seqlens_host, nullptr,
                         ws + w.o, nullptr, w.fws_bytes ? ws + w.fws : nullptr, w.fws_bytes, stream);
     if (st != KDA_OK) return st;

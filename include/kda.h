@@ -312,9 +312,17 @@ kda_status kda_chunk_fwd_host(const kda_fwd_desc *desc, const void *q, const voi
  * S0, dS_T and dS0 must be 16-byte aligned.
  * The derivative of max(g, g_floor) is taken as 1 where g >= g_floor.
  * cu_seqlens_host is required.  Internally the forward runs once with state
- * snapshots every 64 tokens into the workspace, then one CTA per (sequence,
- * head) recomputes each chunk's states from its snapshot and runs the
- * recurrence backwards.  Workspace (device, 256-byte aligned):
+ * snapshots every 64 tokens into the workspace.  Then, for bf16 I/O with
+ * dk = dv = 128 and 16-byte aligned q, k, g, dout and gate, the chunked form:
+ * per 64-token chunk the gradient chain's constants, the chain over the
+ * chunks (a CTA per sequence and head), and every gradient of a chunk from its
+ * start state and the gradient reaching its end (tensor-core products);
+ * otherwise (fp32 I/O, other head sizes, unaligned tensors) one CTA per
+ * (sequence, head) recomputes each chunk's states from its snapshot and runs
+ * the recurrence backwards token by token.  The results match the gradients
+ * of the token recurrence within the parity tolerances (largest error over the
+ * output's RMS: fp32 I/O 1e-4; bf16 I/O 2e-2 beyond half a bf16 ulp).  Workspace
+ * (device, 256-byte aligned):
  * kda_chunk_bwd_workspace_size(desc, cu_seqlens_host) bytes (SIZE_MAX for a
  * bad descriptor).  dk, dv in {64, 128}, else KDA_ERR_UNSUPPORTED;
  * KDA_ERR_INVALID_ARG for null, overlapping or inconsistent arguments,
