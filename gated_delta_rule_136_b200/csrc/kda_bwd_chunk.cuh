@@ -727,10 +727,32 @@ __global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
             b3[e] += d2;
             if (j < r.Lc) b4[e] -= ldn(kin + row(j) + c) * d2;
         });
+    __syncthreads();
+    // nu and dS_C into shared memory (qa, kb and the small tiles are done with): nu over
+    // s1 | s2, dS_C over qa | kb
+    float *snu = s1, *sds = qa;
+    {
+        float4 xn[CD / 4 / NT], xs[DD / 4 / NT];
+#pragma unroll
+        for (int u = 0; u < CD / 4 / NT; ++u) xn[u] = ldn4(nug + 4 * (tid + u * NT));
+#pragma unroll
+        for (int u = 0; u < DD / 4 / NT; ++u) xs[u] = ldn4(dSC + 4 * (tid + u * NT));
+#pragma unroll
+        for (int u = 0; u < CD / 4 / NT; ++u) {
+            const int i = 4 * (tid + u * NT);
+            *reinterpret_cast<float4 *>(snu + xd(i / D, i % D)) = xn[u];
+        }
+#pragma unroll
+        for (int u = 0; u < DD / 4 / NT; ++u) {
+            const int i = 4 * (tid + u * NT);
+            *reinterpret_cast<float4 *>(sds + xd(i / D, i % D)) = xs[u];
+        }
+    }
+    __syncthreads();
     // dkh = bf e^{lgam - r} nu dS_C^T (through Khat): dk = b3 + dkh; k dkh into b3 for dlgam
     gemm<C, D, 4, true>(warp, 0, NW, lane, [](int, int, int &lo, int &hi) { lo = 0; hi = D; },
-        [&](int j, int v) { return ldn(nug + j * D + v); },
-        [&](int j0, int v, int c) { return ldn(dSC + c * D + v) * eG[(j0 >> 4) * D + c]; },
+        [&](int j, int v) { return snu[xd(j, v)]; },
+        [&](int j0, int v, int c) { return sds[xd(c, v)] * eG[(j0 >> 4) * D + c]; },
         [&](int j, int c, float x) {
             const int e = xd(j, c);
             const float dh = x / aa[e];
