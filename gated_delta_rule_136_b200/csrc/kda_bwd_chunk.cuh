@@ -495,64 +495,81 @@ __global__ void __launch_bounds__(NT, 1) chain_prep_kernel(ChunkBwdParams p) {
         [&](int i, int c, float x) { scr[Scratch::WT + i * D + c] = sb[i] * x; });
 }
 
-// shared memory of chain: dS [D][D], dZ, Wt, Kbar [C][D], e^{lgam}
+// The chain: a CTA per (sequence, head, half of the value columns).  dS's
+// columns do not mix (dZ = Et + Wt dS_C and dS0 = F + e^{lgam} dS_C - Kbar^T dZ
+// act on every column alike), so two CTAs of 256 threads take 64 columns each,
+// two per SM.  Shared memory: dS [D][64], dZ [C][64], Wt and Kbar [C][D], e^{lgam}.
+constexpr int CHAIN_NT = 256, CHAIN_NW = CHAIN_NT / 32, DVH = D / 2;
 struct ChainSmem {
-    static constexpr int DS = 0, DZ = DS + DD, WT = DZ + CD, KB = WT + CD, GM = KB + CD;
+    static constexpr int DS = 0, DZ = DS + D * DVH, WT = DZ + C * DVH, KB = WT + CD, GM = KB + CD;
     static constexpr int FLOATS = GM + D;
     static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
 };
+// swizzled offsets of a row-major tile with 64 columns (as xc)
+__device__ __forceinline__ int xh(int r, int c) { return xc(r, c); }
 
 template <bool SPLIT>
-__global__ void __launch_bounds__(NT, 1) chain_kernel(ChunkBwdParams p) {
+__global__ void __launch_bounds__(CHAIN_NT, 2) chain_kernel(ChunkBwdParams p) {
     using S = ChainSmem;
+    constexpr int NTC = CHAIN_NT;
     extern __shared__ float4 bwdc_smem4[];
     float *sm = reinterpret_cast<float *>(bwdc_smem4);
     float *dS = sm + S::DS, *dZ = sm + S::DZ, *Wt = sm + S::WT, *Kb = sm + S::KB, *gam = sm + S::GM;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t H = p.num_heads, n = blockIdx.x / H, h = blockIdx.x % H;
+    const int64_t H = p.num_heads, unit = blockIdx.x >> 1, n = unit / H, h = unit % H;
+    const int v0 = (blockIdx.x & 1) * DVH;
     const int64_t L = (int64_t)p.cu_seqlens[n + 1] - p.cu_seqlens[n];
     const int64_t nch = (L + C - 1) / C;
     const float *dST = p.dS_T ? p.dS_T + (n * H + h) * DD : nullptr;
-    for (int i = tid; i < DD; i += NT) {
-        const int c = i / D, v = i % D;
-        dS[xd(c, v)] = dST ? dST[i] : 0.0f;
+    for (int i = tid; i < D * DVH / 4; i += NTC) {        // float4 pieces of this half
+        const int c = i / (DVH / 4), v = (i % (DVH / 4)) * 4;
+        *reinterpret_cast<float4 *>(dS + xh(c, v)) = dST ? ldn4(dST + c * D + v0 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     for (int64_t ci = nch - 1; ci >= 0; --ci) {
         float *scr = p.scratch + ((p.chunk_base[n] + ci) * H + h) * Scratch::FLOATS;
         float *dsc = scr + Scratch::DSC;
         __syncthreads();
-        for (int i = tid; i < DD; i += NT) {
-            const int c = i / D, v = i % D;
-            dsc[i] = dS[xd(c, v)];
+        {
+            float4 xw[CD / 4 / NTC], xk[CD / 4 / NTC];
+#pragma unroll
+            for (int u = 0; u < CD / 4 / NTC; ++u) {
+                xw[u] = ldn4(scr + Scratch::WT + 4 * (tid + u * NTC));
+                xk[u] = ldn4(scr + Scratch::KBAR + 4 * (tid + u * NTC));
+            }
+            for (int i = tid; i < D * DVH / 4; i += NTC) {
+                const int c = i / (DVH / 4), v = (i % (DVH / 4)) * 4;
+                *reinterpret_cast<float4 *>(dsc + c * D + v0 + v) = *reinterpret_cast<const float4 *>(dS + xh(c, v));
+            }
+#pragma unroll
+            for (int u = 0; u < CD / 4 / NTC; ++u) {
+                const int i = 4 * (tid + u * NTC);
+                *reinterpret_cast<float4 *>(Wt + xd(i / D, i % D)) = xw[u];
+                *reinterpret_cast<float4 *>(Kb + xd(i / D, i % D)) = xk[u];
+            }
+            if (tid < D) gam[tid] = ldn(scr + Scratch::GAM + tid);
         }
-        for (int i = tid; i < CD; i += NT) {
-            const int j = i / D, c = i % D;
-            Wt[xd(j, c)] = scr[Scratch::WT + i];
-            Kb[xd(j, c)] = scr[Scratch::KBAR + i];
-        }
-        if (tid < D) gam[tid] = scr[Scratch::GAM + tid];
         __syncthreads();
-        // dZ = Et + Wt dS
-        gemm<C, D, 4, SPLIT>(warp, 0, NW, lane, [](int, int, int &lo, int &hi) { lo = 0; hi = D; },
+        // dZ = Et + Wt dS (this half's columns)
+        gemm<C, DVH, 4, SPLIT>(warp, 0, CHAIN_NW, lane, [](int, int, int &lo, int &hi) { lo = 0; hi = D; },
             [&](int j, int c) { return Wt[xd(j, c)]; },
-            [&](int, int c, int v) { return dS[xd(c, v)]; },
-            [&](int j, int v, float x) { dZ[xd(j, v)] = scr[Scratch::ET + j * D + v] + x; });
+            [&](int, int c, int v) { return dS[xh(c, v)]; },
+            [&](int j, int v, float x) { dZ[xh(j, v)] = ldn(scr + Scratch::ET + j * D + v0 + v) + x; });
         __syncthreads();
         // dS <- F + e^{lgam} dS - Kbar^T dZ (each element read and written by its own thread)
-        gemm<D, D, 4, SPLIT>(warp, 0, NW, lane, [](int, int, int &lo, int &hi) { lo = 0; hi = C; },
+        gemm<D, DVH, 4, SPLIT>(warp, 0, CHAIN_NW, lane, [](int, int, int &lo, int &hi) { lo = 0; hi = C; },
             [&](int c, int j) { return Kb[xd(j, c)]; },
-            [&](int, int j, int v) { return dZ[xd(j, v)]; },
+            [&](int, int j, int v) { return dZ[xh(j, v)]; },
             [&](int c, int v, float x) {
-                const int e = xd(c, v);
-                dS[e] = scr[Scratch::F + c * D + v] + gam[c] * dS[e] - x;
+                const int e = xh(c, v);
+                dS[e] = ldn(scr + Scratch::F + c * D + v0 + v) + gam[c] * dS[e] - x;
             });
     }
     __syncthreads();
     if (p.dS0) {
         float *out = p.dS0 + (n * H + h) * DD;
-        for (int i = tid; i < DD; i += NT) {
-            const int c = i / D, v = i % D;
-            out[i] = dS[xd(c, v)];
+        for (int i = tid; i < D * DVH / 4; i += NTC) {
+            const int c = i / (DVH / 4), v = (i % (DVH / 4)) * 4;
+            *reinterpret_cast<float4 *>(out + c * D + v0 + v) = *reinterpret_cast<const float4 *>(dS + xh(c, v));
         }
     }
 }

@@ -710,7 +710,7 @@ cudaError_t launch_bwd_chunked(const kda::bwdc::ChunkBwdParams &bp, int64_t chun
     }
     {
         NvtxRange r("kda.bwd.chain");
-        chain<<<(unsigned)units, NT, ChainSmem::BYTES, stream>>>(bp);
+        chain<<<(unsigned)(2 * units), CHAIN_NT, ChainSmem::BYTES, stream>>>(bp);   // two column halves
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (chunk_heads > 0) {
