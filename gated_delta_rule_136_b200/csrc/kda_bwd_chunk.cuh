@@ -198,42 +198,41 @@ __device__ __forceinline__ const float *start_state(const ChunkBwdParams &p, con
 // m[bi][bj] = e^{r_bi - r_bj} (bi >= bj, else 0), eR[b] = e^{r_b},
 // eG[b] = e^{lgam - r_b}, gam = e^{lgam}.  Every exponent is a sum of at most
 // 16 terms or of block totals, never a difference of long running sums.
-// Threads 0 .. D-1, one channel each.
+// Thread (b, c) = (tid / D, tid % D) runs block b of channel c; the block
+// totals meet in eG's rows.  Every thread of the CTA calls it (block barriers).
 __device__ __forceinline__ void decay_tables(int tid, float *gc, float *a_out, float *m, float *eR,
                                              float *eG, float *gam) {
-    if (tid >= D) return;
-    const int c = tid;
-    float tot[NB];                       // block totals of gc
+    static_assert(NT == NB * D, "one thread per (block, channel)");
+    const int c = tid % D, b = tid / D;
+    float x = 0.0f;
 #pragma unroll
-    for (int b = 0; b < NB; ++b) {
-        float x = 0.0f;
-#pragma unroll 4
-        for (int t = 16 * b; t < 16 * b + 16; ++t) {
-            x += gc[xd(t, c)];
-            a_out[xd(t, c)] = expf(x);
-        }
-        tot[b] = x;
+    for (int t = 16 * b; t < 16 * b + 16; ++t) {
+        x += gc[xd(t, c)];
+        a_out[xd(t, c)] = expf(x);
     }
+    eG[b * D + c] = x;                   // block total, for a moment
+    __syncthreads();
+    float tot[NB];
 #pragma unroll
-    for (int bi = 0; bi < NB; ++bi) {
-        float r = 0.0f, rest = 0.0f;
+    for (int bb = 0; bb < NB; ++bb) tot[bb] = eG[bb * D + c];
+    __syncthreads();
+    float r = 0.0f, rest = 0.0f;
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-            if (b < bi) r += tot[b];
-            else rest += tot[b];
-        }
-        eR[bi * D + c] = expf(r);
-        eG[bi * D + c] = expf(rest);
-#pragma unroll
-        for (int bj = 0; bj < NB; ++bj) {
-            float x = 0.0f;
-#pragma unroll
-            for (int b = 0; b < NB; ++b)
-                if (b >= bj && b < bi) x += tot[b];
-            m[(bi * NB + bj) * D + c] = bj <= bi ? expf(x) : 0.0f;
-        }
+    for (int bb = 0; bb < NB; ++bb) {
+        if (bb < b) r += tot[bb];
+        else rest += tot[bb];
     }
-    gam[c] = expf((tot[0] + tot[1]) + (tot[2] + tot[3]));
+    eR[b * D + c] = expf(r);
+    eG[b * D + c] = expf(rest);
+#pragma unroll
+    for (int bj = 0; bj < NB; ++bj) {
+        float y = 0.0f;
+#pragma unroll
+        for (int bb = 0; bb < NB; ++bb)
+            if (bb >= bj && bb < b) y += tot[bb];
+        m[(b * NB + bj) * D + c] = bj <= b ? expf(y) : 0.0f;
+    }
+    if (b == 0) gam[c] = expf((tot[0] + tot[1]) + (tot[2] + tot[3]));
 }
 
 // T = (I + Diag(beta) At)^-1 (unit lower triangular, 64 x 64, swizzled [C][C]
