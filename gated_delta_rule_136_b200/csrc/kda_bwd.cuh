@@ -46,6 +46,8 @@ struct BwdParams {
     float *dS0;
     int32_t num_heads;
     float scale, g_floor;
+    int64_t total_tokens;         // for the debug build's unit checks
+    int64_t slots;                // snapshot slots (the same)
 };
 
 // shared memory, floats: key-side [SB][DK] x 4, value-side [SB][DV] x 5, beta,
@@ -136,6 +138,12 @@ __global__ void __launch_bounds__(NT, 1) bwd_kernel(BwdParams p)
     const int64_t n = unit / H, h = unit % H;
     const int64_t tb = p.cu_seqlens[n];
     const int64_t L = (int64_t)p.cu_seqlens[n + 1] - tb;
+    // debug build: the sequence's tokens and snapshots as the host validated them (uniform over the CTA)
+    if (kDebugChecks && (tb < 0 || L < 0 || tb + L > p.total_tokens ||
+                         p.ckpt_base[n] + L / CH != p.ckpt_base[n + 1] || p.ckpt_base[n + 1] > p.slots)) {
+        if (tid == 0) raise_error(ERR_BOUNDS);
+        return;
+    }
     float *scr = p.scratch + unit * SCRATCH_FLOATS;      // [3][DK][DV] sub-block starts, [SB][DK][DV] states
     float *scr_st = scr + (int64_t)(CH / SB - 1) * DK * DV;
 

@@ -70,6 +70,8 @@ struct ChunkBwdParams {
     float *dS0;
     int32_t num_heads;
     float scale, g_floor;
+    int64_t total_tokens;                             // for the debug build's unit checks
+    int32_t num_seqs;                                 // (the same)
 };
 
 // XOR-swizzled element offsets of row-major fp32 tiles (128 or 64 columns):
@@ -168,6 +170,7 @@ struct ChunkRef {
     int64_t tok0;       // first token (packed row) of the chunk
     int Lc;             // tokens in the chunk
     int64_t L;          // tokens in the sequence
+    bool ok;            // debug build: the chunk lies where the host said (else it is skipped)
 };
 
 __device__ __forceinline__ ChunkRef chunk_ref(const ChunkBwdParams &p) {
@@ -178,11 +181,22 @@ __device__ __forceinline__ ChunkRef chunk_ref(const ChunkBwdParams &p) {
     r.u = blockIdx.x;
     r.n = p.chunk_seq[c];
     r.ci = p.chunk_idx[c];
+    r.ok = true;
+    if (kDebugChecks && (r.n < 0 || r.n >= p.num_seqs || r.ci < 0)) {
+        r.ok = false;
+        r.n = 0;
+        r.ci = 0;
+    }
     const int64_t tb = p.cu_seqlens[r.n];
     r.L = (int64_t)p.cu_seqlens[r.n + 1] - tb;
     r.tok0 = tb + r.ci * C;
     const int64_t left = r.L - r.ci * C;
     r.Lc = (int)(left < C ? left : C);
+    // debug build: the device cu_seqlens agree with the host's chunk table (uniform over the CTA)
+    if (kDebugChecks && (tb < 0 || r.L < 0 || tb + r.L > p.total_tokens || left <= 0 ||
+                         p.chunk_base[r.n] + r.ci >= p.chunk_base[r.n + 1] ||
+                         (r.ci > 0 && p.ckpt_base[r.n] + r.ci > p.ckpt_base[r.n + 1])))
+        r.ok = false;
     return r;
 }
 
@@ -385,6 +399,10 @@ __global__ void __launch_bounds__(NT, 1) chain_prep_kernel(ChunkBwdParams p) {
     float *m = sm + S::M, *eR = sm + S::ER, *eG = sm + S::EG, *gam = sm + S::GM, *sb = sm + S::BT;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const ChunkRef r = chunk_ref(p);
+    if (kDebugChecks && !r.ok) {
+        if (threadIdx.x == 0) raise_error(ERR_BOUNDS);
+        return;
+    }
     const int64_t H = p.num_heads;
     float *scr = p.scratch + r.u * Scratch::FLOATS;
     const float *S0p = start_state(p, r);
@@ -519,6 +537,12 @@ __global__ void __launch_bounds__(CHAIN_NT, 2) chain_kernel(ChunkBwdParams p) {
     const int v0 = (blockIdx.x & 1) * DVH;
     const int64_t L = (int64_t)p.cu_seqlens[n + 1] - p.cu_seqlens[n];
     const int64_t nch = (L + C - 1) / C;
+    // debug build: the device cu_seqlens agree with the host's chunk table (uniform over the CTA)
+    if (kDebugChecks && (p.cu_seqlens[n] < 0 || L < 0 || p.cu_seqlens[n] + L > p.total_tokens ||
+                         p.chunk_base[n] + nch != p.chunk_base[n + 1])) {
+        if (tid == 0) raise_error(ERR_BOUNDS);
+        return;
+    }
     const float *dST = p.dS_T ? p.dS_T + (n * H + h) * DD : nullptr;
     for (int i = tid; i < D * DVH / 4; i += NTC) {        // float4 pieces of this half
         const int c = i / (DVH / 4), v = (i % (DVH / 4)) * 4;
@@ -595,6 +619,10 @@ __global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
     uint32_t *gmask = reinterpret_cast<uint32_t *>(sm + S::MK);   // [g >= floor] bits, [C][D / 32]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const ChunkRef r = chunk_ref(p);
+    if (kDebugChecks && !r.ok) {
+        if (threadIdx.x == 0) raise_error(ERR_BOUNDS);
+        return;
+    }
     const int64_t H = p.num_heads;
     float *scr = p.scratch + r.u * Scratch::FLOATS;
     const float *S0p = start_state(p, r);

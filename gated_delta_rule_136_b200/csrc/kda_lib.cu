@@ -829,7 +829,7 @@ kda_status kda_chunk_bwd(const kda_fwd_desc *desc, const void *q, const void *k,
         kda::bwdc::ChunkBwdParams cp{q, k, v, g, beta, gate, dout, S0, dS_T, cu_seqlens, states, base_dev,
                                      cmap_dev, cmap_dev + w.chunks, cbase_dev,
                                      reinterpret_cast<float *>(ws + w.scratch), dq, dk, dv, dg, dbeta, dgate, dS0,
-                                     H, d.scale, d.g_floor};
+                                     H, d.scale, d.g_floor, d.total_tokens, N};
         NvtxRange r("kda.bwd");
         const int64_t ch = w.chunks * H, units = (int64_t)N * H;
         const cudaError_t e = launch_bwd_chunked(cp, ch, units, stream);
@@ -838,7 +838,7 @@ kda_status kda_chunk_bwd(const kda_fwd_desc *desc, const void *q, const void *k,
 
     kda::bwd::BwdParams bp{q, k, v, g, beta, gate, dout, S0, dS_T, cu_seqlens, states, base_dev,
                            reinterpret_cast<float *>(ws + w.scratch), dq, dk, dv, dg, dbeta, dgate, dS0,
-                           H, d.scale, d.g_floor};
+                           H, d.scale, d.g_floor, d.total_tokens, w.slots};
     NvtxRange r("kda.bwd");
     const cudaError_t e = d.io_dtype == KDA_BF16 ? dispatch_bwd<__nv_bfloat16>(d.dk, d.dv, bp, (int64_t)N * H, stream)
                                                  : dispatch_bwd<float>(d.dk, d.dv, bp, (int64_t)N * H, stream);

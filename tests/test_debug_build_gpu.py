@@ -3,7 +3,8 @@ KDA_DEBUG_LIBRARY=1): its results match the oracle, and a unit whose token
 range lies outside the launch (device cu_seqlens that disagree with the
 host copy the call was validated with) is refused on the device --
 KDA_ERR_DEVICE_BOUNDS in the error word, nothing touched -- by both prefill
-kernels.  Run in a child process, since a process loads one library."""
+kernels and both backward paths (chunked and per-token).  Run in a child
+process, since a process loads one library."""
 import os
 import subprocess
 import sys
@@ -20,7 +21,7 @@ CHILD = textwrap.dedent("""
     sys.path.insert(0, {root!r}); sys.path.insert(0, {tests!r})
     import numpy as np, torch
     import oracle
-    from gated_delta_rule_136_b200 import chunk_fwd, device_status, inputs, kda
+    from gated_delta_rule_136_b200 import chunk_bwd, chunk_fwd, device_status, inputs, kda
     from parity import TOL_BF16, TOL_FP32, rel_max, rel_max_beyond_bf16
     assert kda.library_path().endswith("libkda_b200_debug.so")
     cpu = lambda t: None if t is None else t.detach().cpu()
@@ -45,6 +46,28 @@ CHILD = textwrap.dedent("""
         st = device_status()
         assert st == 6, st          # KDA_ERR_DEVICE_BOUNDS
         assert device_status() == 0  # (the word is cleared by reading it)
+    # 3. the backward of the debug build against the oracle (bf16: the chunked kernels)
+    inp = inputs.prefill_inputs([150, 70], H=2, device="cuda", seed=91, s0_std=0.05, gate=True)
+    gen = torch.Generator(device="cuda").manual_seed(92)
+    dout = torch.randn(inp["v"].shape, generator=gen, device="cuda").to(torch.bfloat16)
+    got = chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], dout, cu_seqlens=inp["cu_seqlens"],
+                    cu_seqlens_host=inp["cu_seqlens_host"], S0=inp["S0"], gate=inp["gate"])
+    ref = oracle.kda_bwd_ref(*(cpu(inp[n]) for n in ("q", "k", "v", "g", "beta")), cpu(dout),
+                             cu_seqlens=np.array(inp["cu_seqlens_host"]), S0=cpu(inp["S0"]), gate=cpu(inp["gate"]))
+    for name, r in ref.items():
+        e = rel_max_beyond_bf16(got[name], r) if name != "dS0" else rel_max(got[name], r)
+        assert e <= TOL_BF16, (name, e)
+    assert device_status() == 0
+    # 4. the backward with device cu_seqlens past the validated tokens: refused on the device
+    for dtype in (torch.bfloat16, torch.float32):      # the chunked and the per-token kernels
+        inp = inputs.prefill_inputs([300, 200], H=2, dtype=dtype, device="cuda", seed=97)
+        dout = torch.randn(inp["v"].shape, generator=gen, device="cuda").to(dtype)
+        bad = torch.tensor([0, 300, 564], dtype=torch.int32, device="cuda")
+        chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], dout, cu_seqlens=bad,
+                  cu_seqlens_host=[0, 300, 500])
+        st = device_status()
+        assert st == 6, (dtype, st)
+        assert device_status() == 0
     print("debug build ok")
 """)
 
