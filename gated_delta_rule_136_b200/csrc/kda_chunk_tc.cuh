@@ -911,9 +911,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 *reinterpret_cast<float2 *>(D + gq * ld + 2 * tq) = make_float2(sign * acc[0], sign * acc[1]);
                 *reinterpret_cast<float2 *>(D + (gq + 8) * ld + 2 * tq) = make_float2(sign * acc[2], sign * acc[3]);
             };
-            if (warp < 2) {
-                const int o = 32 * warp;                       // blocks o/16 and o/16 + 1
-                {   // diagonal blocks: lane = (block, column jj)
+            if (warp < 4) {
+                // pair p = warp % 2 (blocks 2p, 2p + 1, rows and columns o .. o + 31) is
+                // merged by warps p (diagonal blocks; n-tile 0) and p + 2 (n-tile 1),
+                // which meet at named barrier 2 + p
+                const int p = warp & 1, half = warp >> 1, o = 32 * p;
+                auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(2 + p) : "memory"); };
+                if (half == 0) {   // diagonal blocks: lane = (block, column jj)
                     const int d0 = o + 16 * (lane >> 4), jj = lane & 15;
                     const float *A = scr + d0 * SCR_LD + d0;
                     float t[16];
@@ -933,35 +937,30 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int i = 0; i < 16; ++i) Tb[i * SCR_LD + jj] = t[i];
                     __syncwarp();
                 }
-                // 16 -> 32: X = A[o+16.., o..] T[o.., o..] over A's block, then T21 = -T22 X
-                float x[2][4];
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    x[nt][0] = x[nt][1] = x[nt][2] = x[nt][3] = 0.0f;
-                    mma_tile(x[nt], scr + (o + 16) * SCR_LD + o, SCR_LD, scr + o * SCR_LD + o + 8 * nt, SCR_LD, 16);
-                }
-                float *blk21 = scr + (o + 16) * SCR_LD + o;
+                pair_sync();                                   // T11, T22 of the pair
+                // 16 -> 32, n-tile `half`: X = A[o+16.., o..] T11[:, tile], then
+                // T21[:, tile] = -T22 X[:, tile]; X replaces A21 only after both warps read it
+                float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                mma_tile(x, scr + (o + 16) * SCR_LD + o, SCR_LD, scr + o * SCR_LD + o + 8 * half, SCR_LD, 16);
+                float *blk21 = scr + (o + 16) * SCR_LD + o + 8 * half;
+                pair_sync();                                   // A21 is read
+                put_tile(blk21, SCR_LD, x, 1.0f);
                 __syncwarp();
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) put_tile(blk21 + 8 * nt, SCR_LD, x[nt], 1.0f);
+                x[0] = x[1] = x[2] = x[3] = 0.0f;
+                mma_tile(x, scr + (o + 16) * SCR_LD + o + 16, SCR_LD, blk21, SCR_LD, 16);
                 __syncwarp();
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    x[nt][0] = x[nt][1] = x[nt][2] = x[nt][3] = 0.0f;
-                    mma_tile(x[nt], scr + (o + 16) * SCR_LD + o + 16, SCR_LD, blk21 + 8 * nt, SCR_LD, 16);
-                }
-                __syncwarp();
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) put_tile(blk21 + 8 * nt, SCR_LD, x[nt], -1.0f);
-                __syncwarp();
+                put_tile(blk21, SCR_LD, x, -1.0f);
+                pair_sync();                                   // T21 of the pair is complete
                 // T' rows o..o+31 (lane = row), tf32 K-major [i x j] in two 32-column
-                // K-blocks: columns o..o+31 from T, the other 32 zero for rows 0-31;
-                // rows 32-63, columns 0-31 are written by the 32 -> 64 step
+                // K-blocks: columns o..o+31 from T (this warp: column groups 2 half,
+                // 2 half + 1), the other 32 zero for rows 0-31; rows 32-63, columns
+                // 0-31 are written by the 32 -> 64 step
                 const int i = o + lane;
                 // also as bf16 (K-major [i x j], one 128-byte row) for the T' V product
-                unsigned char *tpr = sm + OFF_TP + (uint32_t)warp * 8192u;   // K-block of columns o..o+31
+                unsigned char *tpr = sm + OFF_TP + (uint32_t)p * 8192u;   // K-block of columns o..o+31
 #pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8) {
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c8 = 2 * half + cc;
                     const int j0 = o + 8 * c8;
                     const float4 ta = *reinterpret_cast<const float4 *>(scr + i * SCR_LD + j0);
                     const float4 tb = *reinterpret_cast<const float4 *>(scr + i * SCR_LD + j0 + 4);
@@ -974,11 +973,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     *reinterpret_cast<uint4 *>(sm + OFF_TPB + sw128((uint32_t)i, (uint32_t)j0 * 2u)) =
                         make_uint4(pack_bf16(va.x, va.y), pack_bf16(va.z, va.w), pack_bf16(vb.x, vb.y), pack_bf16(vb.z, vb.w));
                 }
-                if (warp == 0) {
+                if (warp == 0) {                               // rows 0-31, columns 32-63: zero
 #pragma unroll
                     for (int c4 = 0; c4 < 8; ++c4)
                         *reinterpret_cast<float4 *>(sm + OFF_TP + 8192u + sw128((uint32_t)i, (uint32_t)c4 * 16u)) =
                             make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                } else if (warp == 2) {
 #pragma unroll
                     for (int c8 = 4; c8 < 8; ++c8)
                         *reinterpret_cast<uint4 *>(sm + OFF_TPB + sw128((uint32_t)i, (uint32_t)c8 * 16u)) = make_uint4(0u, 0u, 0u, 0u);
