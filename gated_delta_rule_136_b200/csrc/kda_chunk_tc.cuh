@@ -36,7 +36,7 @@
 // One CTA (512 threads) carries one (sequence, head) unit; its phases per
 // chunk run in order:
 //   prep (2 passes of 64 key channels; TMA tiles of q, k, g)  ->  A MMAs (tf32)
-//   -> A readout -> block-triangular inverse (warps 0-3)
+//   -> A readout -> block-triangular inverse (warps 0-7)
 //   -> Vn = T' V - T' Y MMAs (Y = (K e^G) S from an MMA issued behind the A MMAs)
 //   -> A_qk Vn, K^T Vn MMAs (tf32)
 //   -> state update + output epilogue.
@@ -871,7 +871,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bool z_ok = true;
         ++y_issued;
         // [O1 | -Y]^T = S^T [Q e^G | -K e^G]^T (bf16, A = S^T from TMEM as its leading and
-        // low parts), issued by warp 8 while warps 0-3 run the inverse: the tensor pipe
+        // low parts), issued by warp 8 while warps 0-7 run the inverse: the tensor pipe
         // is idle then, and no prep warp waits on the issue
         if (warp == 8) {
 #pragma unroll 1
@@ -884,12 +884,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (leader) mma_commit(bar_y);
             __syncwarp();
         }
-        // ================================================= T = (I + A_kk)^-1, then T' = T Diag(beta) (warps 0-3)
+        // ================================================= T = (I + A_kk)^-1, then T' = T Diag(beta) (warps 0-7)
         // Blocked inverse of the unit lower-triangular 64x64 matrix: 16x16
-        // diagonal blocks by forward substitution, then the block merges
+        // diagonal blocks by forward substitution (warps 0-1), then the block merges
         //   [[T11, 0], [T21, T22]]:  T21 = -T22 (A21 T11)
-        // for 16 -> 32 and 32 -> 64.  Each warp owns what it merges, so only one
-        // barrier (among warps 0-3) separates the two merge levels.
+        // for 16 -> 32 (warps 0-3, two per pair) and 32 -> 64 (warps 0-7, two per
+        // column group); the warps that share a merge meet at named barriers.
         {
             const int gq = lane >> 2, tq = lane & 3;
             // acc[16 x 8] += X[16 x K] Y[K x 8] on the warp-level tensor cores
@@ -984,36 +984,32 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         *reinterpret_cast<uint4 *>(sm + OFF_TPB + sw128((uint32_t)i, (uint32_t)c8 * 16u)) = make_uint4(0u, 0u, 0u, 0u);
                 }
             }
-            if (warp < 4) {
-                asm volatile("bar.sync 1, 128;" ::: "memory");   // warps 0-3 only
-                // 32 -> 64 for columns 8 warp .. 8 warp + 7:
-                //   X = A[32:64, 0:32] T[0:32, cols],  T[32:64, cols] = -T[32:64, 32:64] X
-                float *xs = reinterpret_cast<float *>(sm + OFF_XS) + warp * 32 * XS_LD;
-                const int n0 = 8 * warp;
-                float x[2][4];
-#pragma unroll
-                for (int rt = 0; rt < 2; ++rt) {
-                    x[rt][0] = x[rt][1] = x[rt][2] = x[rt][3] = 0.0f;
-                    mma_tile(x[rt], scr + (32 + 16 * rt) * SCR_LD, SCR_LD, scr + n0, SCR_LD, 32);
-                    put_tile(xs + 16 * rt * XS_LD, XS_LD, x[rt], 1.0f);
-                }
-                __syncwarp();
-#pragma unroll
-                for (int rt = 0; rt < 2; ++rt) {
-                    x[rt][0] = x[rt][1] = x[rt][2] = x[rt][3] = 0.0f;
-                    mma_tile(x[rt], scr + (32 + 16 * rt) * SCR_LD + 32, SCR_LD, xs, XS_LD, 32);
-                    const int j = n0 + 2 * tq;            // columns 0-31: K-block 0
-                    const float b0 = -s_beta[j], b1 = -s_beta[j + 1];
-                    const int i0 = 32 + 16 * rt + gq;
-                    *reinterpret_cast<float2 *>(sm + OFF_TP + sw128((uint32_t)i0, (uint32_t)j * 4u)) =
-                        make_float2(x[rt][0] * b0, x[rt][1] * b1);
-                    *reinterpret_cast<float2 *>(sm + OFF_TP + sw128((uint32_t)i0 + 8u, (uint32_t)j * 4u)) =
-                        make_float2(x[rt][2] * b0, x[rt][3] * b1);
-                    *reinterpret_cast<uint32_t *>(sm + OFF_TPB + sw128((uint32_t)i0, (uint32_t)j * 2u)) =
-                        pack_bf16(x[rt][0] * b0, x[rt][1] * b1);
-                    *reinterpret_cast<uint32_t *>(sm + OFF_TPB + sw128((uint32_t)i0 + 8u, (uint32_t)j * 2u)) =
-                        pack_bf16(x[rt][2] * b0, x[rt][3] * b1);
-                }
+            if (warp < 8) {
+                asm volatile("bar.sync 1, 256;" ::: "memory");   // warps 0-7 only
+                // 32 -> 64 for columns 8 cg .. 8 cg + 7 (cg = warp % 4), rows 32 + 16 rt ..
+                // + 15 (rt = warp / 4):
+                //   X = A[32:64, 0:32] T[0:32, cols],  T[32:64, cols] = -T[32:64, 32:64] X;
+                // the two row tiles of a column group meet at named barrier 4 + cg
+                const int cg = warp & 3, rt = warp >> 2;
+                float *xs = reinterpret_cast<float *>(sm + OFF_XS) + cg * 32 * XS_LD;
+                const int n0 = 8 * cg;
+                float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                mma_tile(x, scr + (32 + 16 * rt) * SCR_LD, SCR_LD, scr + n0, SCR_LD, 32);
+                put_tile(xs + 16 * rt * XS_LD, XS_LD, x, 1.0f);
+                asm volatile("bar.sync %0, 64;" ::"r"(4 + cg) : "memory");   // both row tiles of X
+                x[0] = x[1] = x[2] = x[3] = 0.0f;
+                mma_tile(x, scr + (32 + 16 * rt) * SCR_LD + 32, SCR_LD, xs, XS_LD, 32);
+                const int j = n0 + 2 * tq;                // columns 0-31: K-block 0
+                const float b0 = -s_beta[j], b1 = -s_beta[j + 1];
+                const int i0 = 32 + 16 * rt + gq;
+                *reinterpret_cast<float2 *>(sm + OFF_TP + sw128((uint32_t)i0, (uint32_t)j * 4u)) =
+                    make_float2(x[0] * b0, x[1] * b1);
+                *reinterpret_cast<float2 *>(sm + OFF_TP + sw128((uint32_t)i0 + 8u, (uint32_t)j * 4u)) =
+                    make_float2(x[2] * b0, x[3] * b1);
+                *reinterpret_cast<uint32_t *>(sm + OFF_TPB + sw128((uint32_t)i0, (uint32_t)j * 2u)) =
+                    pack_bf16(x[0] * b0, x[1] * b1);
+                *reinterpret_cast<uint32_t *>(sm + OFF_TPB + sw128((uint32_t)i0 + 8u, (uint32_t)j * 2u)) =
+                    pack_bf16(x[2] * b0, x[3] * b1);
             }
         }
         if (tid == 0) z_ok = mbar_wait(bar_v, ld_par) && mbar_wait(bar_y, y_phase & 1);
