@@ -35,10 +35,11 @@
 //
 // One CTA (512 threads) carries one (sequence, head) unit; its phases per
 // chunk run in order:
-//   prep (2 passes of 64 key channels; TMA tiles of q, k, g)  ->  A MMAs (tf32)
+//   prep (2 passes of 64 key channels; TMA tiles of q, k, g)  ->  A MMAs (tf32 diagonal
+//   blocks, fp16 off-diagonal)
 //   -> A readout -> block-triangular inverse (warps 0-7)
 //   -> Vn = T' V - T' Y MMAs (Y = (K e^G) S from an MMA issued behind the A MMAs)
-//   -> A_qk Vn, K^T Vn MMAs (tf32)
+//   -> A_qk Vn, K^T Vn MMAs (fp16, power-of-two scales)
 //   -> state update + output epilogue.
 // The next chunk's q, k, g, v tiles are loaded by TMA while the current
 // chunk's later phases run.
