@@ -82,3 +82,12 @@ def test_backward_floor_stress(dtype):
     chunked form reach e^{16 |floor|}, and clamped entries must pass no gradient."""
     got, ref = _run([200, 64, 33], H=2, dtype=dtype, seed=113, g_mode="floor_stress")
     _check(got, ref, dtype)
+
+
+def test_backward_many_sequences():
+    """Twelve sequences of lengths around the chunk and block sizes (empty, 1,
+    one chunk exactly, one token past it, ...): the chunk tables, the chain
+    over each sequence's chunks and the gradients at every sequence boundary."""
+    lengths = [0, 1, 15, 16, 63, 64, 65, 127, 128, 129, 200, 7]
+    got, ref = _run(lengths, H=2, dtype=torch.bfloat16, seed=127)
+    _check(got, ref, torch.bfloat16)
