@@ -91,3 +91,23 @@ def test_backward_many_sequences():
     lengths = [0, 1, 15, 16, 63, 64, 65, 127, 128, 129, 200, 7]
     got, ref = _run(lengths, H=2, dtype=torch.bfloat16, seed=127)
     _check(got, ref, torch.bfloat16)
+
+
+def test_backward_bench_shape_sampled_units():
+    """The bench's backward workload as launched (8 x 4096 tokens x 32 heads,
+    bf16, no gate, S0 = 0, the bench's input recipe); two (sequence, head)
+    units -- the first and the last of the launch -- against the oracle."""
+    B, T, H = 8, 4096, 32
+    inp = inputs.prefill_inputs([T] * B, H=H, device="cuda", seed=0)
+    gen = torch.Generator(device="cuda").manual_seed(200)
+    dout = torch.randn(inp["v"].shape, generator=gen, device="cuda").to(torch.bfloat16)
+    got = chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], dout, cu_seqlens=inp["cu_seqlens"],
+                    cu_seqlens_host=inp["cu_seqlens_host"], want_dS0=False)
+    assert device_status() == 0
+    for n, h in ((0, 0), (B - 1, H - 1)):
+        sl = slice(n * T, (n + 1) * T)
+        part = lambda t: _cpu(t[sl, h:h + 1]).contiguous()
+        ref = oracle.kda_bwd_ref(*(part(inp[x]) for x in ("q", "k", "v", "g", "beta")), part(dout),
+                                 cu_seqlens=np.array([0, T]))
+        mine = {name: got[name][sl, h:h + 1] for name in ref}
+        _check(mine, ref, torch.bfloat16)
