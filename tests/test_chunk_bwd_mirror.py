@@ -64,3 +64,11 @@ def test_chunk_bwd_mirror_floor_stress():
     assert _rel(o, o_ref) < 1e-10
     for name in ref:
         assert _rel(got[name], ref[name]) < 1e-9, name
+
+
+def test_chunk_bwd_mirror_kernel_head_size():
+    """dk = dv = 128, the chunked kernels' head size: three chunks, the last one ragged."""
+    got, ref, o, o_ref = _run([150], H=1, dk=128, dv=128, seed=17, gate=True, s0=True, dS_T_on=True)
+    assert _rel(o, o_ref) < 1e-10
+    for name in ref:
+        assert _rel(got[name], ref[name]) < 1e-9, name
