@@ -288,8 +288,11 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 // SNAP: the variant that stores state snapshots (TcParams::snap); the other
-// compiles without that code.
-template <bool SNAP>
+// compiles without that code.  NOOUT: for launches whose units store no outputs
+// (the long-sequence split's first pass, context-parallel summaries): the q
+// side (Q~, Q e^G, A_qk, O1, O2) is not formed; the state products run as their
+// K e^G and K^ parts alone (N = 64 and N = 128).
+template <bool SNAP, bool NOOUT = false>
 __global__ void __launch_bounds__(NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
@@ -337,7 +340,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     if (kDebugChecks) {   // the unit must lie inside the launch's extents
         const bool bad = t_begin < 0 || t_end < t_begin || t_end > p.total_tokens || hh < 0 || hh >= H ||
-                         snap_n < 0 || snap_n >= p.num_seqs;
+                         snap_n < 0 || snap_n >= p.num_seqs || (NOOUT && (flags & UNIT_STORE_O));
         if (bad) {
             if (tid == 0) raise_error(ERR_BOUNDS);
             return;                      // (uniform over the CTA, before any shared or TMEM state)
@@ -500,10 +503,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // MMA descriptors that do not depend on the chunk (start addresses advance per K-step)
     const uint32_t id_d = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 64, 128);
     const uint32_t id_o = instr_desc(FMT_F16, K_MAJOR, K_MAJOR, 64, 32);
-    const uint32_t id_1 = instr_desc(FMT_BF16, K_MAJOR, MN_MAJOR, 128, 128);
+    const uint32_t id_1 = instr_desc(FMT_BF16, K_MAJOR, MN_MAJOR, 128, NOOUT ? 64 : 128);
     const uint32_t id_vn = instr_desc(FMT_TF32, K_MAJOR, K_MAJOR, 128, 64);
     const uint32_t id_u = instr_desc(FMT_BF16, MN_MAJOR, K_MAJOR, 128, 64);
-    const uint32_t id_2 = instr_desc(FMT_F16, K_MAJOR, K_MAJOR, 128, 192);
+    const uint32_t id_2 = instr_desc(FMT_F16, K_MAJOR, K_MAJOR, 128, NOOUT ? 128 : 192);
     const uint64_t d_k16 = smem_desc_sw128(smb, 16, 1024);          // K-major template
     const uint64_t d_qk = smem_desc_sw128(smb, OFF_KG - OFF_QG, 1024);  // [Q e^G | -K e^G] MN-major
     const uint64_t d_mnv = smem_desc_sw128(smb, 8192, 1024);             // v: MN blocks 8 KB apart
@@ -689,14 +692,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         const float2 gt = make_float2(ex2_approx(t2.x), ex2_approx(t2.y));       // Gt_i
                         const float2 ig = make_float2(ex2_approx(u2.x), ex2_approx(u2.y));       // 1 / Gt_i
                         const uint32_t qoff = raw + QKG_Q + sw128((uint32_t)i, (uint32_t)cA * 2u);
-                        const float2 q2 = unpack_bf16x2(ld_shared_u32(qoff));
-                        const float2 k2 = unpack_bf16x2(ld_shared_u32(qoff + (QKG_K - QKG_Q)));
-                        qt[bb][hr] = __fmul2_rn(q2, gt);
-                        kt[bb][hr] = __fmul2_rn(k2, gt);
-                        kbar[bb][hr] = __fmul2_rn(k2, ig);                                        // Kbar_i
-                        const float2 qg = __fmul2_rn(qt[bb][hr], Eb), kg = __fmul2_rn(kt[bb][hr], Eb);
-                        pq[hr] = pack_bf16(qg.x, qg.y);
-                        pk[hr] = pack_bf16(-kg.x, -kg.y);   // -K e^G: the MMA then yields -Y
+                        if constexpr (!NOOUT) {
+                            const float2 q2 = unpack_bf16x2(ld_shared_u32(qoff));
+                            const float2 k2 = unpack_bf16x2(ld_shared_u32(qoff + (QKG_K - QKG_Q)));
+                            qt[bb][hr] = __fmul2_rn(q2, gt);
+                            kt[bb][hr] = __fmul2_rn(k2, gt);
+                            kbar[bb][hr] = __fmul2_rn(k2, ig);                                        // Kbar_i
+                            const float2 qg = __fmul2_rn(qt[bb][hr], Eb), kg = __fmul2_rn(kt[bb][hr], Eb);
+                            pq[hr] = pack_bf16(qg.x, qg.y);
+                            pk[hr] = pack_bf16(-kg.x, -kg.y);   // -K e^G: the MMA then yields -Y
+                        } else {                                // the k side alone
+                            const float2 k2 = unpack_bf16x2(ld_shared_u32(qoff + (QKG_K - QKG_Q)));
+                            kt[bb][hr] = __fmul2_rn(k2, gt);
+                            kbar[bb][hr] = __fmul2_rn(k2, ig);
+                            const float2 kg = __fmul2_rn(kt[bb][hr], Eb);
+                            pk[hr] = pack_bf16(-kg.x, -kg.y);
+                        }
                         // K^(4)^T [c x j] tf32: two channels of token i; on the first pass the
                         // previous chunk's last MMA may still read these rows: stored later
                         const float2 kh = __fmul2_rn(kbar[bb][hr], eK);
@@ -707,7 +718,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     {
                         const uint32_t row = (uint32_t)(pass * 64 + nt * 8 + (lane & 7));
                         const uint32_t tb2 = (uint32_t)(16 * b + 8 * ((lane >> 3) & 1)) * 2u;
-                        stsm_x2_trans(smb + OFF_QG + sw128(row, tb2), pq[0], pq[1]);
+                        if constexpr (!NOOUT) stsm_x2_trans(smb + OFF_QG + sw128(row, tb2), pq[0], pq[1]);
                         stsm_x2_trans(smb + OFF_KG + sw128(row, tb2), pk[0], pk[1]);
                     }
                 }
@@ -737,11 +748,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         const uint32_t i = (uint32_t)(16 * b + 8 * hr) + (uint32_t)gq;
                         const uint32_t xrow = (uint32_t)(32 * b + 8 * hr) + (uint32_t)gq;
                         auto rnd2 = [](float2 x) { return make_float2(to_tf32(x.x), to_tf32(x.y)); };
-                        *reinterpret_cast<float2 *>(sm + xt_lane + xrow * 128u) = rnd2(qt[bb][hr]);
+                        if constexpr (!NOOUT) *reinterpret_cast<float2 *>(sm + xt_lane + xrow * 128u) = rnd2(qt[bb][hr]);
                         *reinterpret_cast<float2 *>(sm + xt_lane + (xrow + 16u) * 128u) = rnd2(kt[bb][hr]);
                         *reinterpret_cast<float2 *>(sm + kd_lane + i * 128u) = rnd2(kbar[bb][hr]);
                         if (b > 0) {
-                            *reinterpret_cast<uint32_t *>(sm + xb_lane + (xrow - 32u) * 128u) = pack_f16(qt[bb][hr].x, qt[bb][hr].y);
+                            if constexpr (!NOOUT)
+                                *reinterpret_cast<uint32_t *>(sm + xb_lane + (xrow - 32u) * 128u) = pack_f16(qt[bb][hr].x, qt[bb][hr].y);
                             *reinterpret_cast<uint32_t *>(sm + xb_lane + (xrow - 16u) * 128u) = pack_f16(kt[bb][hr].x, kt[bb][hr].y);
                         }
 #pragma unroll
@@ -782,10 +794,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         }
                     }
                     uint32_t r1[16], r2[16];
-                    tmem_ld16(tbase + lane_base + T_O1 + cq * 16, r1);
-                    tmem_ld16(tbase + lane_base + T_O2 + cq * 16, r2);
-                    tmem_wait_ld();
-                    if (store_o) {
+                    if constexpr (!NOOUT) {
+                        tmem_ld16(tbase + lane_base + T_O1 + cq * 16, r1);
+                        tmem_ld16(tbase + lane_base + T_O2 + cq * 16, r2);
+                        tmem_wait_ld();
+                    }
+                    if (!NOOUT && store_o) {
                         float x[16];
 #pragma unroll
                         for (int e = 0; e < 16; ++e) x[e] = p.scale * (__uint_as_float(r1[e]) + __uint_as_float(r2[e]));
@@ -860,7 +874,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const int i = 16 * cq + e;
                     const float aq = j <= i ? __uint_as_float(ra[e]) : 0.0f;
                     const float ak = j < i ? s_beta[i] * __uint_as_float(rk[e]) : 0.0f;
-                    *reinterpret_cast<__half *>(sm + OFF_AQK + sw128(i, (uint32_t)j * 2u)) = __float2half_rn(aq * 256.0f);
+                    if constexpr (!NOOUT)
+                        *reinterpret_cast<__half *>(sm + OFF_AQK + sw128(i, (uint32_t)j * 2u)) = __float2half_rn(aq * 256.0f);
                     scr[i * SCR_LD + j] = ak;
                 }
             }
@@ -877,10 +892,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (warp == 8) {
 #pragma unroll 1
             for (int ks = 0; ks < 8; ++ks) {       // K = 128 key channels in steps of 16
-                if (leader) mma_bf16_ts(tbase + T_O1, tbase + T_S + 8u * (uint32_t)ks,
-                                        at(d_qk, OFF_QG + 2048u * (uint32_t)ks), id_1, ks > 0);
-                if (leader) mma_bf16_ts(tbase + T_O1, tbase + T_LO + 8u * (uint32_t)ks,
-                                        at(d_qk, OFF_QG + 2048u * (uint32_t)ks), id_1, 1u);
+                // (NOOUT: the -K e^G half alone, into -Y's columns)
+                const uint32_t dcol = NOOUT ? T_Z : T_O1, bsrc = (NOOUT ? OFF_KG : OFF_QG) + 2048u * (uint32_t)ks;
+                if (leader) mma_bf16_ts(tbase + dcol, tbase + T_S + 8u * (uint32_t)ks, at(d_qk, bsrc), id_1, ks > 0);
+                if (leader) mma_bf16_ts(tbase + dcol, tbase + T_LO + 8u * (uint32_t)ks, at(d_qk, bsrc), id_1, 1u);
             }
             if (leader) mma_commit(bar_y);
             __syncwarp();
@@ -1064,7 +1079,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (warp == 0) {
 #pragma unroll
             for (int s = 0; s < 4; ++s)            // K = 64 tokens in steps of 16
-                if (leader) mma_bf16_ts(tbase + T_O2, tbase + T_LO + 8u * s, at(d_k16, OFF_AK + 32u * s), id_2, s > 0);
+                if (leader)   // (NOOUT: the K^ rows alone, into dS's columns)
+                    mma_bf16_ts(tbase + (NOOUT ? T_DS : T_O2), tbase + T_LO + 8u * s,
+                                at(d_k16, (NOOUT ? OFF_KHT : OFF_AK) + 32u * s), id_2, s > 0);
             if (leader) mma_commit(bar_mma);
         }
     }

@@ -271,16 +271,18 @@ bool tc_path_applies(const kda_fwd_desc &d, const void *q, const void *k, const 
 
 cudaError_t launch_tc_units(const kda_fwd_desc &d, const void *q, const void *k, const void *v,
                             const void *g, const kda::tck::TcParams &p, int64_t blocks,
-                            cudaStream_t stream);
+                            cudaStream_t stream, bool no_out = false);
 
 cudaError_t launch_tc(const kda_fwd_desc &d, const void *q, const void *k, const void *v,
                       const void *g, const kda::tck::TcParams &p, cudaStream_t stream) {
     return launch_tc_units(d, q, k, v, g, p, (int64_t)d.num_seqs * d.num_heads, stream);
 }
 
+// no_out: no unit of the launch stores outputs (the split's first pass, the
+// context-parallel summaries): the kernel instance without the q side.
 cudaError_t launch_tc_units(const kda_fwd_desc &d, const void *q, const void *k, const void *v,
                             const void *g, const kda::tck::TcParams &p, int64_t blocks,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, bool no_out) {
     CUtensorMap tq, tk, tg, tv, to;
     const uint64_t rows = (uint64_t)d.total_tokens, cols = (uint64_t)d.num_heads * 128u;
     if (!encode_bf16_2d(&tq, q, rows, cols) || !encode_bf16_2d(&tk, k, rows, cols) ||
@@ -289,7 +291,8 @@ cudaError_t launch_tc_units(const kda_fwd_desc &d, const void *q, const void *k,
         // no unit carries UNIT_STORE_O; q stands in for a valid address
         !encode_bf16_2d(&to, p.o ? p.o : q, rows, cols))
         return cudaErrorInvalidValue;
-    auto kern = p.snap.states ? kda::tck::chunk_tc_kernel<true> : kda::tck::chunk_tc_kernel<false>;
+    auto kern = p.snap.states ? kda::tck::chunk_tc_kernel<true>
+                              : no_out ? kda::tck::chunk_tc_kernel<false, true> : kda::tck::chunk_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kda::tck::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
@@ -382,7 +385,7 @@ cudaError_t launch_split(const kda_fwd_desc &d, const SegPlan &pl, const int32_t
     if (!p1.empty()) {
         tp.units = d1;
         NvtxRange r("kda.split.pass1");
-        if ((e = launch_tc_units(d, q, k, v, g, tp, (int64_t)p1.size(), stream)) != cudaSuccess) return e;
+        if ((e = launch_tc_units(d, q, k, v, g, tp, (int64_t)p1.size(), stream, true)) != cudaSuccess) return e;
     }
     const size_t scan_smem = 2u * DD * sizeof(float);
     if ((e = cudaFuncSetAttribute(kda::segment_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1007,7 +1010,7 @@ kda_status kda_segment_summary(const kda_fwd_desc *desc, const void *q, const vo
                           d.g_floor, du, kda::SnapOut{nullptr, nullptr, 0, 64}, d.total_tokens, d.num_seqs};
     {
         NvtxRange r("kda.summary.chains");
-        if (launch_tc_units(d, q, k, v, g, tp, (int64_t)units.size(), stream) != cudaSuccess) return KDA_ERR_CUDA;
+        if (launch_tc_units(d, q, k, v, g, tp, (int64_t)units.size(), stream, true) != cudaSuccess) return KDA_ERR_CUDA;
     }
     if (jobs.empty()) return KDA_OK;
     kda::ScanJob *dj = reinterpret_cast<kda::ScanJob *>(ws + w.jobs);
