@@ -61,7 +61,7 @@ def bytes_per_token_head(dk=DK, dv=DV, esz=2):
 # DRAM traffic per unit from the ncu captures under profiles/ (bytes), valid only
 # for the kernel source they were taken from (sha1 prefix); otherwise null.
 PROFILED_TRAFFIC = {
-    "csrc/kda_chunk_tc.cuh": {"sha1": "9c5fe5a82873", "bytes_per_token_head": (269.035264e6 + 51.734272e6) / 262144,
+    "csrc/kda_chunk_tc.cuh": {"sha1": "372ef2e0393a", "bytes_per_token_head": (269.303296e6 + 52.576000e6) / 262144,
                               "profile": "profiles/chunk_tc_kernel_prefill_4x4096x16.md"},
     "csrc/kda_decode.cuh": {"sha1": "8e75484b34f3", "bytes_per_head_step": (273.707520e6 + 212.401408e6) / 4096,
                             "profile": "profiles/decode_kernel_64x64.md"},
