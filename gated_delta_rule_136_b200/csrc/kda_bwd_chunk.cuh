@@ -696,6 +696,18 @@ __global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
         [&](int, int v, int j) { return sb[j] * ldn(Zg + j * D + v); },
         [&](int i, int j, float x) { s1[xc(i, j)] = x; });
     __syncthreads();
+    // nu (scratch) into b4 for dA_qk (dnu is done with), beside X
+    const float *nug = scr + Scratch::NU;
+    {
+        float4 xn[CD / 4 / NT];
+#pragma unroll
+        for (int u = 0; u < CD / 4 / NT; ++u) xn[u] = ldn4(nug + 4 * (tid + u * NT));
+#pragma unroll
+        for (int u = 0; u < CD / 4 / NT; ++u) {
+            const int i = 4 * (tid + u * NT);
+            *reinterpret_cast<float4 *>(b4 + xd(i / D, i % D)) = xn[u];
+        }
+    }
     // X = dT T^T (into s2), then dA_kk = -T^T X, j < i (into s1)
     gemm<C, C, 4, SPLIT>(warp, 0, NW, lane, [](int, int, int &lo, int &hi) { lo = 0; hi = C; },
         [&](int i, int b) { return s1[xc(i, b)]; },
@@ -707,11 +719,10 @@ __global__ void __launch_bounds__(NT, 1) chain_grad_kernel(ChunkBwdParams p) {
         [&](int, int a, int j) { return s2[xc(a, j)]; },
         [&](int i, int j, float x) { s1[xc(i, j)] = j < i ? -x : 0.0f; });
     __syncthreads();
-    // dA_qk = scale go nu^T, j <= i (into s2)
-    const float *nug = scr + Scratch::NU;
+    // dA_qk = scale go nu^T, j <= i (into s2; nu staged in b4)
     gemm<C, C, 4, SPLIT>(warp, 0, NW, lane, [](int i0, int j0, int &lo, int &hi) { lo = 0; hi = j0 > i0 + 15 ? 0 : D; },
         [&](int i, int v) { return b3[xd(i, v)]; },
-        [&](int, int v, int j) { return ldn(nug + j * D + v); },
+        [&](int, int v, int j) { return b4[xd(j, v)]; },
         [&](int i, int j, float x) { s2[xc(i, j)] = j <= i ? scale * x : 0.0f; });
     __syncthreads();
     // dbeta = rowsum(dY o Z) + rowsum(dA_kk o At): a warp per row
