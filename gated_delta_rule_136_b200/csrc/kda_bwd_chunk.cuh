@@ -17,7 +17,7 @@
 //       Et = Diag(beta) T^T (scale A_qk^T go),  Wt = Diag(beta) T^T Khat,
 //       F = scale Qbar^T go,  Kbar,  e^{lgam},  with go = do sigmoid(z);
 //       and Z, nu, T, At, A_qk for the last kernel, dz of the output gate.
-//   chain       (a CTA per sequence x head, chunks last first):
+//   chain       (two CTAs per sequence x head, 64 value columns each; chunks last first):
 //       dZ = Et + Wt dS_C,  dS0 = F + e^{lgam} dS_C - Kbar^T dZ  (dS_C of every chunk kept).
 //   chain_grad  (a CTA per chunk x head): with dS_C,
 //       dnu = scale A_qk^T go + Khat dS_C,  dY = T^T dnu,  dv = Diag(beta) dY,
