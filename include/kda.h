@@ -315,8 +315,9 @@ kda_status kda_chunk_fwd_host(const kda_fwd_desc *desc, const void *q, const voi
  * snapshots every 64 tokens into the workspace.  Then, for bf16 I/O with
  * dk = dv = 128 and 16-byte aligned q, k, g, dout and gate, the chunked form:
  * per 64-token chunk the gradient chain's constants, the chain over the
- * chunks (two CTAs per sequence and head, half the value columns each), and every gradient of a chunk from its
- * start state and the gradient reaching its end (tensor-core products);
+ * chunks (two CTAs per sequence and head, half the value columns each),
+ * and every gradient of a chunk from its start state and the gradient
+ * reaching its end (tensor-core products);
  * otherwise (fp32 I/O, other head sizes, unaligned tensors) one CTA per
  * (sequence, head) recomputes each chunk's states from its snapshot and runs
  * the recurrence backwards token by token.  The results match the gradients
