@@ -309,13 +309,16 @@ __device__ void invert_T(int tid, int warp, int lane, const float *At, const flo
     __syncthreads();
 }
 
-// shared memory of chain_prep: 4 [C][D] tiles, 3 [C][C] tiles, tables
+// shared memory of chain_prep: 3 [C][D] tiles, 3 [C][C] tiles, tables, and
+// last kb's [C][D] tile with a second one after it: once kb is spent the two
+// hold S0 [D][D] in the same swizzle.
 struct PrepSmem {
-    static constexpr int B0 = 0, B1 = B0 + CD, B2 = B1 + CD, B3 = B2 + CD;
+    static constexpr int B0 = 0, B1 = B0 + CD, B3 = B1 + CD;
     static constexpr int AQ = B3 + CD, AT = AQ + CC, TT = AT + CC;
     static constexpr int M = TT + CC, ER = M + NB * NB * D, EG = ER + NB * D, GM = EG + NB * D;
-    static constexpr int BT = GM + D, FLOATS = BT + C;
+    static constexpr int BT = GM + D, B2 = BT + C, FLOATS = B2 + DD;
     static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
+    static_assert(B2 % 4 == 0, "S0 is staged in 16-byte pieces");
 };
 
 // Loads of data that no thread writes during the launch (inputs, and what
@@ -435,11 +438,34 @@ __global__ void __launch_bounds__(NT, 1) chain_prep_kernel(ChunkBwdParams p) {
     __syncthreads();
     invert_T<SPLIT>(tid, warp, lane, At, sb, Tm, b3);   // b3 (a) is not needed any more
 
+    // Wt = Diag(beta) T^T Khat (to scratch): kb's last use
+    gemm<C, D, 4, SPLIT>(warp, 0, NW, lane, [](int i0, int, int &lo, int &hi) { lo = i0; hi = C; },
+        [&](int i, int l) { return Tm[xc(l, i)]; },
+        [&](int, int l, int c) { return kb[xd(l, c)] * eG[(l >> 4) * D + c]; },
+        [&](int i, int c, float x) { scr[Scratch::WT + i * D + c] = sb[i] * x; });
+    // S0 into kb's tile and the one after it, for the two products that read it
+    constexpr int SU = DD / 4 / NT;
+    float4 xs[SU];
+    if (S0p) {
+#pragma unroll
+        for (int u = 0; u < SU; ++u) xs[u] = ldn4(S0p + 4 * (tid + u * NT));
+    }
+    __syncthreads();
+    float *s0s = kb;
+    if (S0p) {
+#pragma unroll
+        for (int u = 0; u < SU; ++u) {
+            const int piece = tid + u * NT, row = piece / (D / 4), c4 = (piece % (D / 4)) * 4;
+            *reinterpret_cast<float4 *>(s0s + xd(row, c4)) = xs[u];
+        }
+    }
+    __syncthreads();
+
     // Z = V - Kbar S0 (into b3), Kbar and the small tiles to scratch
     gemm<C, D, 4, SPLIT>(warp, 0, NW, lane,
         [&](int, int, int &lo, int &hi) { lo = 0; hi = S0p ? D : 0; },
         [&](int i, int c) { return ka[xd(i, c)] * eR[(i >> 4) * D + c]; },
-        [&](int, int c, int v) { return ldn(S0p + c * D + v); },
+        [&](int, int c, int v) { return s0s[xd(c, v)]; },
         [&](int i, int v, float x) {
             const float vi = i < r.Lc ? ldn(vin + ((r.tok0 + i) * H + r.h) * D + v) : 0.0f;
             const float z = vi - x;
@@ -473,7 +499,7 @@ __global__ void __launch_bounds__(NT, 1) chain_prep_kernel(ChunkBwdParams p) {
     gemm<C, D, 4, SPLIT>(warp, 0, NW, lane,
         [&](int i0, int, int &lo, int &hi) { lo = S0p ? 0 : D; hi = D + i0 + 16; },
         [&](int i, int k) { return k < D ? qa[xd(i, k)] * eR[(i >> 4) * D + k] : Aq[xc(i, k - D)]; },
-        [&](int, int k, int v) { return k < D ? ldn(S0p + k * D + v) : nu[xd(k - D, v)]; },
+        [&](int, int k, int v) { return k < D ? s0s[xd(k, v)] : nu[xd(k - D, v)]; },
         [&](int i, int v, float x) {
             float go = 0.0f;
             if (i < r.Lc) {
@@ -501,15 +527,11 @@ __global__ void __launch_bounds__(NT, 1) chain_prep_kernel(ChunkBwdParams p) {
         [&](int, int i, int v) { return b3[xd(i, v)]; },
         [&](int j, int v, float x) { E[xd(j, v)] = scale * x; });
     __syncthreads();
-    // Et = Diag(beta) T^T E, Wt = Diag(beta) T^T Khat (to scratch)
+    // Et = Diag(beta) T^T E (to scratch)
     gemm<C, D, 4, SPLIT>(warp, 0, NW, lane, [](int i0, int, int &lo, int &hi) { lo = i0; hi = C; },
         [&](int i, int l) { return Tm[xc(l, i)]; },
         [&](int, int l, int v) { return E[xd(l, v)]; },
         [&](int i, int v, float x) { scr[Scratch::ET + i * D + v] = sb[i] * x; });
-    gemm<C, D, 4, SPLIT>(warp, 0, NW, lane, [](int i0, int, int &lo, int &hi) { lo = i0; hi = C; },
-        [&](int i, int l) { return Tm[xc(l, i)]; },
-        [&](int, int l, int c) { return kb[xd(l, c)] * eG[(l >> 4) * D + c]; },
-        [&](int i, int c, float x) { scr[Scratch::WT + i * D + c] = sb[i] * x; });
 }
 
 // The chain: a CTA per (sequence, head, half of the value columns).  dS's
