@@ -70,7 +70,7 @@ PROFILED_TRAFFIC = {
                           "bytes_per_head_round": (579.116800e6 + 4.305920e6 + 555.884544e6 + 477.843968e6) / 8192,
                           "profile": "profiles/spec_kernel_verify_commit_128x64.md"},
     # chunked backward's gradient kernel (chain_grad) at 1 x 4096 x 32 (bf16): per token-head
-    "csrc/kda_bwd_chunk.cuh": {"sha1": "95b8793fe139", "bytes_per_token_head": (638.781952e6 + 183.433984e6) / 131072,
+    "csrc/kda_bwd_chunk.cuh": {"sha1": "572415ff7970", "bytes_per_token_head": (638.781952e6 + 183.433984e6) / 131072,
                                "profile": "profiles/bwd_chunk_kernels_1x4096x32.md"},
 }
 

@@ -319,6 +319,7 @@ struct PrepSmem {
     static constexpr int BT = GM + D, B2 = BT + C, FLOATS = B2 + DD;
     static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
     static_assert(B2 % 4 == 0, "S0 is staged in 16-byte pieces");
+    static_assert(BYTES <= 232448, "fits in 227 KB");
 };
 
 // Loads of data that no thread writes during the launch (inputs, and what
@@ -543,6 +544,8 @@ struct ChainSmem {
     static constexpr int DS = 0, DZ = DS + D * DVH, WT = DZ + C * DVH, KB = WT + CD, GM = KB + CD;
     static constexpr int FLOATS = GM + D;
     static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
+    // two CTAs per SM: 228 KB per SM, 1 KB of it reserved per CTA
+    static_assert(2 * (BYTES + 1024) <= 233472, "two CTAs fit on an SM");
 };
 // swizzled offsets of a row-major tile with 64 columns (as xc)
 __device__ __forceinline__ int xh(int r, int c) { return xc(r, c); }
@@ -626,6 +629,7 @@ struct GradSmem {
     static constexpr int M = S2 + CC, ER = M + NB * NB * D, EG = ER + NB * D, GM = EG + NB * D;
     static constexpr int BT = GM + D, DL = BT + C, MK = DL + D, FLOATS = MK + C * D / 32;
     static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
+    static_assert(BYTES <= 232448, "fits in 227 KB");
 };
 
 template <typename TIO, bool SPLIT>
