@@ -33,3 +33,22 @@ def test_unknown_extra_workload_is_rejected():
     out = subprocess.run([sys.executable, "bench.py", "--extra", "nonsense"], cwd=ROOT, capture_output=True,
                          text=True, timeout=120)
     assert out.returncode != 0 and "unknown workload" in out.stderr
+
+
+def test_profiled_traffic_matches_sources():
+    """Each DRAM-traffic figure the bench reports comes from an ncu capture of
+    the kernel source as it stands: the recorded sha1 prefix is the source's,
+    and the profile summary it cites names that prefix."""
+    import hashlib
+    import importlib.util
+
+    spec = importlib.util.spec_from_file_location("bench_records", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    assert bench.PROFILED_TRAFFIC
+    for src, rec in bench.PROFILED_TRAFFIC.items():
+        with open(os.path.join(ROOT, "gated_delta_rule_136_b200", src), "rb") as f:
+            assert hashlib.sha1(f.read()).hexdigest()[:12] == rec["sha1"], src
+        with open(os.path.join(ROOT, rec["profile"])) as f:
+            assert rec["sha1"] in f.read(), rec["profile"]
+        assert any(k.startswith("bytes_per_") and v > 0 for k, v in rec.items()), src
