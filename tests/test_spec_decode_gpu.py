@@ -26,7 +26,7 @@ def _cpu(x):
 
 
 @pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
-@pytest.mark.parametrize("D", [1, 5])
+@pytest.mark.parametrize("D", [1, 4, 5, 8])
 def test_verify_and_commit_match_oracle(dtype, d, D):
     B, H = 3, 2
     inp, x, S = _draft(B, D, H, d, dtype, seed=31 + D)
