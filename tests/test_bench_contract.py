@@ -35,16 +35,33 @@ def test_unknown_extra_workload_is_rejected():
     assert out.returncode != 0 and "unknown workload" in out.stderr
 
 
-def test_profiled_traffic_matches_sources():
-    """Each DRAM-traffic figure the bench reports comes from an ncu capture of
-    the kernel source as it stands: the recorded sha1 prefix is the source's,
-    and the profile summary it cites names that prefix."""
-    import hashlib
+def _bench_module():
     import importlib.util
 
     spec = importlib.util.spec_from_file_location("bench_records", os.path.join(ROOT, "bench.py"))
     bench = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(bench)
+    return bench
+
+
+def test_roofline_unit_figures():
+    """The per-unit figures behind `roofline.achieved`: per token and head at
+    dk = dv = 128 in bf16, q, k, g (3 x 256 B), v (256 B), beta (2 B) read and
+    o (256 B) written; FLOPs 6 dk dv for the state products, C (3 dk + 2 dv)
+    for the intra-chunk ones at C = 64, C^2 / 3 for the inverse."""
+    bench = _bench_module()
+    assert bench.bytes_per_token_head() == 1282
+    assert bench.bytes_per_token_head(esz=4) == 2564
+    assert abs(bench.flops_per_token_head() - (98304 + 40960 + 4096 / 3)) < 1e-9
+
+
+def test_profiled_traffic_matches_sources():
+    """Each DRAM-traffic figure the bench reports comes from an ncu capture of
+    the kernel source as it stands: the recorded sha1 prefix is the source's,
+    and the profile summary it cites names that prefix."""
+    import hashlib
+
+    bench = _bench_module()
     assert bench.PROFILED_TRAFFIC
     for src, rec in bench.PROFILED_TRAFFIC.items():
         with open(os.path.join(ROOT, "gated_delta_rule_136_b200", src), "rb") as f:
